@@ -1,0 +1,434 @@
+"""Benchmark of the gated delta rule forward on B200.
+
+python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+One step = one gdr_chunk_fwd call over the whole workload (cumulative decay, WY
+construction, state propagation and output for every chunk of every sequence-
+head), inputs resident in HBM.  Workloads (synthetic, seeded; workload/):
+  gdn2_t4k   (default) B=8, H=16, T=4096, dk=dv=128, chunk 64, bf16, Gated DeltaNet-2
+  gdn_t2k    B=4, H=16, T=2048, Gated DeltaNet (scalar gates)
+  gdn2_t16k  B=1, H=16, T=16384;  gdn2_t16k_kda: the tied KDA mode on the same inputs
+  decode     256 sequences x 16 heads, one token per step, state in place
+Metric: token-heads/s (tokens/s per head-layer) = B*H*T / step time (decode:
+step-heads/s).  With N ranks every rank runs its own copy of the workload on its
+GPU (sequence-heads are independent: weak scaling, no collective on the data
+path) and value = all ranks' units / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workload  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ---------------------------------------------------------------------------------------
+# algorithmic counts (each input read once, each output written once)
+def chunk_bytes(wl: workload.Workload, mode: str) -> float:
+    e = 2 if wl.dtype == "bf16" else 4
+    dk, dv = wl.dk, wl.dv
+    per_tok = (2 * dk + dv) * e + dv * e               # q, k, v in; o out
+    if mode == "gdn2":
+        per_tok += dk * 4 + dk * e + dv * e             # g [dk] fp32, b [dk], w [dv]
+    elif mode == "kda":
+        per_tok += dk * 4 + e                           # g [dk], beta
+    else:
+        per_tok += 4 + e                                # g scalar, beta
+    per_head_state = (2 if wl.s0_std > 0 else 1) * dk * dv * 4   # S_T write (+ S0 read)
+    return wl.units * per_tok + wl.B * wl.H * per_head_state
+
+
+def chunk_flops(wl: workload.Workload) -> float:
+    """Dense products of the chunkwise form per token-head: 6 dk dv + 10 C d
+    (A, P, W, U, W S, Q S, P E, K^T E; the triangular inverse is not counted)."""
+    d = max(wl.dk, wl.dv)
+    return wl.units * (6.0 * wl.dk * wl.dv + 10.0 * wl.chunk * d)
+
+
+def decode_bytes(cfg) -> float:
+    e = 2 if cfg["dtype"] == "bf16" else 4
+    dk, dv = cfg["dk"], cfg["dv"]
+    per = 2 * dk * dv * 4 + (2 * dk + dv) * e + dk * 4 + dk * e + dv * e + dv * e
+    return cfg["N"] * cfg["H"] * per
+
+
+def load_peaks():
+    try:
+        p = json.load(open(PEAKS_FILE))
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_workload(name: str, rank: int):
+    """Each rank's own share: the named workload's shape with a rank-specific seed."""
+    if name == "decode":
+        cfg = dict(workload.DECODE)
+        cfg["seed"] = cfg["seed"] + 1000 * rank
+        return cfg, "gdn2"
+    base, mode = name, None
+    if name.endswith("_kda"):
+        base, mode = name[:-4], "kda"
+    wl = workload.CONFIGS[base]
+    if rank:
+        from dataclasses import replace
+        wl = replace(wl, seed=wl.seed + 1000 * rank)
+    return wl, mode or wl.mode
+
+
+# ---------------------------------------------------------------------------------------
+def cpu_oracle_sample(name, target_cpu_s=15.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload."""
+    import oracle
+    cores = oracle.default_threads()
+    if name == "decode":
+        cfg = workload.DECODE
+        pool = workload.make_decode_pool(cfg, N=16, pool=4)
+        S = pool["S0"]
+        n_heads = 16 * cfg["H"]
+        steps = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < target_cpu_s / cores and steps < 1000:
+            p = steps % 4
+            _, S = oracle.decode(pool["q"][p], pool["k"][p], pool["v"][p], pool["g"][p],
+                                 pool["b"][p], pool["w"][p], S=S, mode="gdn2", nthreads=cores)
+            steps += 1
+        dt = time.perf_counter() - t0
+        return dict(value=steps * n_heads / dt, unit="step-heads/s", cores=cores, kind="oracle",
+                    sample=f"{steps} decode steps of 16 sequences x {cfg['H']} heads (of 256 x {cfg['H']})")
+    wl, mode = rank_workload(name, 0)
+    T = wl.T
+    small = workload.Workload("sample", B=1, H=1, T=T, dk=wl.dk, dv=wl.dv, chunk=wl.chunk,
+                              dtype=wl.dtype, mode=wl.mode, seed=wl.seed, g_scale=wl.g_scale,
+                              s0_std=wl.s0_std)
+    d = workload.make_inputs(small, mode=mode)
+    t0 = time.perf_counter()
+    oracle.fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=mode, nthreads=1)
+    t_head = time.perf_counter() - t0
+    n_heads = max(cores, int(round(target_cpu_s / max(t_head, 1e-3) / cores)) * cores)
+    n_heads = min(n_heads, wl.B * wl.H)
+    rep = lambda x: None if x is None else x.expand(n_heads, *x.shape[1:]).contiguous()
+    dd = {k: rep(d[k]) for k in ("q", "k", "v", "g", "b", "w", "S0")}
+    t0 = time.perf_counter()
+    oracle.fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["b"], dd["w"], dd["S0"], mode=mode,
+               nthreads=cores)
+    dt = time.perf_counter() - t0
+    return dict(value=n_heads * T / dt, unit="token-heads/s", cores=min(cores, n_heads),
+                kind="oracle", sample=f"{n_heads} sequence-heads x T={T} of {name}")
+
+
+# ---------------------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    name = args.workload
+    steps_cpu = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(name, target_cpu_s=2.0)
+    for _ in range(args.steps):
+        steps_cpu.append(cpu_oracle_sample(name, target_cpu_s=args.ref_cpu_s))
+    v = statistics.median(s["value"] for s in steps_cpu)
+    unit = steps_cpu[0]["unit"]
+    line = {"impl": "reference", "metric": metric_name(name), "value": v, "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+            "config": config_of(name, world),
+            "cpu_baseline": {"value": v, "unit": unit, "cores": steps_cpu[0]["cores"],
+                             "kind": "oracle", "sample": steps_cpu[0]["sample"]},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "vs_baseline": None}
+    print(json.dumps(line), flush=True)
+
+
+def metric_name(name):
+    if name == "decode":
+        return "decode step-heads/s (256 seqs x 16 heads, dk=dv=128); % HBM roofline"
+    return "chunked fwd tokens/s per head·layer at T=4K; % tensor-pipe / HBM roofline"
+
+
+def config_of(name, world):
+    if name == "decode":
+        c = workload.DECODE
+        return {"workload": "gdn2_decode", "N": c["N"], "H": c["H"], "dk": c["dk"], "dv": c["dv"],
+                "mode": "gdn2", "state": "fp32 in place", "inputs": "bf16",
+                "l2": "state 537 MB per step > L2", "parallelism": f"replicas{world}"}
+    wl, mode = rank_workload(name, 0)
+    return {"workload": name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk, "dv": wl.dv,
+            "chunk": wl.chunk, "mode": mode, "inputs": wl.dtype, "state": "fp32",
+            "l2": "inputs larger than L2 (no flush)" if chunk_bytes(wl, mode) > 126e6
+            else "L2 flushed between steps", "parallelism": f"replicas{world}"}
+
+
+def run_ours(args, rank, world, local):
+    import linear_attention_recurrence_wy_b200 as gdr
+    gdr.lib()
+    name = args.workload
+    dev = torch.device("cuda", local)
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+    wl, mode = rank_workload(name, rank)
+    stream = torch.cuda.current_stream(dev)
+    flush = None
+
+    if name == "decode":
+        pool = workload.make_decode_pool(wl)
+        d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in pool.items()}
+        S = d["S0"].clone()
+        P = wl["pool"]
+        n_inner = wl["steps"]
+
+        def step():
+            for s in range(n_inner):
+                p = s % P
+                gdr.decode_step(d["q"][p], d["k"][p], d["v"][p], d["g"][p], d["b"][p], d["w"][p], S,
+                                mode="gdn2")
+        units = wl["N"] * wl["H"] * n_inner
+        bytes_per_launch = decode_bytes(wl)
+        launches_per_step = n_inner
+        unit = "step-heads/s"
+    else:
+        inp = workload.make_inputs(wl, mode=mode)
+        d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
+        o = torch.empty(wl.B, wl.H, wl.T, wl.dv, dtype=d["q"].dtype, device=dev)
+        ST = torch.empty(wl.B, wl.H, wl.dk, wl.dv, dtype=torch.float32, device=dev)
+        if chunk_bytes(wl, mode) <= 126e6:
+            flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+        def step():
+            if flush is not None:
+                flush.zero_()
+            gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=mode,
+                          chunk=wl.chunk, o=o, S_T=ST)
+        units = wl.units
+        bytes_per_launch = chunk_bytes(wl, mode)
+        launches_per_step = 1
+        unit = "token-heads/s"
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc = gdr.gdr_last_device_error(stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"device error after warm-up: {gdr.gdr_status_string(rc)}")
+
+    # kernel-only timing: events around each step on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            ev[i][0].record(stream)
+            if name == "decode":
+                step()
+            else:
+                gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=mode,
+                              chunk=wl.chunk, o=o, S_T=ST)
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = t_start.elapsed_time(t_end)
+    kern_ms = sum(step_ms) / len(step_ms)
+    ms_per_step = max_over_ranks(kern_ms, world)
+    value = units * world / (ms_per_step * 1e-3)
+    rc = gdr.gdr_last_device_error(stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"device error in timed region: {gdr.gdr_status_string(rc)}")
+
+    # end to end through the public API with host buffers (pinned), copies inside
+    e2e = None
+    if not args.no_e2e and name != "decode":
+        hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v))
+        outh = (torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
+                torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True))
+        d2h = sum(x.numel() * x.element_size() for x in outh)
+        n_e2e = max(1, min(args.steps, 5))
+        gdr.chunk_fwd_host(hin["q"], hin["k"], hin["v"], hin["g"], hin["b"], hin["w"], hin["S0"],
+                           mode=mode, chunk=wl.chunk, device=dev, out=outh)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            gdr.chunk_fwd_host(hin["q"], hin["k"], hin["v"], hin["g"], hin["b"], hin["w"], hin["S0"],
+                               mode=mode, chunk=wl.chunk, device=dev, out=outh)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+        e2e = {"value": units * world / (e2e_ms * 1e-3), "unit": unit,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    elif name == "decode":
+        e2e = None
+
+    if rank != 0:
+        return
+    launch_ms = kern_ms / launches_per_step
+    achieved = bytes_per_launch / (launch_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": args.traffic, "peak_source": f"{peak_src} hbm_gbs",
+            "kernel": "gdr decode_kernel" if name == "decode" else kernel_name(wl, mode)}
+    if name != "decode":
+        fl = chunk_flops(wl)
+        roof["tensor_context"] = {"flops_per_launch": fl,
+                                  "achieved_tflops": fl / (launch_ms * 1e-3) / 1e12,
+                                  "peak_tflops": tf_burst,
+                                  "frac": fl / (launch_ms * 1e-3) / 1e12 / tf_burst}
+    line = {"metric": metric_name(name), "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if (name == "decode" or wl.dtype == "bf16") else "f32",
+            "data": "synthetic", "config": config_of(name, world), "roofline": roof,
+            "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps,
+            "e2e": e2e, "wall_total_ms": total_ms}
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(name, target_cpu_s=args.ref_cpu_s)
+    print(json.dumps(line), flush=True)
+
+
+def kernel_name(wl, mode):
+    if wl.dtype == "bf16" and wl.dk == 128 and wl.dv == 128 and wl.chunk == 64:
+        return "gdr chunk_tc_kernel (tcgen05)"
+    return "gdr chunk_simt_kernel"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gdn2_t4k",
+                    choices=["gdn2_t4k", "gdn_t2k", "gdn2_t16k", "gdn2_t16k_kda", "gdn2_tiny", "decode"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-cpu-s", type=float, default=15.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel, if captured for this build")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

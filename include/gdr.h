@@ -1,0 +1,121 @@
+/*
+ * gdr.h -- C ABI of libgdr, the gated delta rule forward for NVIDIA B200 (sm_100a).
+ *
+ * The operation (Gated DeltaNet-2 Q&A page, Q3 "update equation"; Gated DeltaNet-2
+ * Review §3-1; Gated DeltaNet explainer, "Mechanism" for the read-out):
+ *
+ *     S_t = (I - k_t (b_t . k_t)^T) diag(exp(g_t)) S_{t-1} + k_t (w_t . v_t)^T
+ *     o_t = S_t^T q_t
+ *
+ * per sequence and head, with state S in R^{dk x dv} (fp32), channel-wise log-decay
+ * g_t in R^{dk} (fp32), erase gate b_t in [0,1]^{dk} and write gate w_t in [0,1]^{dv}.
+ * The tied modes are the reductions named on the same Q3: KDA (b = w = beta * 1) and
+ * Gated DeltaNet (additionally a scalar decay, S_t = alpha_t (I - beta_t k k^T)
+ * S_{t-1} + beta_t k v^T with alpha_t = exp(g_t)).
+ *
+ * Common conventions
+ *   - Every pointer is a DEVICE pointer on the current CUDA device; the caller owns
+ *     every buffer.  The library allocates no device memory and keeps no state
+ *     between calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and the call returns without synchronising.  Arguments are
+ *     validated on the host first: on any error nothing is launched.
+ *   - Layouts are row-major and contiguous:
+ *       q, k   [B, H, T, dk]          v, o   [B, H, T, dv]
+ *       g_log  [B, H, T, dk] fp32     (GDR_MODE_GDN: [B, H, T])
+ *       b      [B, H, T, dk]          (KDA, GDN: beta [B, H, T])
+ *       w      [B, H, T, dv]          (KDA, GDN: ignored, may be NULL)
+ *       S0,S_T [B, H, dk, dv] fp32
+ *   - q, k, v, b, w, o have the element type `dtype`; g_log and states are fp32.
+ *   - Every pointer must be 16-byte aligned (GDR_ERR_ALIGN otherwise).
+ *   - Supported sizes: dk, dv in {16, 32, 64, 128}; chunk in {16, 32, 64}; any
+ *     T >= 0; B, H >= 0.  Sizes are int; B*H*T*max(dk,dv) must fit in int64.
+ *   - The decay is meant to forget: g_log <= 0.  Positive values are computed as
+ *     written but can overflow fp32 over long chunks.
+ */
+#ifndef GDR_H
+#define GDR_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDR_OK = 0,
+    GDR_ERR_NULL = -1,     /* a required pointer is NULL */
+    GDR_ERR_DIM = -2,      /* unsupported size (dk, dv, chunk) or negative B, H, T, N */
+    GDR_ERR_MODE = -3,     /* unknown gdr_mode_t */
+    GDR_ERR_DTYPE = -4,    /* unknown gdr_dtype_t */
+    GDR_ERR_ALIGN = -5,    /* a pointer is not 16-byte aligned */
+    GDR_ERR_CUDA = -6,     /* a CUDA launch or attribute call failed */
+    GDR_ERR_TIMEOUT = -7   /* a bounded device-side wait gave up (tensor-core path) */
+} gdr_status_t;
+
+typedef enum {
+    GDR_MODE_GDN2 = 0,     /* Gated DeltaNet-2: g [dk], b [dk], w [dv] per token */
+    GDR_MODE_KDA = 1,      /* KDA: g [dk], beta per token in b; w ignored */
+    GDR_MODE_GDN = 2       /* Gated DeltaNet: scalar g, beta per token in b; w ignored */
+} gdr_mode_t;
+
+typedef enum {
+    GDR_F32 = 0,           /* q, k, v, b, w, o are float */
+    GDR_BF16 = 1           /* q, k, v, b, w, o are bfloat16 */
+} gdr_dtype_t;
+
+/*
+ * gdr_chunk_fwd -- chunkwise-parallel forward over whole sequences.
+ *
+ * Computes o_t for t = 0..T-1 and the final state S_T from the initial state S0 by
+ * the chunkwise WY form of the recurrence (Gated DeltaNet-2 Q&A page, Q4; Gated
+ * DeltaNet-2 Review §3-2.5): within a chunk of `chunk` tokens the cumulative
+ * channel-wise decay is absorbed into the rank-one erase factor, the token
+ * interactions become dense products, and only the state crosses chunk borders.
+ * The result equals the sequential recurrence up to rounding.
+ *
+ *   S0   NULL = zero initial state.
+ *   S_T  NULL = do not write the final state.  S_T may equal S0 (in-place update).
+ *   o    [B,H,T,dv], written for every t.  Must not overlap any input.
+ *   T == 0 writes S_T = S0 (or zeros) and nothing else.
+ *
+ * Paths: dtype == GDR_BF16 with dk == dv == 128 and chunk == 64 runs on the
+ * tcgen05 tensor cores (bf16 operands, fp32 accumulation and state); every other
+ * case runs the fp32 CUDA-core kernel.  Returns GDR_OK once the work is enqueued.
+ * A bounded wait that expired inside the tensor-core kernel of an earlier call is
+ * reported as GDR_ERR_TIMEOUT by gdr_last_device_error().
+ */
+gdr_status_t gdr_chunk_fwd(const void *q, const void *k, const void *v, const float *g_log,
+                           const void *b, const void *w, const float *S0, void *o, float *S_T,
+                           int B, int H, int T, int dk, int dv, int chunk, gdr_mode_t mode,
+                           gdr_dtype_t dtype, void *stream);
+
+/*
+ * gdr_decode_step -- one-token recurrent update for N sequences x H heads.
+ *
+ * The recurrent form used for constant-memory decoding (Gated DeltaNet-2 Q&A page,
+ * introduction; Gated DeltaNet-2 Review §3-2.1): S <- update(S) in place and
+ * o = S_new^T q.  Layout is the forward's with T = 1 and N in place of B:
+ * q, k [N,H,dk]; v, o [N,H,dv]; g_log [N,H,dk] (GDN: [N,H]); b [N,H,dk]
+ * (KDA, GDN: beta [N,H]); w [N,H,dv]; S [N,H,dk,dv] fp32, read and written.
+ * o must not overlap S or any input.  Runs on CUDA cores (bandwidth-bound).
+ */
+gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const float *g_log,
+                             const void *b, const void *w, float *S, void *o, int N, int H,
+                             int dk, int dv, gdr_mode_t mode, gdr_dtype_t dtype, void *stream);
+
+/*
+ * gdr_last_device_error -- read and clear the device-side error word.
+ *
+ * Synchronises `stream`, then returns GDR_ERR_TIMEOUT if a bounded wait inside a
+ * tensor-core kernel gave up since the last call (the kernel then skipped its
+ * remaining work and released its tensor memory), GDR_ERR_CUDA if the stream
+ * reports a CUDA error, else GDR_OK.
+ */
+gdr_status_t gdr_last_device_error(void *stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *gdr_status_string(gdr_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDR_H */

@@ -1,0 +1,167 @@
+"""Gated delta rule forward on NVIDIA B200 (sm_100a): thin Python binding of libgdr.
+
+The arithmetic runs in libgdr.so's CUDA kernels; this module only checks tensor
+shapes and dtypes, allocates outputs with PyTorch and passes raw device pointers
+and the current CUDA stream to the C ABI (include/gdr.h).  There is no CPU or
+PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raised.
+
+Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_decode_step,
+gdr_last_device_error, gdr_status_string.
+Tensor wrappers:  chunk_fwd, chunk_fwd_host, decode_step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdr.so")
+MODES = {"gdn2": 0, "kda": 1, "gdn": 2}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+_lib = None
+
+
+class GdrError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {gdr_status_string(code)} ({code})")
+
+
+def lib():
+    """Load libgdr.so (built in-tree by build.py); raises if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libgdr.so not built: run python -m linear_attention_recurrence_wy_b200.build "
+                              f"(expected at {LIB_PATH})")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci = ctypes.c_void_p, ctypes.c_int
+        L.gdr_chunk_fwd.argtypes = [vp] * 9 + [ci] * 8 + [vp]
+        L.gdr_chunk_fwd.restype = ci
+        L.gdr_decode_step.argtypes = [vp] * 8 + [ci] * 6 + [vp]
+        L.gdr_decode_step.restype = ci
+        L.gdr_last_device_error.argtypes = [vp]
+        L.gdr_last_device_error.restype = ci
+        L.gdr_status_string.argtypes = [ci]
+        L.gdr_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+# ---- raw C-ABI names -------------------------------------------------------------------
+def gdr_chunk_fwd(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype, stream):
+    return lib().gdr_chunk_fwd(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode,
+                               dtype, stream)
+
+
+def gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, stream):
+    return lib().gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, stream)
+
+
+def gdr_last_device_error(stream=None):
+    return lib().gdr_last_device_error(stream)
+
+
+def gdr_status_string(code: int) -> str:
+    return lib().gdr_status_string(int(code)).decode()
+
+
+# ---- tensor wrappers -------------------------------------------------------------------
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(t, name, shape, dtype, device):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype} != {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+
+
+def _gate_shapes(mode, lead, dk, dv):
+    if mode == "gdn2":
+        return (*lead, dk), (*lead, dk), (*lead, dv)
+    if mode == "kda":
+        return (*lead, dk), tuple(lead), None
+    return tuple(lead), tuple(lead), None
+
+
+def chunk_fwd(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, o=None, S_T=None,
+              return_state=True):
+    """Chunkwise forward.  q,k [B,H,T,dk], v [B,H,T,dv] (fp32 or bf16, CUDA), g fp32,
+    b (beta for kda/gdn), w (gdn2 only), S0 fp32 [B,H,dk,dv] or None.
+    Returns (o, S_T) with S_T None when return_state is False."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    if dt not in DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    gshape, bshape, wshape = _gate_shapes(mode, (B, H, T), dk, dv)
+    _check(q, "q", (B, H, T, dk), dt, dev)
+    _check(k, "k", (B, H, T, dk), dt, dev)
+    _check(v, "v", (B, H, T, dv), dt, dev)
+    _check(g, "g", gshape, torch.float32, dev)
+    _check(b, "b", bshape, dt, dev)
+    if mode == "gdn2":
+        _check(w, "w", wshape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=dt, device=dev)
+    if S_T is None and return_state:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    rc = gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
+                       _ptr(w) if mode == "gdn2" else None, _ptr(S0), _ptr(o), _ptr(S_T),
+                       B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd")
+    return o, S_T
+
+
+def chunk_fwd_host(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, device="cuda",
+                   out=None):
+    """End-to-end call on host tensors: copies the inputs (pinned host memory is
+    copied asynchronously) to the device, runs chunk_fwd and copies o and S_T back
+    into host tensors (`out` = (o_host, S_T_host) to reuse pinned buffers)."""
+    nb = q.is_pinned()
+    to = lambda t: None if t is None else t.to(device, non_blocking=nb)
+    o_d, S_d = chunk_fwd(to(q), to(k), to(v), to(g), to(b), to(w), to(S0), mode=mode, chunk=chunk)
+    if out is None:
+        out = (torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True),
+               torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True))
+    out[0].copy_(o_d, non_blocking=True)
+    out[1].copy_(S_d, non_blocking=True)
+    return out
+
+
+def decode_step(q, k, v, g, b, w, S, *, mode="gdn2", o=None):
+    """One-token step; S [N,H,dk,dv] fp32 is updated in place.  Returns o [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    gshape, bshape, wshape = _gate_shapes(mode, (N, H), dk, dv)
+    _check(k, "k", (N, H, dk), dt, dev)
+    _check(v, "v", (N, H, dv), dt, dev)
+    _check(g, "g", gshape, torch.float32, dev)
+    _check(b, "b", bshape, dt, dev)
+    if mode == "gdn2":
+        _check(w, "w", wshape, dt, dev)
+    _check(S, "S", (N, H, dk, dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=dt, device=dev)
+    rc = gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
+                         _ptr(w) if mode == "gdn2" else None, _ptr(S), _ptr(o),
+                         N, H, dk, dv, MODES[mode], DTYPES[dt], _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_decode_step")
+    return o

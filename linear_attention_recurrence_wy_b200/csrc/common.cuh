@@ -1,0 +1,43 @@
+// common.cuh -- shared argument block, element loads and launch helpers of libgdr.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/gdr.h"
+
+namespace gdr {
+
+// Everything a chunked-forward kernel needs; built once by the C-ABI layer.
+struct ChunkArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *g, *S0;
+    void *o;
+    float *ST;
+    int B, H, T, dk, dv, chunk, mode, dtype;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *g;
+    float *S;
+    void *o;
+    int N, H, dk, dv, mode, dtype;
+};
+
+__device__ __forceinline__ float ld_elem(const void *p, size_t i, int dtype) {
+    if (dtype == GDR_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
+    return reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ void st_elem(void *p, size_t i, int dtype, float x) {
+    if (dtype == GDR_BF16) reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+    else reinterpret_cast<float *>(p)[i] = x;
+}
+
+// Launch wrappers (one per kernel family); each returns GDR_OK or GDR_ERR_CUDA.
+gdr_status_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
+gdr_status_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+gdr_status_t launch_state_copy(const ChunkArgs &a, cudaStream_t s);
+
+}  // namespace gdr

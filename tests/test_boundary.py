@@ -1,0 +1,106 @@
+"""Host-only tests of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments with the documented status before launching anything.
+None of these calls reaches a CUDA API (validation returns first)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_recurrence_wy_b200 as gdr
+from linear_attention_recurrence_wy_b200 import build as gbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdr.h")
+
+OK, NULL, DIM, MODE, DTYPE, ALIGN = 0, -1, -2, -3, -4, -5
+
+
+@pytest.fixture(scope="module")
+def L():
+    gbuild.build()
+    return gdr.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdr_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gdr_chunk_fwd", "gdr_decode_step", "gdr_last_device_error", "gdr_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        s = gdr.gdr_status_string(code)
+        assert s.startswith("GDR_")
+    assert "unknown" in gdr.gdr_status_string(42)
+
+
+A = 4096  # a 16-byte aligned fake address: never dereferenced, validation fails first
+
+
+def call_fwd(q=A, k=A, v=A, g=A, b=A, w=A, S0=None, o=A, ST=None, B=1, H=1, T=8, dk=64, dv=64,
+             chunk=64, mode=0, dtype=0):
+    return gdr.gdr_chunk_fwd(q, k, v, g, b, w, S0, o, ST, B, H, T, dk, dv, chunk, mode, dtype, None)
+
+
+def call_dec(q=A, k=A, v=A, g=A, b=A, w=A, S=A, o=A, N=1, H=1, dk=64, dv=64, mode=0, dtype=0):
+    return gdr.gdr_decode_step(q, k, v, g, b, w, S, o, N, H, dk, dv, mode, dtype, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=3), MODE), (dict(mode=-1), MODE), (dict(dtype=2), DTYPE),
+    (dict(dk=48), DIM), (dict(dv=256), DIM), (dict(chunk=128), DIM), (dict(chunk=8), DIM),
+    (dict(B=-1), DIM), (dict(T=-1), DIM), (dict(H=-2), DIM),
+    (dict(q=None), NULL), (dict(k=None), NULL), (dict(v=None), NULL), (dict(g=None), NULL),
+    (dict(b=None), NULL), (dict(o=None), NULL), (dict(w=None), NULL),
+    (dict(q=A + 4), ALIGN), (dict(o=A + 2), ALIGN), (dict(S0=A + 8), ALIGN), (dict(ST=A + 12), ALIGN),
+    (dict(w=A + 8), ALIGN),
+])
+def test_chunk_fwd_rejects(L, kw, code):
+    assert call_fwd(**kw) == code
+
+
+def test_chunk_fwd_tied_modes_do_not_need_w(L):
+    # w is ignored in KDA/GDN modes; with B = 0 nothing is launched
+    assert call_fwd(w=None, mode=1, B=0) == OK
+    assert call_fwd(w=None, mode=2, B=0) == OK
+    assert call_fwd(w=None, mode=0, B=1) == NULL
+
+
+def test_chunk_fwd_empty_batch_is_a_no_op(L):
+    assert call_fwd(q=None, k=None, v=None, g=None, b=None, w=None, o=None, B=0) == OK
+    assert call_fwd(q=None, k=None, v=None, g=None, b=None, w=None, o=None, H=0) == OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=5), MODE), (dict(dtype=-1), DTYPE), (dict(dk=100), DIM), (dict(N=-1), DIM),
+    (dict(S=None), NULL), (dict(o=None), NULL), (dict(w=None), NULL), (dict(g=None), NULL),
+    (dict(S=A + 4), ALIGN), (dict(q=A + 2), ALIGN),
+])
+def test_decode_rejects(L, kw, code):
+    assert call_dec(**kw) == code
+
+
+def test_decode_empty_is_a_no_op(L):
+    assert call_dec(N=0, S=None, q=None) == OK
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.dirname(gdr.__file__)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                for bad in ("import oracle", "from oracle", "gdr_oracle", "libgdr_oracle"):
+                    assert bad not in txt, (f, bad)

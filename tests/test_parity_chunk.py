@@ -1,0 +1,137 @@
+"""GPU parity of gdr_chunk_fwd (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workload
+from util import assert_close, gpu_fwd, np64, to_dev
+
+gdr = pytest.importorskip("linear_attention_recurrence_wy_b200")
+pytestmark = pytest.mark.gpu
+
+
+def oracle_full(d):
+    return oracle.fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=d["mode"])
+
+
+def check_case(d_cpu, chunk, dtype):
+    d = to_dev(d_cpu)
+    o, ST = gpu_fwd(gdr, d, chunk=chunk)
+    torch.cuda.synchronize()
+    o_ref, S_ref = oracle_full(d_cpu)
+    e1 = assert_close("o", np64(o), o_ref, dtype)
+    e2 = assert_close("S_T", np64(ST), S_ref, dtype)
+    return e1, e2
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 200])
+def test_small_shapes_modes(cuda_ok, dtype, mode, T):
+    d = workload.make_small(2, 3, T, 64, 64, mode=mode, dtype=dtype, seed=T, g_scale=0.5,
+                            s0_std=0.1)
+    check_case(d, 64, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 64), (64, 32), (128, 128), (16, 128), (128, 16)])
+def test_dims_and_chunks(cuda_ok, dtype, chunk, dk, dv):
+    d = workload.make_small(1, 2, 150, dk, dv, mode="gdn2", dtype=dtype, seed=dk + dv + chunk,
+                            g_scale=0.3, s0_std=0.05)
+    check_case(d, chunk, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["gdn2", "gdn"])
+def test_without_initial_state(cuda_ok, dtype, mode):
+    d = workload.make_small(2, 2, 130, 128, 128, mode=mode, dtype=dtype, seed=7, s0_std=0.0)
+    assert d["S0"] is None
+    check_case(d, 64, dtype)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("g_const", [-20.0, -3.0, 0.0])
+def test_extreme_and_zero_decay(cuda_ok, dtype, g_const):
+    d = workload.make_small(1, 2, 160, 128, 128, mode="gdn2", dtype=dtype, seed=3, s0_std=0.1,
+                            g_const=g_const)
+    check_case(d, 64, dtype)
+
+
+def test_mixed_extreme_decay_channels(cuda_ok):
+    # half the channels forget almost everything per token, half barely decay
+    d = workload.make_small(2, 2, 192, 128, 128, mode="gdn2", dtype="bf16", seed=4, s0_std=0.1)
+    g = d["g"].clone()
+    g[..., ::2] = -25.0
+    g[..., 1::2] = -1e-3
+    d["g"] = g
+    check_case(d, 64, "bf16")
+
+
+def test_empty_sequence_copies_state(cuda_ok):
+    d = to_dev(workload.make_small(2, 2, 0, 64, 64, s0_std=0.2))
+    o, ST = gpu_fwd(gdr, d)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 2, 0, 64)
+    assert torch.equal(ST, d["S0"])
+
+
+def test_in_place_state_and_split_sequence(cuda_ok):
+    d_cpu = workload.make_small(2, 2, 200, 128, 128, mode="gdn2", dtype="f32", seed=9, s0_std=0.1)
+    d = to_dev(d_cpu)
+    o_full, S_full = gpu_fwd(gdr, d)
+    cut = 77   # not a multiple of the chunk
+    part = lambda x, s: None if x is None else x[:, :, s].contiguous()
+    S = d["S0"].clone()
+    outs = []
+    for sl in (slice(0, cut), slice(cut, None)):
+        dd = {k: part(d[k], sl) for k in ("q", "k", "v", "g", "b", "w")}
+        o, _ = gdr.chunk_fwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["b"], dd["w"], S,
+                             mode="gdn2", S_T=S)       # S_T aliases S0: in-place update
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert_close("o split", np64(torch.cat(outs, 2)), np64(o_full), "f32")
+    assert_close("S split", np64(S), np64(S_full), "f32")
+
+
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+def test_decode_steps_equal_chunk_forward(cuda_ok, mode):
+    d_cpu = workload.make_small(2, 2, 40, 64, 64, mode=mode, dtype="f32", seed=11, s0_std=0.1)
+    d = to_dev(d_cpu)
+    o_full, S_full = gpu_fwd(gdr, d, chunk=16)
+    S = d["S0"].clone()
+    step = lambda x, t: None if x is None else x[:, :, t].contiguous()
+    for t in range(40):
+        o_t = gdr.decode_step(*(step(d[k], t) for k in ("q", "k", "v", "g", "b", "w")), S, mode=mode)
+        assert_close(f"o[{t}]", np64(o_t), np64(o_full[:, :, t]), "f32")
+    torch.cuda.synchronize()
+    assert_close("S", np64(S), np64(S_full), "f32")
+
+
+# ---- the measured workloads, at full size; sampled sequence-heads vs the oracle ----------
+SAMPLE = {"gdn_t2k": 8, "gdn2_t4k": 8, "gdn2_t16k": 3}
+
+
+@pytest.mark.parametrize("name,mode", [("gdn2_tiny", "gdn2"), ("gdn_t2k", "gdn"),
+                                       ("gdn2_t4k", "gdn2"), ("gdn2_t16k", "gdn2"),
+                                       ("gdn2_t16k", "kda")])
+def test_workloads_full_size(cuda_ok, name, mode):
+    wl = workload.CONFIGS[name]
+    d_cpu = workload.make_inputs(wl, mode=mode)
+    d = to_dev(d_cpu)
+    o, ST = gpu_fwd(gdr, d, chunk=wl.chunk)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(ST).all()
+    n = SAMPLE.get(name)
+    if n is None:
+        heads = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    else:
+        rng = np.random.default_rng(123)
+        flat = rng.choice(wl.B * wl.H, size=n, replace=False)
+        heads = [(int(i) // wl.H, int(i) % wl.H) for i in flat]
+    o_ref, S_ref = oracle.fwd_heads(d_cpu, heads)
+    o_s = np.stack([np64(o[b, h]) for b, h in heads])
+    S_s = np.stack([np64(ST[b, h]) for b, h in heads])
+    assert_close(f"{name} o", o_s, o_ref, wl.dtype)
+    assert_close(f"{name} S_T", S_s, S_ref, wl.dtype)
