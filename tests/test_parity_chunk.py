@@ -59,6 +59,15 @@ def test_extreme_and_zero_decay(cuda_ok, dtype, g_const):
     check_case(d, 64, dtype)
 
 
+@pytest.mark.parametrize("g_scale", [1.0, 1.3])
+def test_decay_near_fast_path_limit(cuda_ok, g_scale):
+    # cumulative chunk decays of about 50-70 nats: some chunks on either side of the
+    # tensor-core kernel's factorisation limit
+    d = workload.make_small(2, 4, 256, 128, 128, mode="gdn2", dtype="bf16", seed=5,
+                            g_scale=g_scale, s0_std=0.05)
+    check_case(d, 64, "bf16")
+
+
 def test_mixed_extreme_decay_channels(cuda_ok):
     # half the channels forget almost everything per token, half barely decay
     d = workload.make_small(2, 2, 192, 128, 128, mode="gdn2", dtype="bf16", seed=4, s0_std=0.1)
