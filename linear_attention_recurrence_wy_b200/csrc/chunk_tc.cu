@@ -41,7 +41,7 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64, DK = 128, DV = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kFastLimit = 60.f;
 constexpr int kAS = tri::LD;   // fp32 row stride of the A / T scratch
@@ -65,10 +65,11 @@ constexpr int OFF_WV = OFF_KB + 16384;          // WV    bf16 [64 t][128 v] 16 K
 constexpr int OFF_P = OFF_WV + 16384;           // P     bf16 [64 t][64 j]   8 KB
 constexpr int OFF_T = OFF_P + 8192;             // T     bf16 [64 t][64 j]   8 KB
 constexpr int OFF_WT = OFF_T + 8192;            // W^T   bf16 [128 d][64 t] 16 KB
-constexpr int OFF_SCAN = OFF_WT + 16384;        // scan totals fp32 [16][128] 8 KB
-constexpr int OFF_GC = OFF_SCAN + 8192;         // gamma_C fp32 [128]
-constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [128]
-constexpr int OFF_BAR = OFF_EGC + 512;          // 2 mbarriers + TMEM slot
+constexpr int OFF_TOT = OFF_WT + 16384;         // scan: quarter totals fp32 [4][128]
+constexpr int OFF_GS = OFF_TOT + 2048;          // scalar g_log of the chunk (GDN) fp32 [64]
+constexpr int OFF_GC = OFF_GS + 256;            // gamma_C fp32 [128]
+constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [2][128], by chunk parity
+constexpr int OFF_BAR = OFF_EGC + 1024;         // 2 mbarriers + TMEM slot
 constexpr int SMEM_BYTES = OFF_BAR + 64 + 1024; // + alignment slack
 
 // TMEM columns
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;   // TMEM lanes this warp may access: 32 * quarter + [0, 32)
     const int bh = blockIdx.x;
     const int T = a.T, mode = a.mode;
     const size_t tok0 = (size_t)bh * T;
@@ -135,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     float *sT32 = reinterpret_cast<float *>(sm + OFF_T32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
     float *sGam = reinterpret_cast<float *>(sm + RAW_G);
-    float *sScan = reinterpret_cast<float *>(sm + OFF_SCAN);
+    float *sTot = reinterpret_cast<float *>(sm + OFF_TOT);
+    float *sGs = reinterpret_cast<float *>(sm + OFF_GS);
     float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
     float *sEGC = reinterpret_cast<float *>(sm + OFF_EGC);
     const uint32_t bar_mma = sbase + OFF_BAR, bar_raw = sbase + OFF_BAR + 8;
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
     // raw inputs of chunk c -> staging (one bulk copy per tensor), thread 0 only
     auto issue_raw = [&](int c) {
@@ -199,10 +202,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     }
     int raw_issued = 1, raw_done = 0;   // uniform across the block
 
-    // ---- initial state -> TMEM: fp32 S^T and its bf16 operand copy ----
-    if (warp >= 4) {
-        const int v = (warp - 4) * 32 + lane;
-        for (int d0 = 0; d0 < DK; d0 += 32) {
+    // ---- initial state -> TMEM: fp32 S^T and its bf16 operand copy (warps 8-15) ----
+    if (warp >= 8) {
+        const int v = quarter * 32 + lane, dlo = ((warp - 8) >> 2) * 64;
+        for (int d0 = dlo; d0 < dlo + 64; d0 += 32) {
             float x[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -216,129 +219,149 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     __syncthreads();
     tc_fence_after();
 
+    // Output rows and state update of the previous chunk (warps 8-15).  Runs while
+    // warps 0-7 build the next chunk's operands: that chunk's first MMA is the first
+    // reader of what is written here.
+    auto finish_chunk = [&](int t0p, int np, bool exactp, const float *egc, bool last) {
+        if (warp < 12) {
+            const int v = quarter * 32 + lane;
+            for (int t0c = 0; t0c < 64; t0c += 16) {
+                float x[16];
+                tmem_ld16(tmem + lane_base + TM_O + t0c, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (t0c + j < np) O[(tok0 + t0p + t0c + j) * DV + v] = __float2bfloat16_rn(x[j]);
+            }
+        } else {
+            const int v = quarter * 32 + lane;
+            for (int d0 = 0; d0 < DK; d0 += 16) {
+                float x[16];
+                tmem_ld16(tmem + lane_base + TM_S + d0, x);
+                tmem_wait_ld();
+                if (!exactp) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) x[j] *= egc[d0 + j];
+                    tmem_st16(tmem + lane_base + TM_S + d0, reinterpret_cast<const uint32_t(&)[16]>(x));
+                }
+                uint32_t pk[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+                tmem_st8(tmem + lane_base + TM_SB + d0 / 2, pk);
+                if (last && a.ST) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) a.ST[((size_t)bh * DK + d0 + j) * DV + v] = x[j];
+                }
+            }
+            tmem_wait_st();
+        }
+    };
+
     Waiter Wm{bar_mma, 0u}, Wr{bar_raw, 0u};
-    bool ok = true;
-    const int tg = tid >> 4, cg = tid & 15;   // build mapping: 4 tokens x 8 channels
+    bool ok = true, exact_prev = false;
+    int t0_prev = 0, n_prev = 0;
 
     for (int c = 0; c < nchunks; ++c) {
         const int t0 = c * C, n = min(C, T - t0);
-        // ===== P1: operands from the staged raw inputs =====
+        float *egc = sEGC + (c & 1) * 128;
+        // ===== P1: cumulative log-decay, then operands =====
         if (!Wr.all()) { ok = false; break; }
         raw_done = c + 1;
         if (tid == 0 && c + 2 < nchunks) prefetch_inputs(c + 2);
-        float gam[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = tg * 4 + i;
-            if (vec_g) {
-                const float *gr = sGam + t * DK + cg * 8;
-                const float4 g0 = *reinterpret_cast<const float4 *>(gr);
-                const float4 g1 = *reinterpret_cast<const float4 *>(gr + 4);
-                const bool in = t < n;
-                gam[i][0] = in ? g0.x : 0.f; gam[i][1] = in ? g0.y : 0.f;
-                gam[i][2] = in ? g0.z : 0.f; gam[i][3] = in ? g0.w : 0.f;
-                gam[i][4] = in ? g1.x : 0.f; gam[i][5] = in ? g1.y : 0.f;
-                gam[i][6] = in ? g1.z : 0.f; gam[i][7] = in ? g1.w : 0.f;
-            } else {
-                const float gs = (t < n) ? a.g[tok0 + t0 + t] : 0.f;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) gam[i][j] = gs;
-            }
+        if (!vec_g) {
+            if (tid < 64) sGs[tid] = (tid < n) ? a.g[tok0 + t0 + tid] : 0.f;
+            __syncthreads();
         }
-        // inclusive cumulative sum over the chunk: within 4 tokens, then across groups
-#pragma unroll
-        for (int i = 1; i < 4; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) gam[i][j] += gam[i - 1][j];
+        // gamma: each thread scans 16 tokens of one key channel, then adds the totals of
+        // the earlier quarters of the chunk.  Tokens past the end contribute zero.
+        const int sd = tid & 127, sq = tid >> 7;
         {
-            float4 *dst = reinterpret_cast<float4 *>(sScan + tg * 128 + cg * 8);
-            dst[0] = make_float4(gam[3][0], gam[3][1], gam[3][2], gam[3][3]);
-            dst[1] = make_float4(gam[3][4], gam[3][5], gam[3][6], gam[3][7]);
+            float acc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int t = sq * 16 + i;
+                const float g = (t < n) ? (vec_g ? sGam[t * DK + sd] : sGs[t]) : 0.f;
+                acc += g;
+                sGam[t * DK + sd] = acc;
+            }
+            sTot[sq * 128 + sd] = acc;
         }
         __syncthreads();
-        {
-            float off[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int u = 0; u < 15; ++u) {
-                const float4 x0 = *reinterpret_cast<const float4 *>(sScan + u * 128 + cg * 8);
-                const float4 x1 = *reinterpret_cast<const float4 *>(sScan + u * 128 + cg * 8 + 4);
-                const float m = (u < tg) ? 1.f : 0.f;
-                off[0] = fmaf(m, x0.x, off[0]); off[1] = fmaf(m, x0.y, off[1]);
-                off[2] = fmaf(m, x0.z, off[2]); off[3] = fmaf(m, x0.w, off[3]);
-                off[4] = fmaf(m, x1.x, off[4]); off[5] = fmaf(m, x1.y, off[5]);
-                off[6] = fmaf(m, x1.z, off[6]); off[7] = fmaf(m, x1.w, off[7]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) gam[i][j] += off[j];
-        }
-        if (tg == 15) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                sGC[cg * 8 + j] = gam[3][j];
-                sEGC[cg * 8 + j] = __expf(gam[3][j]);
-            }
-        }
         bool big = false;
+        {
+            float off = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+            for (int u = 0; u < 3; ++u)
+                if (u < sq) off += sTot[u * 128 + sd];
+            float gm = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) big |= fabsf(gam[i][j]) > kFastLimit;
-        const bool exact = __syncthreads_or(big);   // also publishes sGC / sEGC
-        if (exact) {
-            // gamma replaces this thread's own g_log elements: the per-pair decays need it
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float4 *dst = reinterpret_cast<float4 *>(sGam + (tg * 4 + i) * DK + cg * 8);
-                dst[0] = make_float4(gam[i][0], gam[i][1], gam[i][2], gam[i][3]);
-                dst[1] = make_float4(gam[i][4], gam[i][5], gam[i][6], gam[i][7]);
+            for (int i = 0; i < 16; ++i) {
+                const int t = sq * 16 + i;
+                gm = sGam[t * DK + sd] + off;
+                sGam[t * DK + sd] = gm;
+                big |= fabsf(gm) > kFastLimit;
+            }
+            if (sq == 3) {
+                sGC[sd] = gm;
+                egc[sd] = __expf(gm);
             }
         }
+        const bool exact = __syncthreads_or(big);   // also publishes gamma, gamma_C
+
+        if (warp < 8) {
+            // operands: thread (tg, cg) owns tokens 4 tg .. 4 tg + 3, channels 8 cg .. 8 cg + 7
+            const int tg = tid >> 4, cg = tid & 15;
+#pragma unroll 1
+            for (int i = 0; i < 4; ++i) {
+                const int t = tg * 4 + i;
+                const bool in = t < n;
+                const uint32_t ro = (uint32_t)(t * DK * 2 + cg * 16);
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                const uint4 uq = in ? *reinterpret_cast<const uint4 *>(sm + RAW_Q + ro) : z;
+                const uint4 uk = in ? *reinterpret_cast<const uint4 *>(sm + RAW_K + ro) : z;
+                const uint4 uv = in ? *reinterpret_cast<const uint4 *>(sm + RAW_V + ro) : z;
+                const float4 g0 = *reinterpret_cast<const float4 *>(sGam + t * DK + cg * 8);
+                const float4 g1 = *reinterpret_cast<const float4 *>(sGam + t * DK + cg * 8 + 4);
+                const float gam[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                float fq[8], fk[8], fv[8], fb[8], fw[8];
+                bf16x8_to_f32(uq, fq);
+                bf16x8_to_f32(uk, fk);
+                bf16x8_to_f32(uv, fv);
+                if (gdn2) {
+                    const uint4 ub = in ? *reinterpret_cast<const uint4 *>(sm + RAW_B + ro) : z;
+                    const uint4 uw = in ? *reinterpret_cast<const uint4 *>(sm + RAW_W + ro) : z;
+                    bf16x8_to_f32(ub, fb);
+                    bf16x8_to_f32(uw, fw);
+                } else {
+                    const float beta = in ? __bfloat162float(Bg[tok0 + t0 + t]) : 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = tg * 4 + i;
-            const bool in = t < n;
-            const uint32_t ro = (uint32_t)(t * DK * 2 + cg * 16);
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            const uint4 uq = in ? *reinterpret_cast<const uint4 *>(sm + RAW_Q + ro) : z;
-            const uint4 uk = in ? *reinterpret_cast<const uint4 *>(sm + RAW_K + ro) : z;
-            const uint4 uv = in ? *reinterpret_cast<const uint4 *>(sm + RAW_V + ro) : z;
-            float fq[8], fk[8], fv[8], fb[8], fw[8];
-            bf16x8_to_f32(uq, fq);
-            bf16x8_to_f32(uk, fk);
-            bf16x8_to_f32(uv, fv);
-            if (gdn2) {
-                const uint4 ub = in ? *reinterpret_cast<const uint4 *>(sm + RAW_B + ro) : z;
-                const uint4 uw = in ? *reinterpret_cast<const uint4 *>(sm + RAW_W + ro) : z;
-                bf16x8_to_f32(ub, fb);
-                bf16x8_to_f32(uw, fw);
-            } else {
-                const float beta = in ? __bfloat162float(Bg[tok0 + t0 + t]) : 0.f;
+                    for (int j = 0; j < 8; ++j) fb[j] = fw[j] = beta;
+                }
+                float kh[8], qg[8], kb[8], wv[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) fb[j] = fw[j] = beta;
+                for (int j = 0; j < 8; ++j) {
+                    const float e = __expf(gam[j]);
+                    kh[j] = fb[j] * fk[j] * e;
+                    qg[j] = fq[j] * e;
+                    wv[j] = fw[j] * fv[j];
+                }
+                if (exact) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(sGC[cg * 8 + j] - gam[j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(-gam[j]);
+                }
+                st_chunk(sbase + OFF_QK + tile_chunk(128, t, cg), kh);
+                st_chunk(sbase + OFF_QK + tile_chunk(128, 64 + t, cg), qg);
+                st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
+                st_chunk(sbase + OFF_WV + tile_chunk(64, t, cg), wv);
             }
-            float kh[8], qg[8], kb[8], wv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float e = __expf(gam[i][j]);
-                kh[j] = fb[j] * fk[j] * e;
-                qg[j] = fq[j] * e;
-                wv[j] = fw[j] * fv[j];
-            }
-            if (exact) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(sGC[cg * 8 + j] - gam[i][j]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(-gam[i][j]);
-            }
-            st_chunk(sbase + OFF_QK + tile_chunk(128, t, cg), kh);
-            st_chunk(sbase + OFF_QK + tile_chunk(128, 64 + t, cg), qg);
-            st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
-            st_chunk(sbase + OFF_WV + tile_chunk(64, t, cg), wv);
+        } else if (c > 0) {
+            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((c - 1) & 1) * 128, false);
         }
         fence_async_smem();
+        tc_fence_before();
         __syncthreads();
 
         // ===== P2: [A;P] = [Kh;Qg] Kb^T  and  O^T = S^T Qg^T =====
@@ -361,38 +384,34 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
 
         // ===== P3: A (fp32, strictly lower) and P (bf16, lower incl.) =====
         if (!exact) {
-            if (warp < 4) {
-                const int r = warp * 32 + lane;          // TMEM lane = row of [A; P]
-                for (int j0 = 0; j0 < 64; j0 += 32) {
-                    float x[32];
-                    tmem_ld32(tmem + lane_base + TM_AP + j0, x);
-                    tmem_wait_ld();
-                    if (r < 64) {
-                        float4 *dst = reinterpret_cast<float4 *>(sA32 + r * kAS + j0);
+            const int r = quarter * 32 + lane, j0 = (warp >> 2) * 16;   // row of [A; P], columns
+            float x[16];
+            tmem_ld16(tmem + lane_base + TM_AP + j0, x);
+            tmem_wait_ld();
+            if (r < 64) {
+                float4 *dst = reinterpret_cast<float4 *>(sA32 + r * kAS + j0);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float y[4];
+                for (int q = 0; q < 4; ++q) {
+                    float y[4];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
-                            dst[q] = make_float4(y[0], y[1], y[2], y[3]);
-                        }
-                    } else {
-                        const int t = r - 64;
+                    for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
+                    dst[q] = make_float4(y[0], y[1], y[2], y[3]);
+                }
+            } else {
+                const int t = r - 64;
 #pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8) {
-                            float f[8];
+                for (int h = 0; h < 2; ++h) {
+                    float f[8];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) f[j] = (j0 + q8 * 8 + j <= t) ? x[q8 * 8 + j] : 0.f;
-                            st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + q8), f);
-                        }
-                    }
+                    for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
+                    st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
                 }
             }
         } else {
             // exact per-pair decays (strong-decay chunks only), from the staged raw inputs
-            float av[16], pv[16];
+            float av[8], pv[8];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int p = tid + u * kThreads, i = p >> 6, j = p & 63;
                 float sa = 0.f, sp = 0.f;
                 if (j <= i && i < n) {
@@ -414,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             }
             __syncthreads();   // raw b is read above and overlaps the A scratch
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int p = tid + u * kThreads, i = p >> 6, j = p & 63;
                 sA32[i * kAS + j] = av[u];
                 *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_P + tile_off(64, i, j)) = __float2bfloat16_rn(pv[u]);
@@ -427,18 +446,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         __syncthreads();
         {
             // T (unit lower triangular) -> bf16 operand, zeros above the diagonal
-            const int t = tid >> 2, q = tid & 3;
+            const int t = tid >> 3, c8 = tid & 7;
+            float f[8];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int c8 = q * 2 + h;
-                float f[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int col = c8 * 8 + j;
-                    f[j] = (col <= t) ? sT32[t * kAS + col] : 0.f;
-                }
-                st_chunk(sbase + OFF_T + tile_chunk(64, t, c8), f);
+            for (int j = 0; j < 8; ++j) {
+                const int col = c8 * 8 + j;
+                f[j] = (col <= t) ? sT32[t * kAS + col] : 0.f;
             }
+            st_chunk(sbase + OFF_T + tile_chunk(64, t, c8), f);
         }
         fence_async_smem();
         __syncthreads();
@@ -464,27 +479,26 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         if (!Wm.all()) { ok = false; break; }
 
         // ===== P6: W^T -> bf16 operand (MN-major B); exact chunks pre-scale the state =====
-        if (warp < 4) {
-            const int d = warp * 32 + lane;
-            for (int t0c = 0; t0c < 64; t0c += 32) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_W + t0c, x);
-                tmem_wait_ld();
+        if (warp < 8) {
+            const int d = quarter * 32 + lane, t0c = (warp >> 2) * 32;
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_W + t0c, x);
+            tmem_wait_ld();
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    float f[8];
+            for (int q8 = 0; q8 < 4; ++q8) {
+                float f[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = x[q8 * 8 + j];
-                    st_chunk(sbase + OFF_WT + tile_chunk(128, d, t0c / 8 + q8), f);
-                }
+                for (int j = 0; j < 8; ++j) f[j] = x[q8 * 8 + j];
+                st_chunk(sbase + OFF_WT + tile_chunk(128, d, t0c / 8 + q8), f);
             }
         } else if (exact) {
-            for (int d0 = 0; d0 < DK; d0 += 32) {
+            const int dlo = ((warp - 8) >> 2) * 64;
+            for (int d0 = dlo; d0 < dlo + 64; d0 += 32) {
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_S + d0, x);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] *= sEGC[d0 + j];
+                for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
                 tmem_st32(tmem + lane_base + TM_S + d0, x);
             }
             tmem_wait_st();
@@ -506,13 +520,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         if (!Wm.all()) { ok = false; break; }
 
         // ===== P8: E^T -> bf16 operand in TMEM =====
-        if (warp < 4) {
-            for (int t0c = 0; t0c < 64; t0c += 32) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_E + t0c, x);
-                tmem_wait_ld();
-                st_tmem_bf16(tmem + lane_base + TM_EB + t0c / 2, x);
-            }
+        {
+            const int t0c = (warp >> 2) * 16;
+            float x[16];
+            tmem_ld16(tmem + lane_base + TM_E + t0c, x);
+            tmem_wait_ld();
+            uint32_t pk[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+            tmem_st8(tmem + lane_base + TM_EB + t0c / 2, pk);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -533,43 +549,18 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             mma_commit(bar_mma);
         }
         if (!Wm.all()) { ok = false; break; }
-
-        // ===== P10: output rows; state scaled, kept in fp32 and as the bf16 operand =====
-        if (warp < 4) {
-            const int v = warp * 32 + lane;
-            for (int t0c = 0; t0c < 64; t0c += 32) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_O + t0c, x);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (t0c + j < n) O[(tok0 + t0 + t0c + j) * DV + v] = __float2bfloat16_rn(x[j]);
-            }
-        } else {
-            const int v = (warp - 4) * 32 + lane;
-            const bool last = (c == nchunks - 1);
-            for (int d0 = 0; d0 < DK; d0 += 32) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_S + d0, x);
-                tmem_wait_ld();
-                if (!exact) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) x[j] *= sEGC[d0 + j];
-                    tmem_st32(tmem + lane_base + TM_S + d0, x);
-                }
-                st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
-                if (last && a.ST) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) a.ST[((size_t)bh * DK + d0 + j) * DV + v] = x[j];
-                }
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        exact_prev = exact;
+        t0_prev = t0;
+        n_prev = n;
     }
 
+    if (ok && nchunks > 0) {
+        // ===== P10 of the last chunk: output rows, final state =====
+        if (warp >= 8)
+            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((nchunks - 1) & 1) * 128, true);
+        tc_fence_before();
+        __syncthreads();
+    }
     if (!ok) {
         if (tid == 0) atomicExch(&g_tc_error, 1);
         // drain: committed tensor-core work and an outstanding raw copy (bounded waits)
