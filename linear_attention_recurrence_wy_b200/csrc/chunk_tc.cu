@@ -24,6 +24,9 @@
 // Data movement: each chunk's raw inputs arrive by bulk copies (one per tensor) into a
 // staging area, issued one chunk ahead and backed by L2 prefetches two chunks ahead.
 // The bf16 copies of S^T and E^T that feed the MMAs as A operands stay in TMEM.
+// Schedule (16 warps): all warps build the operands; warps 0-3 invert while warps 8-15
+// write the previous chunk's output rows and scale its state, whose first reader is this
+// chunk's S^T Qg^T MMA, issued together with W^T and U^T.
 //
 // Every wait on an mbarrier is bounded; on expiry the kernel records the failure in
 // g_tc_error, stops issuing work, waits (bounded) for its own bulk copies and
@@ -104,6 +107,18 @@ __device__ __forceinline__ void st_tmem_bf16(uint32_t taddr, const float (&x)[32
     for (int j = 0; j < 16; ++j) r[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
     tmem_st16(taddr, r);
 }
+
+// Final values of T (from the inverse) straight into the bf16 operand tile.
+struct TileOut {
+    uint32_t tile;   // shared address of the T tile ([64 t][64 j], 128-byte swizzled)
+    __device__ __forceinline__ void chunk(int row, int c8, const float (&v)[8]) {
+        st_chunk(tile + tile_chunk(64, row, c8), v);
+    }
+    __device__ __forceinline__ void pair(int row, int col, float v0, float v1) {
+        const uint32_t x = pack_bf16(v0, v1);
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(tile + tile_off(64, row, col)), "r"(x) : "memory");
+    }
+};
 
 // barrier over warps 0-3 (named barrier 1)
 struct Bar128 {
@@ -202,6 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     }
     int raw_issued = 1, raw_done = 0;   // uniform across the block
 
+    // the T tile's blocks above the diagonal are never written: zero the tile once
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid] = make_uint4(0, 0, 0, 0);
+    static_assert(kThreads * 16 == 8192, "one 16-byte store per thread clears the T tile");
     // ---- initial state -> TMEM: fp32 S^T and its bf16 operand copy (warps 8-15) ----
     if (warp >= 8) {
         const int v = quarter * 32 + lane, dlo = ((warp - 8) >> 2) * 64;
@@ -308,12 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         }
         const bool exact = __syncthreads_or(big);   // also publishes gamma, gamma_C
 
-        if (warp < 8) {
-            // operands: thread (tg, cg) owns tokens 4 tg .. 4 tg + 3, channels 8 cg .. 8 cg + 7
+        {
+            // operands: thread (tg, cg) owns tokens 2 tg, 2 tg + 1, channels 8 cg .. 8 cg + 7
             const int tg = tid >> 4, cg = tid & 15;
 #pragma unroll 1
-            for (int i = 0; i < 4; ++i) {
-                const int t = tg * 4 + i;
+            for (int i = 0; i < 2; ++i) {
+                const int t = tg * 2 + i;
                 const bool in = t < n;
                 const uint32_t ro = (uint32_t)(t * DK * 2 + cg * 16);
                 const uint4 z = make_uint4(0, 0, 0, 0);
@@ -357,30 +375,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
                 st_chunk(sbase + OFF_WV + tile_chunk(64, t, cg), wv);
             }
-        } else if (c > 0) {
-            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((c - 1) & 1) * 128, false);
         }
         fence_async_smem();
-        tc_fence_before();
         __syncthreads();
 
-        // ===== P2: [A;P] = [Kh;Qg] Kb^T  and  O^T = S^T Qg^T =====
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, false, false);
-            if (!exact) {
+        // ===== P2: [A;P] = [Kh;Qg] Kb^T =====
+        if (!exact) {
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, false, false);
 #pragma unroll
                 for (int s = 0; s < DK / 16; ++s)
                     mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s),
                              desc_kmajor(sbase + OFF_KB, 64, 0, s), id, s > 0);
+                mma_commit(bar_mma);
             }
-#pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                mma_bf16_ts(tmem + TM_O, tmem + TM_SB + s * 8, desc_kmajor(sbase + OFF_QK, 128, 64, s),
-                            id, s > 0);
-            mma_commit(bar_mma);
+            if (!Wm.all()) { ok = false; break; }
         }
-        if (!Wm.all()) { ok = false; break; }
 
         // ===== P3: A (fp32, strictly lower) and P (bf16, lower incl.) =====
         if (!exact) {
@@ -441,21 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         }
         __syncthreads();
 
-        // ===== P4: T = (I + A)^-1 =====
-        if (warp < 4) tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{});
-        __syncthreads();
-        {
-            // T (unit lower triangular) -> bf16 operand, zeros above the diagonal
-            const int t = tid >> 3, c8 = tid & 7;
-            float f[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int col = c8 * 8 + j;
-                f[j] = (col <= t) ? sT32[t * kAS + col] : 0.f;
-            }
-            st_chunk(sbase + OFF_T + tile_chunk(64, t, c8), f);
+        // ===== P4: T = (I + A)^-1 (warps 0-3) | previous chunk's outputs and state (8-15) =====
+        if (warp < 4) {
+            tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
+        } else if (warp >= 8 && c > 0) {
+            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((c - 1) & 1) * 128, false);
         }
         fence_async_smem();
+        tc_fence_before();
         __syncthreads();
         // the staging area is free again: the next chunk's raw inputs travel from now on
         if (c + 1 < nchunks) {
@@ -463,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             if (tid == 0) issue_raw(c + 1);
         }
 
-        // ===== P5: W^T = Kh^T T^T,  U^T = WV^T T^T =====
+        // ===== P5: W^T = Kh^T T^T,  U^T = WV^T T^T,  O^T = S^T Qg^T =====
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id = idesc_bf16(128, 64, true, false, false);
@@ -474,6 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 mma_bf16(tmem + TM_E, desc_mnmajor(sbase + OFF_WV, 64, 0, s),
                          desc_kmajor(sbase + OFF_T, 64, 0, s), id, s > 0);
             }
+            const uint32_t ido = idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+            for (int s = 0; s < DK / 16; ++s)
+                mma_bf16_ts(tmem + TM_O, tmem + TM_SB + s * 8, desc_kmajor(sbase + OFF_QK, 128, 64, s),
+                            ido, s > 0);
             mma_commit(bar_mma);
         }
         if (!Wm.all()) { ok = false; break; }

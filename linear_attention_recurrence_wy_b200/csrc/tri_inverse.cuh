@@ -72,9 +72,11 @@ __device__ __forceinline__ void block_store(float *Dm, int ldd, int r0, int c0, 
     }
 }
 
-// T_IJ = -T_II (A[I rows, J..I-1 blocks] T[J..I-1 blocks, J cols]) by one warp
-template <int NK>
-__device__ __forceinline__ void off_block(const float *A, float *T, float *X, int I, int J, int lane) {
+// T_IJ = -T_II (A[I rows, J..I-1 blocks] T[J..I-1 blocks, J cols]) by one warp; the final
+// block also goes to out.pair(row, col, T[row][col], T[row][col+1]) (col even).
+template <int NK, class Out>
+__device__ __forceinline__ void off_block(const float *A, float *T, float *X, int I, int J, int lane,
+                                          Out &out) {
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     block_mma<16 * NK>(acc, A, LD, 16 * I, 16 * J, T, LD, 16 * J, 16 * J, lane);
     block_store(X, XLD, 0, 0, acc, 1.f, lane);
@@ -82,16 +84,32 @@ __device__ __forceinline__ void off_block(const float *A, float *T, float *X, in
     float acc2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     block_mma<16>(acc2, T, LD, 16 * I, 16 * I, X, XLD, 0, 0, lane);
     block_store(T, LD, 16 * I, 16 * J, acc2, -1.f, lane);
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const int col = 16 * J + nh * 8 + 2 * t;
+        out.pair(16 * I + g, col, -acc2[nh][0], -acc2[nh][1]);
+        out.pair(16 * I + g + 8, col, -acc2[nh][2], -acc2[nh][3]);
+    }
 }
 
+// Output hook that discards the copy (callers that only need the fp32 T).
+struct NoOut {
+    __device__ __forceinline__ void chunk(int, int, const float (&)[8]) {}
+    __device__ __forceinline__ void pair(int, int, float, float) {}
+};
+
 // Called by four whole warps (warp = 0..3 within the group, lane = 0..31).  A, T: fp32
-// [64][LD]; A must hold zeros on and above its diagonal.  X: 4 x 16 x XLD fp32 scratch.
+// [64][LD]; only the strictly lower triangle of A is read.  X: 4 x 16 x XLD fp32 scratch.
 // sync() must be a barrier over exactly the four calling warps.  On return T holds the
 // full lower triangle (unit diagonal) and zeros above the diagonal of each diagonal
-// block; the strictly upper off-diagonal blocks of T are not written.
-template <class Sync>
+// block; the strictly upper off-diagonal blocks of T are not written.  Every final value
+// is also handed to `out`: out.chunk(row, c8, v[8]) for columns 8 c8 .. 8 c8 + 7 of the
+// diagonal blocks (zeros above the diagonal included) and out.pair for the off-diagonal
+// blocks.
+template <class Sync, class Out>
 __device__ __forceinline__ void inverse64(const float *A, float *T, float *X, int warp, int lane,
-                                          Sync sync) {
+                                          Sync sync, Out out) {
     {
         // diagonal block T_ww: lane (i = lane & 15, h = lane >> 4) owns row i, columns
         // 8h..8h+7, and holds row i of A_ww in registers.  Row m of T is final after step
@@ -118,14 +136,15 @@ __device__ __forceinline__ void inverse64(const float *A, float *T, float *X, in
         float4 *dst = reinterpret_cast<float4 *>(T + (o + i) * LD + o + 8 * h);
         dst[0] = make_float4(tr[0], tr[1], tr[2], tr[3]);
         dst[1] = make_float4(tr[4], tr[5], tr[6], tr[7]);
+        out.chunk(o + i, (o >> 3) + h, tr);
     }
     sync();
     float *Xw = X + warp * 16 * XLD;
-    if (warp < 3) off_block<1>(A, T, Xw, warp + 1, warp, lane);        // T10, T21, T32
+    if (warp < 3) off_block<1>(A, T, Xw, warp + 1, warp, lane, out);   // T10, T21, T32
     sync();
-    if (warp < 2) off_block<2>(A, T, Xw, warp + 2, warp, lane);        // T20, T31
+    if (warp < 2) off_block<2>(A, T, Xw, warp + 2, warp, lane, out);   // T20, T31
     sync();
-    if (warp == 0) off_block<3>(A, T, Xw, 3, 0, lane);                 // T30
+    if (warp == 0) off_block<3>(A, T, Xw, 3, 0, lane, out);            // T30
     sync();
 }
 

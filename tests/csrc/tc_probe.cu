@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(128) tri_probe_kernel(const float *A, float *T
         sA[r * gdr::tri::LD + c] = (c < r) ? Am[i] : 0.f;
     }
     __syncthreads();
-    gdr::tri::inverse64(sA, sT, sX, threadIdx.x >> 5, threadIdx.x & 31, ProbeBar128{});
+    gdr::tri::inverse64(sA, sT, sX, threadIdx.x >> 5, threadIdx.x & 31, ProbeBar128{},
+                         gdr::tri::NoOut{});
     __syncthreads();
     for (int i = threadIdx.x; i < 64 * 64; i += 128) {
         const int r = i / 64, c = i % 64;
