@@ -48,7 +48,8 @@ typedef enum {
     GDR_ERR_DTYPE = -4,    /* unknown gdr_dtype_t */
     GDR_ERR_ALIGN = -5,    /* a pointer is not 16-byte aligned */
     GDR_ERR_CUDA = -6,     /* a CUDA launch or attribute call failed */
-    GDR_ERR_TIMEOUT = -7   /* a bounded device-side wait gave up (tensor-core path) */
+    GDR_ERR_TIMEOUT = -7,  /* a bounded device-side wait gave up (tensor-core path) */
+    GDR_ERR_WORKSPACE = -8 /* workspace missing, misaligned or smaller than required */
 } gdr_status_t;
 
 typedef enum {
@@ -87,6 +88,43 @@ gdr_status_t gdr_chunk_fwd(const void *q, const void *k, const void *v, const fl
                            const void *b, const void *w, const float *S0, void *o, float *S_T,
                            int B, int H, int T, int dk, int dv, int chunk, gdr_mode_t mode,
                            gdr_dtype_t dtype, void *stream);
+
+/*
+ * Sequence split for long sequences with few sequence-heads.
+ *
+ * The recurrence is affine in the state: over a segment of the sequence,
+ * S_end = M S_start + S_local, with M (dk x dk) the product of the segment's per-token
+ * transitions (I - k (b.k)^T) diag(exp g) and S_local the end state reached from a zero
+ * start (Gated DeltaNet-2 Q&A page, Q3 update equation; only the state crosses chunk
+ * borders, Gated DeltaNet-2 Review §3-2.5).  gdr_chunk_fwd_split cuts every sequence into
+ * `nseg` segments of whole chunks and runs, on the stream, three kernels: (1) the end
+ * states S_local and the transitions M of the segments, all segments in parallel;
+ * (2) the chain S_start(s+1) = M_s S_start(s) + S_local(s) in fp32; (3) the forward of
+ * every segment from its own S_start, again in parallel.  Results equal gdr_chunk_fwd up
+ * to rounding; the work is about twice as large, the parallelism nseg times larger.
+ *
+ * Only the tensor-core shape is split (bf16, dk = dv = 128, chunk 64); for any other
+ * shape nseg must be 1.  nseg is clamped to the number of chunks and, after rounding
+ * segments to whole chunks, may shrink.  nseg == 1 is exactly gdr_chunk_fwd (no
+ * workspace needed).  The workspace is caller-owned device memory of at least
+ * gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg) bytes, 16-byte aligned; its
+ * contents are scratch and need no initialisation.  S_T may equal S0.
+ */
+
+/* Recommended segment count for this device and problem (1 = do not split). */
+int gdr_chunk_fwd_split_segments(int B, int H, int T, int dk, int dv, int chunk, gdr_dtype_t dtype);
+
+/* Workspace bytes needed by gdr_chunk_fwd_split (0 for invalid arguments). */
+unsigned long long gdr_chunk_fwd_split_workspace(int B, int H, int dk, int dv, int nseg);
+
+/* As gdr_chunk_fwd, with the sequence cut into nseg segments (see above).
+ * Returns GDR_ERR_WORKSPACE if nseg > 1 needs a workspace that is missing, misaligned or
+ * smaller than gdr_chunk_fwd_split_workspace(). */
+gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const void *v, const float *g_log,
+                                 const void *b, const void *w, const float *S0, void *o,
+                                 float *S_T, int B, int H, int T, int dk, int dv, int chunk,
+                                 gdr_mode_t mode, gdr_dtype_t dtype, int nseg, void *workspace,
+                                 unsigned long long workspace_bytes, void *stream);
 
 /*
  * gdr_decode_step -- one-token recurrent update for N sequences x H heads.

@@ -5,9 +5,10 @@ shapes and dtypes, allocates outputs with PyTorch and passes raw device pointers
 and the current CUDA stream to the C ABI (include/gdr.h).  There is no CPU or
 PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raised.
 
-Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_decode_step,
+Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
+gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace, gdr_decode_step,
 gdr_last_device_error, gdr_status_string.
-Tensor wrappers:  chunk_fwd, chunk_fwd_host, decode_step.
+Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, decode_step.
 """
 from __future__ import annotations
 
@@ -40,6 +41,12 @@ def lib():
         vp, ci = ctypes.c_void_p, ctypes.c_int
         L.gdr_chunk_fwd.argtypes = [vp] * 9 + [ci] * 8 + [vp]
         L.gdr_chunk_fwd.restype = ci
+        L.gdr_chunk_fwd_split.argtypes = [vp] * 9 + [ci] * 9 + [vp, ctypes.c_ulonglong, vp]
+        L.gdr_chunk_fwd_split.restype = ci
+        L.gdr_chunk_fwd_split_segments.argtypes = [ci] * 7
+        L.gdr_chunk_fwd_split_segments.restype = ci
+        L.gdr_chunk_fwd_split_workspace.argtypes = [ci] * 5
+        L.gdr_chunk_fwd_split_workspace.restype = ctypes.c_ulonglong
         L.gdr_decode_step.argtypes = [vp] * 8 + [ci] * 6 + [vp]
         L.gdr_decode_step.restype = ci
         L.gdr_last_device_error.argtypes = [vp]
@@ -54,6 +61,20 @@ def lib():
 def gdr_chunk_fwd(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype, stream):
     return lib().gdr_chunk_fwd(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode,
                                dtype, stream)
+
+
+def gdr_chunk_fwd_split(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype, nseg,
+                        workspace, workspace_bytes, stream):
+    return lib().gdr_chunk_fwd_split(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode,
+                                     dtype, nseg, workspace, workspace_bytes, stream)
+
+
+def gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, dtype):
+    return lib().gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, dtype)
+
+
+def gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg):
+    return lib().gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg)
 
 
 def gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, stream):
@@ -125,6 +146,42 @@ def chunk_fwd(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, o=None, 
                        B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], _stream())
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd")
+    return o, S_T
+
+
+def chunk_fwd_split(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, nseg=None,
+                    workspace=None, o=None, S_T=None, return_state=True):
+    """chunk_fwd with each sequence cut into `nseg` segments processed in parallel (for
+    long sequences with few sequence-heads).  nseg=None asks the library for its
+    recommendation; the workspace (uint8 CUDA tensor) is allocated here when not given."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    if nseg is None:
+        nseg = gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, DTYPES[dt])
+    if nseg <= 1:
+        return chunk_fwd(q, k, v, g, b, w, S0, mode=mode, chunk=chunk, o=o, S_T=S_T,
+                         return_state=return_state)
+    need = gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    gshape, bshape, wshape = _gate_shapes(mode, (B, H, T), dk, dv)
+    for t, name, shape, tdt in ((q, "q", (B, H, T, dk), dt), (k, "k", (B, H, T, dk), dt),
+                                (v, "v", (B, H, T, dv), dt), (g, "g", gshape, torch.float32),
+                                (b, "b", bshape, dt)):
+        _check(t, name, shape, tdt, q.device)
+    if mode == "gdn2":
+        _check(w, "w", wshape, dt, q.device)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=dt, device=q.device)
+    if S_T is None and return_state:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    rc = gdr_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
+                             _ptr(w) if mode == "gdn2" else None, _ptr(S0), _ptr(o), _ptr(S_T),
+                             B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], nseg,
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_split")
     return o, S_T
 
 

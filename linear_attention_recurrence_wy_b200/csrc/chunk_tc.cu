@@ -143,10 +143,27 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;   // TMEM lanes this warp may access: 32 * quarter + [0, 32)
-    const int bh = blockIdx.x;
-    const int T = a.T, mode = a.mode;
-    const size_t tok0 = (size_t)bh * T;
+    // ---- this CTA's job: one sequence-head, one segment of it, one role ----
+    const int roles = a.pass ? max(1, 2 * a.nseg - 3) : a.nseg;
+    const int bh = blockIdx.x / roles, role = blockIdx.x % roles;
+    const bool transfer = a.pass && role > a.nseg - 2;       // transition-matrix run
+    const int seg = transfer ? role - (a.nseg - 2) : role;
+    const int t_begin = seg * a.seg_len;
+    const int T = min(a.seg_len, a.T - t_begin);              // tokens of this segment
+    const int mode = a.mode;
+    const size_t tok0 = (size_t)bh * a.T + t_begin;
     const int nchunks = (T + C - 1) / C;
+    const size_t sidx = ((size_t)bh * a.nseg + seg) * DK * DV;
+    const float *S0p = nullptr;        // initial state (NULL: zero, unless the identity)
+    float *STp = nullptr;              // end state destination (NULL: not written)
+    if (!a.pass) {
+        S0p = a.nseg == 1 ? (a.S0 ? a.S0 + (size_t)bh * DK * DV : nullptr) : a.ws_sstart + sidx;
+        STp = seg == a.nseg - 1 ? (a.ST ? a.ST + (size_t)bh * DK * DV : nullptr) : nullptr;
+    } else {
+        S0p = (!transfer && seg == 0 && a.S0) ? a.S0 + (size_t)bh * DK * DV : nullptr;
+        STp = transfer ? a.ws_m + sidx : a.ws_send + sidx;
+    }
+    const bool write_o = !a.pass;
 
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *sT32 = reinterpret_cast<float *>(sm + OFF_T32);
@@ -227,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             float x[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j)
-                x[j] = a.S0 ? a.S0[((size_t)bh * DK + d0 + j) * DV + v] : 0.f;
+                x[j] = transfer ? (d0 + j == v ? 1.f : 0.f) : (S0p ? S0p[(size_t)(d0 + j) * DV + v] : 0.f);
             tmem_st32(tmem + lane_base + TM_S + d0, x);
             st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
         }
@@ -249,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (t0c + j < np) O[(tok0 + t0p + t0c + j) * DV + v] = __float2bfloat16_rn(x[j]);
+                    if (write_o && t0c + j < np) O[(tok0 + t0p + t0c + j) * DV + v] = __float2bfloat16_rn(x[j]);
             }
         } else {
             const int v = quarter * 32 + lane;
@@ -266,9 +283,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
                 tmem_st8(tmem + lane_base + TM_SB + d0 / 2, pk);
-                if (last && a.ST) {
+                if (last && STp) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) a.ST[((size_t)bh * DK + d0 + j) * DV + v] = x[j];
+                    for (int j = 0; j < 16; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
                 }
             }
             tmem_wait_st();
@@ -361,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     const float e = __expf(gam[j]);
                     kh[j] = fb[j] * fk[j] * e;
                     qg[j] = fq[j] * e;
-                    wv[j] = fw[j] * fv[j];
+                    wv[j] = transfer ? 0.f : fw[j] * fv[j];
                 }
                 if (exact) {
 #pragma unroll
@@ -593,7 +610,8 @@ gdr_status_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     if (cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
-    chunk_tc_kernel<<<(unsigned)(a.B * a.H), kThreads, SMEM_BYTES, s>>>(a);
+    const int roles = a.pass ? (2 * a.nseg - 3 > 1 ? 2 * a.nseg - 3 : 1) : a.nseg;
+    chunk_tc_kernel<<<(unsigned)(a.B * a.H * roles), kThreads, SMEM_BYTES, s>>>(a);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

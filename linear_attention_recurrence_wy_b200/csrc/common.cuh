@@ -15,6 +15,13 @@ struct ChunkArgs {
     void *o;
     float *ST;
     int B, H, T, dk, dv, chunk, mode, dtype;
+    // Sequence split (tensor-core kernel only).  nseg == 1 is the plain whole-sequence call.
+    // pass 0 writes outputs (segment s starts from S0 if s == 0, else from ws_sstart[bh][s]);
+    // pass 1 writes only end states: the local end state of segments 0 .. nseg-2
+    // (ws_send; segment 0 from S0, others from zero) and the transition matrices of
+    // segments 1 .. nseg-2 (ws_m; identity start state, values taken as zero).
+    int nseg, seg_len, pass;
+    float *ws_send, *ws_m, *ws_sstart;   // [B*H][nseg][dk][dv] fp32 each
 };
 
 struct DecodeArgs {
@@ -39,5 +46,6 @@ __device__ __forceinline__ void st_elem(void *p, size_t i, int dtype, float x) {
 gdr_status_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 gdr_status_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 gdr_status_t launch_state_copy(const ChunkArgs &a, cudaStream_t s);
+gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);
 
 }  // namespace gdr

@@ -23,6 +23,43 @@ gdr_status_t check_common(int mode, int dtype, int n0, int H, int dk, int dv) {
     return GDR_OK;
 }
 
+gdr_status_t check_chunk(const void *q, const void *k, const void *v, const float *g_log,
+                         const void *b, const void *w, const float *S0, const void *o,
+                         const float *S_T, int B, int H, int T, int dk, int dv, int chunk,
+                         int mode, int dtype) {
+    gdr_status_t st = check_common(mode, dtype, B, H, dk, dv);
+    if (st != GDR_OK) return st;
+    if (T < 0 || !chunk_ok(chunk)) return GDR_ERR_DIM;
+    if ((int64_t)B * H > INT32_MAX / 64) return GDR_ERR_DIM;
+    if ((int64_t)B * H * T > 0) {
+        if (!q || !k || !v || !g_log || !b || !o) return GDR_ERR_NULL;
+        if (mode == GDR_MODE_GDN2 && !w) return GDR_ERR_NULL;
+    }
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g_log) || !aligned16(b) ||
+        !aligned16(w) || !aligned16(S0) || !aligned16(o) || !aligned16(S_T))
+        return GDR_ERR_ALIGN;
+    return GDR_OK;
+}
+
+ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_log, const void *b,
+                    const void *w, const float *S0, void *o, float *S_T, int B, int H, int T,
+                    int dk, int dv, int chunk, int mode, int dtype) {
+    ChunkArgs a{q, k, v, b, mode == GDR_MODE_GDN2 ? w : nullptr, g_log, S0, o, S_T,
+                B, H, T, dk, dv, chunk, mode, dtype,
+                1, T, 0, nullptr, nullptr, nullptr};
+    return a;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
 }  // namespace
 
 extern "C" gdr_status_t gdr_chunk_fwd(const void *q, const void *k, const void *v,
@@ -42,13 +79,86 @@ extern "C" gdr_status_t gdr_chunk_fwd(const void *q, const void *k, const void *
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g_log) || !aligned16(b) ||
         !aligned16(w) || !aligned16(S0) || !aligned16(o) || !aligned16(S_T))
         return GDR_ERR_ALIGN;
-    ChunkArgs a{q, k, v, b, mode == GDR_MODE_GDN2 ? w : nullptr, g_log, S0, o, S_T,
-                B, H, T, dk, dv, chunk, (int)mode, (int)dtype};
+    ChunkArgs a = make_args(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((int64_t)B * H == 0) return GDR_OK;
     if (T == 0) return launch_state_copy(a, s);
     if (chunk_tc_supported(a)) return launch_chunk_tc(a, s);
     return launch_chunk_simt(a, s);
+}
+
+// ---- sequence split -------------------------------------------------------------------
+namespace {
+
+// segment length (in chunks) and effective segment count for a requested count
+void split_geometry(int nchunks, int nseg, int *seg_chunks, int *nseg_eff) {
+    if (nseg > nchunks) nseg = nchunks;
+    if (nseg < 1) nseg = 1;
+    *seg_chunks = (nchunks + nseg - 1) / nseg;
+    *nseg_eff = (nchunks + *seg_chunks - 1) / *seg_chunks;
+}
+
+}  // namespace
+
+extern "C" int gdr_chunk_fwd_split_segments(int B, int H, int T, int dk, int dv, int chunk,
+                                            gdr_dtype_t dtype) {
+    if (B <= 0 || H <= 0 || T <= 0 || dtype != GDR_BF16 || dk != 128 || dv != 128 || chunk != 64)
+        return 1;
+    const int units = B * H, sms = sm_count(), nchunks = (T + chunk - 1) / chunk;
+    // time model in chunk-steps: first pass (state only, ~0.9 of a chunk) in waves of
+    // units * (2 nseg - 3) CTAs, second pass in waves of units * nseg CTAs
+    double best = (double)((units + sms - 1) / sms) * nchunks;
+    int best_n = 1;
+    for (int n = 2; n <= 64 && n <= nchunks; ++n) {
+        int sc, ne;
+        split_geometry(nchunks, n, &sc, &ne);
+        if (ne < 2) continue;
+        const int r1 = 2 * ne - 3 > 1 ? 2 * ne - 3 : 1;
+        const double t = 0.9 * ((units * r1 + sms - 1) / sms) * sc + (double)((units * ne + sms - 1) / sms) * sc;
+        if (t < 0.8 * best) {   // split only for a clear gain
+            best = t;
+            best_n = ne;
+        }
+    }
+    return best_n;
+}
+
+extern "C" unsigned long long gdr_chunk_fwd_split_workspace(int B, int H, int dk, int dv, int nseg) {
+    if (B < 0 || H < 0 || !dim_ok(dk) || !dim_ok(dv) || nseg < 1) return 0;
+    return 3ull * (unsigned long long)B * H * nseg * dk * dv * sizeof(float);
+}
+
+extern "C" gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const void *v,
+                                            const float *g_log, const void *b, const void *w,
+                                            const float *S0, void *o, float *S_T, int B, int H,
+                                            int T, int dk, int dv, int chunk, gdr_mode_t mode,
+                                            gdr_dtype_t dtype, int nseg, void *workspace,
+                                            unsigned long long workspace_bytes, void *stream) {
+    gdr_status_t st = check_chunk(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype);
+    if (st != GDR_OK) return st;
+    if (nseg < 1) return GDR_ERR_DIM;
+    ChunkArgs a = make_args(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int seg_chunks = 1, nseg_eff = 1;
+    if (T > 0) split_geometry((T + chunk - 1) / chunk, nseg, &seg_chunks, &nseg_eff);
+    if (nseg_eff > 1 && !chunk_tc_supported(a)) return GDR_ERR_DIM;
+    if (nseg_eff <= 1 || (int64_t)B * H == 0)
+        return gdr_chunk_fwd(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype, stream);
+    const unsigned long long need = gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg_eff);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDR_ERR_WORKSPACE;
+    if ((int64_t)B * H * (2 * nseg_eff) > INT32_MAX) return GDR_ERR_DIM;
+    const size_t per = (size_t)B * H * nseg_eff * dk * dv;
+    float *ws = static_cast<float *>(workspace);
+    a.nseg = nseg_eff;
+    a.seg_len = seg_chunks * chunk;
+    a.ws_send = ws;
+    a.ws_m = ws + per;
+    a.ws_sstart = ws + 2 * per;
+    a.pass = 1;
+    if ((st = launch_chunk_tc(a, s)) != GDR_OK) return st;
+    if ((st = launch_split_combine(a, s)) != GDR_OK) return st;
+    a.pass = 0;
+    return launch_chunk_tc(a, s);
 }
 
 extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v,
@@ -87,6 +197,7 @@ extern "C" const char *gdr_status_string(gdr_status_t status) {
         case GDR_ERR_ALIGN: return "GDR_ERR_ALIGN: pointer not 16-byte aligned";
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: CUDA launch or runtime error";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait expired";
+        case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing, misaligned or too small";
     }
     return "unknown gdr_status_t";
 }

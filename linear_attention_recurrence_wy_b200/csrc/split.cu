@@ -1,0 +1,64 @@
+// split.cu -- chaining the segment states of a sequence split.
+//
+// The recurrence is affine in the state: over a segment, S_end = M S_start + S_local,
+// where M (dk x dk) is the product of the segment's per-token transitions
+// (I - k (b.k)^T) diag(exp g) and S_local is the end state reached from S_start = 0
+// (Gated DeltaNet-2 Q&A page, Q3 update equation; only the state crosses chunk and
+// segment borders, Gated DeltaNet-2 Review §3-2.5).  The first pass of the split
+// computes M and S_local of the inner segments in parallel; this kernel chains them
+// in fp32:
+//     S_start(0) = S0,  S_start(1) = S_end(0),  S_start(s+1) = M_s S_start(s) + S_local(s)
+// and the second pass recomputes every segment from its S_start.
+#include "common.cuh"
+
+namespace gdr {
+namespace {
+
+constexpr int DK = 128, DV = 128, COLS = 16;   // one CTA: one sequence-head, 16 state columns
+
+__global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
+    const int slices = DV / COLS;
+    const int bh = blockIdx.x / slices, c0 = (blockIdx.x % slices) * COLS;
+    const int tid = threadIdx.x, i = tid >> 1, h = tid & 1;   // row i, columns c0 + 8h ..
+    __shared__ float S[DK][COLS + 1];
+    const size_t head = (size_t)bh * a.nseg * DK * DV;
+    const size_t seg_sz = (size_t)DK * DV;
+    float *sstart = a.ws_sstart + head;
+    // S_start(0) = S0 (zeros if absent): the second pass reads every start state from here
+    for (int j = 0; j < 8; ++j) {
+        const int c = c0 + 8 * h + j;
+        sstart[(size_t)i * DV + c] = a.S0 ? a.S0[(size_t)bh * DK * DV + (size_t)i * DV + c] : 0.f;
+        S[i][8 * h + j] = a.ws_send[head + (size_t)i * DV + c];   // S_end(0)
+    }
+    __syncthreads();
+    for (int s = 1; s < a.nseg; ++s) {
+        for (int j = 0; j < 8; ++j) sstart[s * seg_sz + (size_t)i * DV + c0 + 8 * h + j] = S[i][8 * h + j];
+        if (s == a.nseg - 1) break;
+        const float *M = a.ws_m + head + s * seg_sz + (size_t)i * DK;
+        const float *L = a.ws_send + head + s * seg_sz + (size_t)i * DV + c0 + 8 * h;
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = L[j];
+        for (int k0 = 0; k0 < DK; k0 += 4) {
+            const float4 m = *reinterpret_cast<const float4 *>(M + k0);
+            const float mk[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = fmaf(mk[kk], S[k0 + kk][8 * h + j], acc[j]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) S[i][8 * h + j] = acc[j];
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s) {
+    split_combine_kernel<<<(unsigned)(a.B * a.H * (DV / COLS)), 256, 0, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+}  // namespace gdr

@@ -13,7 +13,7 @@ from linear_attention_recurrence_wy_b200 import build as gbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "gdr.h")
 
-OK, NULL, DIM, MODE, DTYPE, ALIGN = 0, -1, -2, -3, -4, -5
+OK, NULL, DIM, MODE, DTYPE, ALIGN, WORKSPACE = 0, -1, -2, -3, -4, -5, -8
 
 
 @pytest.fixture(scope="module")
@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
         s = gdr.gdr_status_string(code)
         assert s.startswith("GDR_")
     assert "unknown" in gdr.gdr_status_string(42)
@@ -104,3 +104,27 @@ def test_product_path_does_not_import_the_oracle():
                 txt = open(os.path.join(dirpath, f)).read()
                 for bad in ("import oracle", "from oracle", "gdr_oracle", "libgdr_oracle"):
                     assert bad not in txt, (f, bad)
+
+
+def call_split(nseg=4, ws=A, ws_bytes=1 << 30, dk=128, dv=128, chunk=64, dtype=1, T=1024, B=1, H=2):
+    return gdr.gdr_chunk_fwd_split(A, A, A, A, A, A, None, A, None, B, H, T, dk, dv, chunk, 0, dtype,
+                                   nseg, ws, ws_bytes, None)
+
+
+def test_split_workspace_size_and_segments(L):
+    assert gdr.gdr_chunk_fwd_split_workspace(2, 3, 128, 128, 4) == 3 * 2 * 3 * 4 * 128 * 128 * 4
+    assert gdr.gdr_chunk_fwd_split_workspace(1, 1, 100, 128, 4) == 0
+    # only the tensor-core shape is split; few sequence-heads and a long sequence do split
+    assert gdr.gdr_chunk_fwd_split_segments(1, 16, 16384, 128, 128, 64, 1) > 1
+    assert gdr.gdr_chunk_fwd_split_segments(8, 16, 4096, 128, 128, 64, 1) == 1
+    assert gdr.gdr_chunk_fwd_split_segments(1, 1, 16384, 64, 64, 64, 1) == 1
+    assert gdr.gdr_chunk_fwd_split_segments(1, 1, 16384, 128, 128, 64, 0) == 1
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), WORKSPACE), (dict(ws_bytes=1000), WORKSPACE), (dict(ws=A + 8), WORKSPACE),
+    (dict(nseg=0), DIM), (dict(dk=64, nseg=2), DIM), (dict(dtype=0, nseg=2), DIM),
+    (dict(chunk=32, nseg=2), DIM),
+])
+def test_split_rejects(L, kw, code):
+    assert call_split(**kw) == code
