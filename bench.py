@@ -296,15 +296,28 @@ def run_ours(args, rank, world, local):
         ST = torch.empty(wl.B, wl.H, wl.dk, wl.dv, dtype=torch.float32, device=dev)
         if chunk_bytes(wl, mode) <= 126e6:
             flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        dt_code = 1 if wl.dtype == "bf16" else 0
+        nseg = gdr.gdr_chunk_fwd_split_segments(wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.chunk, dt_code)
+        ws = None
+        if nseg > 1:
+            ws = torch.empty(gdr.gdr_chunk_fwd_split_workspace(wl.B, wl.H, wl.dk, wl.dv, nseg),
+                             dtype=torch.uint8, device=dev)
+
+        def fwd():
+            if nseg > 1:
+                gdr.chunk_fwd_split(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"],
+                                    mode=mode, chunk=wl.chunk, nseg=nseg, workspace=ws, o=o, S_T=ST)
+            else:
+                gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=mode,
+                              chunk=wl.chunk, o=o, S_T=ST)
 
         def step():
             if flush is not None:
                 flush.zero_()
-            gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=mode,
-                          chunk=wl.chunk, o=o, S_T=ST)
+            fwd()
         units = wl.units
         bytes_per_launch = chunk_bytes(wl, mode)
-        launches_per_step = 1
+        launches_per_step = 3 if nseg > 1 else 1
         unit = "token-heads/s"
 
     for _ in range(args.warmup):
@@ -330,8 +343,7 @@ def run_ours(args, rank, world, local):
             if name == "decode":
                 step()
             else:
-                gdr.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], mode=mode,
-                              chunk=wl.chunk, o=o, S_T=ST)
+                fwd()
             ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
@@ -373,11 +385,19 @@ def run_ours(args, rank, world, local):
 
     if rank != 0:
         return
-    launch_ms = kern_ms / launches_per_step
+    if name == "decode":
+        launch_ms = kern_ms / launches_per_step
+        kname = "gdr decode_kernel"
+    else:
+        # one step = the whole forward; with a sequence split it is three launches
+        # (state pass, combine, output pass) and the step is the unit of the roofline
+        launch_ms = kern_ms
+        kname = kernel_name(wl, mode) if nseg <= 1 else \
+            f"gdr chunk_tc_kernel x2 + split_combine_kernel (sequence split, {nseg} segments)"
     achieved = bytes_per_launch / (launch_ms * 1e-3) / 1e9
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "traffic": args.traffic, "peak_source": f"{peak_src} hbm_gbs",
-            "kernel": "gdr decode_kernel" if name == "decode" else kernel_name(wl, mode)}
+            "frac": achieved / hbm, "traffic": traffic_for(name, kname), "peak_source": f"{peak_src} hbm_gbs",
+            "kernel": kname}
     if name != "decode":
         fl = chunk_flops(wl)
         roof["tensor_context"] = {"flops_per_launch": fl,
@@ -394,6 +414,37 @@ def run_ours(args, rank, world, local):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(name, target_cpu_s=args.ref_cpu_s)
     print(json.dumps(line), flush=True)
+
+
+# ncu dram__bytes_read.sum + dram__bytes_write.sum per launch of the dominant kernel,
+# keyed by workload and by a digest of the kernel's sources at capture time (a changed
+# kernel reports null until it is captured again); see profiles/.
+TRAFFIC = {
+    ("gdn2_t4k", "chunk_tc"): (953.813248e6 + 124.982528e6, "b9da433a"),
+    ("decode", "decode"): (275.789312e6 + 211.644416e6, "938c1bac"),
+}
+
+
+def _src_digest(files):
+    import hashlib
+    h = hashlib.sha1()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "linear_attention_recurrence_wy_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:8]
+
+
+def traffic_for(name, kname):
+    if name == "decode":
+        key, files = ("decode", "decode"), ["decode.cu"]
+    elif "chunk_tc" in kname and "split" not in kname:
+        key, files = (name, "chunk_tc"), ["chunk_tc.cu", "tri_inverse.cuh", "tc_util.cuh"]
+    else:
+        return None
+    rec = TRAFFIC.get(key)
+    if rec is None:
+        return None
+    value, digest = rec
+    return value if _src_digest(files) == digest else None
 
 
 def kernel_name(wl, mode):
