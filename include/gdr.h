@@ -127,6 +127,33 @@ gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const void *v, co
                                  unsigned long long workspace_bytes, void *stream);
 
 /*
+ * gdr_chunk_fwd_split_noalloc -- gdr_chunk_fwd_split without a caller workspace.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory: plugins whose host framework owns every device allocation,
+ * and latency-critical loops where a cudaMalloc, which may synchronise the device, is
+ * not acceptable.  Its workspace is a fixed 24 MiB array inside the library (every GPU
+ * that loads the library holds it until the process exits); the call itself allocates
+ * nothing.  Arguments and results are those of gdr_chunk_fwd_split.
+ *
+ *   - Limit: the split's workspace, gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg),
+ *     must fit in 24 MiB (e.g. B*H*nseg <= 128 at dk = dv = 128); larger requests
+ *     return GDR_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture begins.
+ *   - Every call shares the one array, which keeps the previous call's contents; the
+ *     split reads only what the same call wrote, so nothing needs clearing.  Calls
+ *     that overlap on the GPU (for example on two streams) race on the array and must
+ *     be serialised by the caller.
+ */
+gdr_status_t gdr_chunk_fwd_split_noalloc(const void *q, const void *k, const void *v,
+                                         const float *g_log, const void *b, const void *w,
+                                         const float *S0, void *o, float *S_T, int B, int H,
+                                         int T, int dk, int dv, int chunk, gdr_mode_t mode,
+                                         gdr_dtype_t dtype, int nseg, void *stream);
+
+/*
  * gdr_decode_step -- one-token recurrent update for N sequences x H heads.
  *
  * The recurrent form used for constant-memory decoding (Gated DeltaNet-2 Q&A page,

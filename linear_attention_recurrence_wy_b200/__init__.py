@@ -6,7 +6,8 @@ and the current CUDA stream to the C ABI (include/gdr.h).  There is no CPU or
 PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raised.
 
 Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
-gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace, gdr_decode_step,
+gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
+gdr_decode_step,
 gdr_last_device_error, gdr_status_string.
 Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, decode_step.
 """
@@ -43,6 +44,8 @@ def lib():
         L.gdr_chunk_fwd.restype = ci
         L.gdr_chunk_fwd_split.argtypes = [vp] * 9 + [ci] * 9 + [vp, ctypes.c_ulonglong, vp]
         L.gdr_chunk_fwd_split.restype = ci
+        L.gdr_chunk_fwd_split_noalloc.argtypes = [vp] * 9 + [ci] * 9 + [vp]
+        L.gdr_chunk_fwd_split_noalloc.restype = ci
         L.gdr_chunk_fwd_split_segments.argtypes = [ci] * 7
         L.gdr_chunk_fwd_split_segments.restype = ci
         L.gdr_chunk_fwd_split_workspace.argtypes = [ci] * 5
@@ -67,6 +70,12 @@ def gdr_chunk_fwd_split(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk
                         workspace, workspace_bytes, stream):
     return lib().gdr_chunk_fwd_split(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode,
                                      dtype, nseg, workspace, workspace_bytes, stream)
+
+
+def gdr_chunk_fwd_split_noalloc(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode,
+                                dtype, nseg, stream):
+    return lib().gdr_chunk_fwd_split_noalloc(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv,
+                                             chunk, mode, dtype, nseg, stream)
 
 
 def gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, dtype):
