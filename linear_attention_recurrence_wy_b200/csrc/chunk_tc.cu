@@ -24,9 +24,9 @@
 // Data movement: each chunk's raw inputs arrive by bulk copies (one per tensor) into a
 // staging area, issued one chunk ahead and backed by L2 prefetches two chunks ahead.
 // The bf16 copies of S^T and E^T that feed the MMAs as A operands stay in TMEM.
-// Schedule (16 warps): all warps build the operands; warps 0-3 invert while warps 8-15
-// write the previous chunk's output rows and scale its state, whose first reader is this
-// chunk's S^T Qg^T MMA, issued together with W^T and U^T.
+// Schedule (16 warps): all warps build the operands; while the tensor cores form [A; P],
+// warps 8-15 write the previous chunk's output rows and scale its state, whose first
+// reader is this chunk's S^T Qg^T MMA, issued together with W^T and U^T.
 //
 // Every wait on an mbarrier is bounded; on expiry the kernel records the failure in
 // g_tc_error, stops issuing work, waits (bounded) for its own bulk copies and
@@ -258,38 +258,35 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     // warps 0-7 build the next chunk's operands: that chunk's first MMA is the first
     // reader of what is written here.
     auto finish_chunk = [&](int t0p, int np, bool exactp, const float *egc, bool last) {
+        const int v = quarter * 32 + lane;
         if (warp < 12) {
-            const int v = quarter * 32 + lane;
-            for (int t0c = 0; t0c < 64; t0c += 16) {
-                float x[16];
-                tmem_ld16(tmem + lane_base + TM_O + t0c, x);
+            for (int t0c = 0; t0c < 64; t0c += 32) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_O + t0c, x);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
+                for (int j = 0; j < 32; ++j)
                     if (write_o && t0c + j < np) O[(tok0 + t0p + t0c + j) * DV + v] = __float2bfloat16_rn(x[j]);
             }
         } else {
-            const int v = quarter * 32 + lane;
-            for (int d0 = 0; d0 < DK; d0 += 16) {
-                float x[16];
-                tmem_ld16(tmem + lane_base + TM_S + d0, x);
+            for (int d0 = 0; d0 < DK; d0 += 32) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_S + d0, x);
                 tmem_wait_ld();
                 if (!exactp) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) x[j] *= egc[d0 + j];
-                    tmem_st16(tmem + lane_base + TM_S + d0, reinterpret_cast<const uint32_t(&)[16]>(x));
+                    for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
+                    tmem_st32(tmem + lane_base + TM_S + d0, x);
                 }
-                uint32_t pk[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
-                tmem_st8(tmem + lane_base + TM_SB + d0 / 2, pk);
+                st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
                 if (last && STp) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
+                    for (int j = 0; j < 32; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
                 }
             }
             tmem_wait_st();
         }
+        tc_fence_before();
     };
 
     Waiter Wm{bar_mma, 0u}, Wr{bar_raw, 0u};
@@ -396,43 +393,51 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         fence_async_smem();
         __syncthreads();
 
-        // ===== P2: [A;P] = [Kh;Qg] Kb^T =====
-        if (!exact) {
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 64, false, false, false);
+        // ===== P2: [A;P] = [Kh;Qg] Kb^T | previous chunk's outputs and state (warps 8-15) =====
+        if (!exact && tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, false, false, false);
 #pragma unroll
-                for (int s = 0; s < DK / 16; ++s)
-                    mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s),
-                             desc_kmajor(sbase + OFF_KB, 64, 0, s), id, s > 0);
-                mma_commit(bar_mma);
-            }
+            for (int s = 0; s < DK / 16; ++s)
+                mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s),
+                         desc_kmajor(sbase + OFF_KB, 64, 0, s), id, s > 0);
+            mma_commit(bar_mma);
+        }
+        if (warp >= 8 && c > 0)
+            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((c - 1) & 1) * 128, false);
+        if (!exact) {
             if (!Wm.all()) { ok = false; break; }
+        } else {
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
         }
 
         // ===== P3: A (fp32, strictly lower) and P (bf16, lower incl.) =====
         if (!exact) {
-            const int r = quarter * 32 + lane, j0 = (warp >> 2) * 16;   // row of [A; P], columns
-            float x[16];
-            tmem_ld16(tmem + lane_base + TM_AP + j0, x);
-            tmem_wait_ld();
-            if (r < 64) {
-                float4 *dst = reinterpret_cast<float4 *>(sA32 + r * kAS + j0);
+            if (warp < 8) {
+                const int r = quarter * 32 + lane, j0 = (warp >> 2) * 32;   // row of [A; P], columns
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_AP + j0, x);
+                tmem_wait_ld();
+                if (r < 64) {
+                    float4 *dst = reinterpret_cast<float4 *>(sA32 + r * kAS + j0);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float y[4];
+                    for (int q = 0; q < 8; ++q) {
+                        float y[4];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
-                    dst[q] = make_float4(y[0], y[1], y[2], y[3]);
-                }
-            } else {
-                const int t = r - 64;
+                        for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
+                        dst[q] = make_float4(y[0], y[1], y[2], y[3]);
+                    }
+                } else {
+                    const int t = r - 64;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float f[8];
+                    for (int h = 0; h < 4; ++h) {
+                        float f[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
-                    st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+                        for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
+                        st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+                    }
                 }
             }
         } else {
@@ -469,12 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         }
         __syncthreads();
 
-        // ===== P4: T = (I + A)^-1 (warps 0-3) | previous chunk's outputs and state (8-15) =====
-        if (warp < 4) {
-            tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
-        } else if (warp >= 8 && c > 0) {
-            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((c - 1) & 1) * 128, false);
-        }
+        // ===== P4: T = (I + A)^-1 =====
+        if (warp < 4) tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
         fence_async_smem();
         tc_fence_before();
         __syncthreads();

@@ -2,9 +2,10 @@
 // held in shared memory, computed by four warps.
 //
 // Blocked forward substitution on 16 x 16 blocks (the stable order of the plain
-// substitution, reorganised):
-//   T_II = (I + A_II)^-1                                   substitution by rows, fp32
-//   T_IJ = -T_II X_IJ,  X_IJ = sum_{K=J}^{I-1} A_IK T_KJ   for I > J, by levels I - J
+// substitution, reorganised as a 2 x 2 block recursion):
+//   T_II = (I + A_II)^-1                                    substitution by rows, fp32
+//   T_10 = -T_11 A_10 T_00,   T_32 = -T_33 A_32 T_22        (the two 32 x 32 diagonal blocks)
+//   X    = A_[2:4,0:2] T_[0:2,0:2],  T_[2:4,0:2] = -T_[2:4,2:4] X   (the lower-left 32 x 32)
 // The diagonal blocks are solved row-per-lane in registers; every off-diagonal block
 // product runs on warp-level tensor-core MMAs (m16n8k8, TF32 operands rounded to nearest,
 // fp32 accumulation), so the shared-memory traffic is a few fragment loads per product.
@@ -139,12 +140,36 @@ __device__ __forceinline__ void inverse64(const float *A, float *T, float *X, in
         out.chunk(o + i, (o >> 3) + h, tr);
     }
     sync();
-    float *Xw = X + warp * 16 * XLD;
-    if (warp < 3) off_block<1>(A, T, Xw, warp + 1, warp, lane, out);   // T10, T21, T32
+    if (warp < 2) {
+        float *Xw = X + warp * 16 * XLD;
+        off_block<1>(A, T, Xw, 2 * warp + 1, 2 * warp, lane, out);   // T10, T32
+    }
     sync();
-    if (warp < 2) off_block<2>(A, T, Xw, warp + 2, warp, lane, out);   // T20, T31
+    // lower-left 32 x 32 block, one 16 x 16 block (I, J) per warp, I in {2, 3}, J in {0, 1}
+    const int I = 2 + (warp >> 1), J = warp & 1;
+    float *Xb = X + warp * 16 * XLD;   // X_IJ
+    {
+        // X_IJ = sum_{K=J}^{1} A_IK T_KJ  (T_01 = 0)
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if (J == 0) block_mma<32>(acc, A, LD, 16 * I, 0, T, LD, 0, 0, lane);
+        else block_mma<16>(acc, A, LD, 16 * I, 16, T, LD, 16, 16, lane);
+        block_store(Xb, XLD, 0, 0, acc, 1.f, lane);
+    }
     sync();
-    if (warp == 0) off_block<3>(A, T, Xw, 3, 0, lane, out);            // T30
+    {
+        // T_IJ = -sum_{K=2}^{I} T_IK X_KJ
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        block_mma<16>(acc, T, LD, 16 * I, 16 * I, X + ((I - 2) * 2 + J) * 16 * XLD, XLD, 0, 0, lane);
+        if (I == 3) block_mma<16>(acc, T, LD, 48, 32, X + J * 16 * XLD, XLD, 0, 0, lane);
+        block_store(T, LD, 16 * I, 16 * J, acc, -1.f, lane);
+        const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            const int col = 16 * J + nh * 8 + 2 * t;
+            out.pair(16 * I + g, col, -acc[nh][0], -acc[nh][1]);
+            out.pair(16 * I + g + 8, col, -acc[nh][2], -acc[nh][3]);
+        }
+    }
     sync();
 }
 
