@@ -1,18 +1,19 @@
 // chunk_tc.cu -- tcgen05 tensor-core chunkwise WY forward: bf16 operands, fp32 state.
 //
 // Shape: dk = dv = 128, chunk C = 64, bf16 q/k/v/b/w/o, fp32 g_log and state, any mode.
-// One CTA (256 threads) owns one (sequence, head); the fp32 state lives in tensor
-// memory (TMEM) for the whole sequence, transposed (lane = value channel v, column =
-// key channel d).  Per chunk (Gated DeltaNet-2 Review §3-2.5 "Chunkwise WY training";
-// Gated DeltaNet-2 Q&A page, Q4):
+// One CTA (512 threads) owns one (sequence, head) -- or one segment of it under the
+// sequence split -- and keeps the fp32 state in tensor memory (TMEM) for the whole run,
+// transposed (lane = value channel v, column = key channel d).  Per chunk (Gated
+// DeltaNet-2 Review §3-2.5 "Chunkwise WY training"; Gated DeltaNet-2 Q&A page, Q4):
 //
 //   gamma   = chunk-local cumulative sum of g_log (fp32, per key channel)
-//   Kh      = b.k.e^gamma,  Qg = q.e^gamma,  Kb = k.e^-gamma,  WV = w.v      (bf16, smem)
+//   Kh      = b.k.e^gamma,  Qg = q.e^gamma,  Kb = k.e^-gamma                (bf16, smem)
 //   [A; P]  = [Kh; Qg] Kb^T           one M=128 MMA; A strictly lower, P lower incl.
 //   T       = (I + A)^-1              blocked substitution (tri_inverse.cuh)
-//   W^T     = Kh^T T^T,  U^T = WV^T T^T
-//   E^T     = U^T - S^T W^T           (MMA with negated A, accumulating onto U^T)
-//   O^T     = S^T Qg^T + E^T P^T      (read-out of the post-update state)
+//   [X | O] = S^T [Kh; Qg]^T          one N=128 MMA: X = S^T Kh^T, O = S^T Qg^T
+//   R^T     = (w.v)^T - X             w.v formed in fp32 on read-out
+//   E^T     = R^T T^T                 the delta errors E = T (w.v - Kh S) = U - W S
+//   O^T    += E^T P^T                 (read-out of the post-update state)
 //   S^T     = (S^T + E^T Kb) diag(e^gamma_C)
 //
 // Writing Kb = k.e^-gamma and scaling after the state MMA equals S diag(e^gamma_C) +
@@ -21,16 +22,24 @@
 // exact path instead: A and P from per-pair decays exp(gamma_i - gamma_j) on CUDA cores,
 // K_end = k.e^(gamma_C - gamma) in place of Kb, and the state scaled before its MMA.
 //
-// Data movement: each chunk's raw inputs arrive by bulk copies (one per tensor) into a
-// staging area, issued one chunk ahead and backed by L2 prefetches two chunks ahead.
-// The bf16 copies of S^T and E^T that feed the MMAs as A operands stay in TMEM.
-// Schedule (16 warps): all warps build the operands; while the tensor cores form [A; P],
-// warps 8-15 write the previous chunk's output rows and scale its state, whose first
-// reader is this chunk's S^T Qg^T MMA, issued together with W^T and U^T.
+// Warp-specialised pipeline.  Warps 0-7 (the WY group) stage a chunk's q, k, b and g_log
+// (one bulk copy per tensor), scan the log-decay, build the operands, form [A; P] on the
+// tensor cores and invert (I + A).  Warps 8-15 (the state group) meanwhile run the
+// state-dependent chain of an earlier chunk: X and O, R (reading v and w straight from
+// global memory), E, the output and the state update, all on tcgen05 with their A
+// operands (bf16 S^T, R^T, E^T) read from TMEM.  The groups hand over through mbarriers:
+//   H1     operands of chunk c built           WY -> state
+//   H2[2]  T and P of chunk c ready            WY -> state   (by chunk parity)
+//   H3     Kh, Qg of chunk c consumed          state -> WY   (they may be rebuilt)
+//   H4[2]  chunk c finished                    state -> WY   (its P, T, Kb buffers are free)
+// Kb, P and T are double-buffered by chunk parity, so the WY group can run up to two
+// chunks ahead of the state group.  The next chunk's raw inputs are copied as soon as
+// the operands are built (fast path) or A and P are formed (exact path).
 //
-// Every wait on an mbarrier is bounded; on expiry the kernel records the failure in
-// g_tc_error, stops issuing work, waits (bounded) for its own bulk copies and
-// tensor-core work to drain, frees its TMEM and returns.
+// Every wait on an mbarrier is bounded.  On expiry a thread raises a CTA-wide abort flag;
+// both groups leave their loops at their next wait, the kernel records the failure in
+// g_tc_error, waits (bounded) for its own bulk copies and tensor-core work, frees its
+// TMEM and returns.
 #include "chunk_tc.cuh"
 #include "tc_util.cuh"
 #include "tri_inverse.cuh"
@@ -50,40 +59,39 @@ constexpr float kFastLimit = 60.f;
 constexpr int kAS = tri::LD;   // fp32 row stride of the A / T scratch
 
 // shared memory map (byte offsets from a 1024-aligned base)
-constexpr int RAW_Q = 0;                        // raw q bf16 [64][128]   16 KB
-constexpr int RAW_K = RAW_Q + 16384;            // raw k                  16 KB
-constexpr int RAW_V = RAW_K + 16384;            // raw v                  16 KB
-constexpr int RAW_B = RAW_V + 16384;            // raw b (GDN-2)          16 KB
-constexpr int RAW_W = RAW_B + 16384;            // raw w (GDN-2)          16 KB
-constexpr int RAW_G = RAW_W + 16384;            // raw g_log fp32 [64][128] 32 KB; gamma (exact path)
+constexpr int RAW_Q = 0;                        // raw q bf16 [64][128]     16 KB
+constexpr int RAW_K = RAW_Q + 16384;            // raw k                    16 KB
+constexpr int RAW_B = RAW_K + 16384;            // raw b (GDN-2)            16 KB
+constexpr int RAW_G = RAW_B + 16384;            // raw g_log fp32 [64][128] 32 KB, then gamma
 constexpr int RAW_END = RAW_G + 32768;
-// once a chunk's operands are built, raw v, b and w are dead: the inverse's scratch
-constexpr int OFF_A32 = RAW_V;                  // A fp32 [64][68]
-constexpr int OFF_T32 = OFF_A32 + 64 * kAS * 4; // T fp32 [64][68]
-constexpr int OFF_X = OFF_T32 + 64 * kAS * 4;   // 4 x [16][20] fp32
-static_assert(OFF_X + 4 * 16 * tri::XLD * 4 <= RAW_G, "inverse scratch must fit in raw v, b, w");
-constexpr int OFF_QK = RAW_END;                 // [Kh;Qg] bf16 [128][128]  32 KB
-constexpr int OFF_KB = OFF_QK + 32768;          // Kb    bf16 [64 t][128 d] 16 KB
-constexpr int OFF_WV = OFF_KB + 16384;          // WV    bf16 [64 t][128 v] 16 KB
-constexpr int OFF_P = OFF_WV + 16384;           // P     bf16 [64 t][64 j]   8 KB
-constexpr int OFF_T = OFF_P + 8192;             // T     bf16 [64 t][64 j]   8 KB
-constexpr int OFF_WT = OFF_T + 8192;            // W^T   bf16 [128 d][64 t] 16 KB
-constexpr int OFF_TOT = OFF_WT + 16384;         // scan: quarter totals fp32 [4][128]
+constexpr int OFF_A32 = RAW_END;                // inverse scratch: A fp32 [64][68]
+constexpr int OFF_T32 = OFF_A32 + 64 * kAS * 4; //                  T fp32 [64][68]
+constexpr int OFF_X = OFF_T32 + 64 * kAS * 4;   //                  4 x [16][20] fp32
+constexpr int OFF_QK = (OFF_X + 4 * 16 * tri::XLD * 4 + 1023) / 1024 * 1024;
+                                                // [Kh;Qg] bf16 [128][128]  32 KB
+constexpr int OFF_KB = OFF_QK + 32768;          // Kb bf16 [2][64 t][128 d] 32 KB
+constexpr int OFF_P = OFF_KB + 32768;           // P  bf16 [2][64 t][64 j]  16 KB
+constexpr int OFF_T = OFF_P + 16384;            // T  bf16 [2][64 t][64 j]  16 KB
+constexpr int OFF_TOT = OFF_T + 16384;          // scan: quarter totals fp32 [4][128]
 constexpr int OFF_GS = OFF_TOT + 2048;          // scalar g_log of the chunk (GDN) fp32 [64]
 constexpr int OFF_GC = OFF_GS + 256;            // gamma_C fp32 [128]
-constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [2][128], by chunk parity
-constexpr int OFF_BAR = OFF_EGC + 1024;         // 2 mbarriers + TMEM slot
-constexpr int SMEM_BYTES = OFF_BAR + 64 + 1024; // + alignment slack
+constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [4][128], slot c % 4
+constexpr int OFF_FLAG = OFF_EGC + 2048;        // exact flags [4] (slot c % 4), abort flag
+constexpr int OFF_BAR = OFF_FLAG + 64;          // mbarriers + TMEM slot
+constexpr int NBAR = 9;
+constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 8 + 1024;   // + alignment slack
 
 // TMEM columns
-constexpr uint32_t TM_S = 0;     // S^T fp32            128 cols
-constexpr uint32_t TM_O = 128;   // O^T fp32             64
-constexpr uint32_t TM_E = 192;   // U^T, then E^T fp32   64
-constexpr uint32_t TM_W = 256;   // W^T fp32             64
-constexpr uint32_t TM_AP = 320;  // [A; P] fp32          64
-constexpr uint32_t TM_SB = 384;  // S^T bf16 (packed)    64
-constexpr uint32_t TM_EB = 448;  // E^T bf16 (packed)    32
+constexpr uint32_t TM_S = 0;     // S^T fp32                                   128 cols
+constexpr uint32_t TM_XO = 128;  // [X, then E^T | O^T] fp32                  64 + 64
+constexpr uint32_t TM_AP = 256;  // [A; P] fp32                                 64
+constexpr uint32_t TM_SB = 320;  // S^T bf16 (packed)                           64
+constexpr uint32_t TM_XB = 384;  // R^T, then E^T bf16 (packed)                 32
 constexpr uint32_t TM_COLS = 512;
+
+// named barriers (0 is __syncthreads; 1 is warps 0-3, the inverse's; 4 is warps 4-7, the scan's)
+constexpr int BAR_WY = 2;    // warps 0-7
+constexpr int BAR_ST = 3;    // warps 8-15
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
     const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
@@ -93,6 +101,11 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
         f[2 * i] = x.x;
         f[2 * i + 1] = x.y;
     }
+}
+
+// v where in, else zero (a staged row past the end of the input holds stale data)
+__device__ __forceinline__ uint4 sel(bool in, uint4 v) {
+    return make_uint4(in ? v.x : 0u, in ? v.y : 0u, in ? v.z : 0u, in ? v.w : 0u);
 }
 
 __device__ __forceinline__ void st_chunk(uint32_t saddr, const float (&f)[8]) {
@@ -108,6 +121,67 @@ __device__ __forceinline__ void st_tmem_bf16(uint32_t taddr, const float (&x)[32
     tmem_st16(taddr, r);
 }
 
+// barrier over the 256 threads of one warp group
+__device__ __forceinline__ void group_sync(int id) {
+    asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
+}
+// barrier over one warp group that also returns the AND (or the OR) of v over it
+__device__ __forceinline__ bool group_and(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, 256, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool group_or(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, 256, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id)
+        : "memory");
+    return r != 0;
+}
+// the same over 128 threads (warps 4-7 of the WY group)
+__device__ __forceinline__ void bar128_sync(int id) {
+    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool bar128_and(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool bar128_or(int id, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr) : "memory");
+}
+
 // Final values of T (from the inverse) straight into the bf16 operand tile.
 struct TileOut {
     uint32_t tile;   // shared address of the T tile ([64 t][64 j], 128-byte swizzled)
@@ -120,22 +194,18 @@ struct TileOut {
     }
 };
 
-// barrier over warps 0-3 (named barrier 1)
+// barrier over warps 0-3 (named barrier 1), the inverse's warps
 struct Bar128 {
     __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 };
 
-struct Waiter {
-    uint32_t bar, phase;
-    // all threads wait for the barrier's next phase; false (everywhere) if any gave up
-    __device__ __forceinline__ bool all() {
-        const bool mine = mbar_wait(bar, phase, kWaitLimit);
-        phase ^= 1u;
-        const bool ok = !__syncthreads_or(!mine);
-        tc_fence_after();
-        return ok;
-    }
-};
+// After an abort: wait (bounded) until every commit issued on bar has arrived.  The
+// commits complete in order; n of them were issued, so phases n-2 and n-1 are waited
+// for in turn (a parity wait alone cannot tell phase n-1 from phase n-3).
+__device__ __forceinline__ void drain_commits(uint32_t bar, int n) {
+    if (n >= 2) mbar_wait(bar, (uint32_t)((n - 2) & 1), kWaitLimit);
+    if (n >= 1) mbar_wait(bar, (uint32_t)((n - 1) & 1), kWaitLimit);
+}
 
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     extern __shared__ unsigned char smem_raw[];
@@ -143,6 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     const uint32_t sbase = smem_u32(sm);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;   // TMEM lanes this warp may access: 32 * quarter + [0, 32)
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+
     // ---- this CTA's job: one sequence-head, one segment of it, one role ----
     const int roles = a.pass ? max(1, 2 * a.nseg - 3) : a.nseg;
     const int bh = blockIdx.x / roles, role = blockIdx.x % roles;
@@ -173,8 +245,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     float *sGs = reinterpret_cast<float *>(sm + OFF_GS);
     float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
     float *sEGC = reinterpret_cast<float *>(sm + OFF_EGC);
-    const uint32_t bar_mma = sbase + OFF_BAR, bar_raw = sbase + OFF_BAR + 8;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
+    volatile int *sExact = reinterpret_cast<volatile int *>(sm + OFF_FLAG);   // [4]
+    volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_FLAG + 16);
+    const uint32_t bar_wy = sbase + OFF_BAR;     // the WY group's MMA commits
+    const uint32_t bar_st = bar_wy + 8;          // the state group's MMA commits
+    const uint32_t bar_raw = bar_wy + 16;        // raw input copies
+    const uint32_t bar_h1 = bar_wy + 24, bar_h3 = bar_wy + 32;
+    const uint32_t bar_h2 = bar_wy + 40;         // [2], by chunk parity
+    const uint32_t bar_h4 = bar_wy + 56;         // [2], by chunk parity
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + NBAR * 8);
 
     const __nv_bfloat16 *Q = (const __nv_bfloat16 *)a.q, *K = (const __nv_bfloat16 *)a.k;
     const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
@@ -183,39 +262,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     const bool gdn2 = (mode == GDR_MODE_GDN2), vec_g = (mode != GDR_MODE_GDN);
 
     if (tid == 0) {
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_raw, 1);
+        for (int i = 0; i < NBAR; ++i) mbar_init(bar_wy + 8 * i, 1);
+        sAbort[0] = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(tslot), TM_COLS);
         tmem_relinquish();
     }
+    // the T tiles' blocks above the diagonal are never written: zero both tiles once
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid + kThreads] = make_uint4(0, 0, 0, 0);
+    static_assert(kThreads * 32 == 16384, "two 16-byte stores per thread clear the T tiles");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
-    // raw inputs of chunk c -> staging (one bulk copy per tensor), thread 0 only
-    auto issue_raw = [&](int c) {
-        const int t0 = c * C, n = min(C, T - t0);
-        const size_t e = (tok0 + t0) * DK;
-        const uint32_t row16 = (uint32_t)n * DK * 2;
-        uint32_t bytes = 3 * row16;
-        if (gdn2) bytes += 2 * row16;
-        if (vec_g) bytes += 2 * row16;
-        fence_async_smem();
-        mbar_arrive_expect_tx(bar_raw, bytes);
-        bulk_g2s(sbase + RAW_Q, Q + e, row16, bar_raw);
-        bulk_g2s(sbase + RAW_K, K + e, row16, bar_raw);
-        bulk_g2s(sbase + RAW_V, V + e, row16, bar_raw);
-        if (gdn2) {
-            bulk_g2s(sbase + RAW_B, Bg + e, row16, bar_raw);
-            bulk_g2s(sbase + RAW_W, Wg + e, row16, bar_raw);
+    // Bounded wait on an mbarrier phase; gives up early once another thread has aborted.
+    // One thread per group polls; the rest of the group parks on the group's named
+    // barrier (bar.red), which also carries the outcome and orders their later reads
+    // after the phase completed.  Polling by every thread would steal shared-memory and
+    // issue bandwidth from the other group.
+    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        for (uint32_t i = 0; i < kWaitLimit; ++i) {
+            if (mbar_try_wait(bar, parity)) return true;
+            if ((i & 255) == 255 && sAbort[0]) return false;
         }
-        if (vec_g) bulk_g2s(sbase + RAW_G, a.g + e, 2 * row16, bar_raw);
+        sAbort[0] = 1;
+        return false;
     };
+
+    // L2 prefetch of chunk c's inputs (issued by the state group's first thread)
     auto prefetch_inputs = [&](int c) {
         const int t0 = c * C, n = min(C, T - t0);
         const size_t e = (tok0 + t0) * DK;
@@ -228,195 +306,203 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         }
         if (vec_g) prefetch_l2(a.g + e, n * DK * 4);
     };
-    if (tid == 0) {
+
+    int raw_issued = 0, raw_done = 0;   // raw copies (WY group)
+    int mma_wy = 0, mma_st = 0;         // commits issued by each group's MMA thread
+
+    if (warp < 8) {
+        // ============================================================== WY group (0-7)
+        const int wtid = tid;   // 0 .. 255
+        // raw q, k, b, g_log of chunk c -> staging, one bulk copy per tensor, issued by
+        // lane 0 of warps 0-3 (issuing a bulk copy takes the issuing thread a while)
+        auto issue_raw = [&](int c) {
+            if (lane != 0 || warp >= 4) return;
+            const int t0 = c * C, n = min(C, T - t0);
+            const size_t e = (tok0 + t0) * DK;
+            const uint32_t row16 = (uint32_t)n * DK * 2;
+            fence_async_smem();
+            if (warp == 0) {
+                uint32_t bytes = 2 * row16;
+                if (gdn2) bytes += row16;
+                if (vec_g) bytes += 2 * row16;
+                mbar_arrive_expect_tx(bar_raw, bytes);
+                bulk_g2s(sbase + RAW_Q, Q + e, row16, bar_raw);
+            } else if (warp == 1) {
+                bulk_g2s(sbase + RAW_K, K + e, row16, bar_raw);
+            } else if (warp == 2) {
+                if (gdn2) bulk_g2s(sbase + RAW_B, Bg + e, row16, bar_raw);
+            } else if (vec_g) {
+                bulk_g2s(sbase + RAW_G, a.g + e, 2 * row16, bar_raw);
+            }
+        };
+        // Cumulative log-decay of chunk c by warps 4-7 (they run it while warps 0-3 invert
+        // the chunk before).  Waits for the chunk's raw inputs; thread (p, h) scans key
+        // channels 2p, 2p+1 over the quarters 2h, 2h+1 of the chunk (16 tokens each) in
+        // registers, then adds the totals of the earlier quarters.  Tokens past the end
+        // contribute zero.  Leaves gamma in place of the raw g_log, gamma_C, exp(gamma_C)
+        // and the exact-path flag; false if the wait failed.
+        auto scan = [&](int c) -> bool {
+            const int st = wtid - 128;   // 0 .. 127
+            const int t0 = c * C, n = min(C, T - t0);
+            if (!bar128_and(4, st != 0 || wait(bar_raw, (uint32_t)(c & 1)))) return false;
+            if (!vec_g) {
+                if (st < 64) sGs[st] = (st < n) ? a.g[tok0 + t0 + st] : 0.f;
+                bar128_sync(4);
+            }
+            const int sp = st & 63, h = st >> 6;
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const int q = 2 * h + qq;
+                float2 gv[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = q * 16 + i;
+                    if (vec_g) {
+                        gv[i] = *reinterpret_cast<const float2 *>(sGam + t * DK + 2 * sp);
+                    } else {
+                        const float x = sGs[t];
+                        gv[i] = make_float2(x, x);
+                    }
+                }
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const bool in = q * 16 + i < n;
+                    acc.x += in ? gv[i].x : 0.f;
+                    acc.y += in ? gv[i].y : 0.f;
+                    *reinterpret_cast<float2 *>(sGam + (q * 16 + i) * DK + 2 * sp) = acc;
+                }
+                reinterpret_cast<float2 *>(sTot)[q * 64 + sp] = acc;
+            }
+            bar128_sync(4);
+            bool big = false;
+#pragma unroll
+            for (int qq = 0; qq < 2; ++qq) {
+                const int q = 2 * h + qq;
+                float2 off = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int u = 0; u < 3; ++u) {
+                    if (u < q) {
+                        const float2 x = reinterpret_cast<const float2 *>(sTot)[u * 64 + sp];
+                        off.x += x.x;
+                        off.y += x.y;
+                    }
+                }
+                float2 gm = off;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float2 *gp = reinterpret_cast<float2 *>(sGam + (q * 16 + i) * DK + 2 * sp);
+                    gm = *gp;
+                    gm.x += off.x;
+                    gm.y += off.y;
+                    big |= fmaxf(fabsf(gm.x), fabsf(gm.y)) > kFastLimit;
+                    *gp = gm;
+                }
+                if (q == 3) {
+                    *reinterpret_cast<float2 *>(sGC + 2 * sp) = gm;
+                    *reinterpret_cast<float2 *>(sEGC + (c & 3) * 128 + 2 * sp) =
+                        make_float2(__expf(gm.x), __expf(gm.y));
+                }
+            }
+            const bool any = bar128_or(4, big);
+            if (st == 0) sExact[c & 3] = any ? 1 : 0;
+            return true;
+        };
         issue_raw(0);
-        if (nchunks > 1) prefetch_inputs(1);
-    }
-    int raw_issued = 1, raw_done = 0;   // uniform across the block
-
-    // the T tile's blocks above the diagonal are never written: zero the tile once
-    reinterpret_cast<uint4 *>(sm + OFF_T)[tid] = make_uint4(0, 0, 0, 0);
-    static_assert(kThreads * 16 == 8192, "one 16-byte store per thread clears the T tile");
-    // ---- initial state -> TMEM: fp32 S^T and its bf16 operand copy (warps 8-15) ----
-    if (warp >= 8) {
-        const int v = quarter * 32 + lane, dlo = ((warp - 8) >> 2) * 64;
-        for (int d0 = dlo; d0 < dlo + 64; d0 += 32) {
-            float x[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                x[j] = transfer ? (d0 + j == v ? 1.f : 0.f) : (S0p ? S0p[(size_t)(d0 + j) * DV + v] : 0.f);
-            tmem_st32(tmem + lane_base + TM_S + d0, x);
-            st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
-        }
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // Output rows and state update of the previous chunk (warps 8-15).  Runs while
-    // warps 0-7 build the next chunk's operands: that chunk's first MMA is the first
-    // reader of what is written here.
-    auto finish_chunk = [&](int t0p, int np, bool exactp, const float *egc, bool last) {
-        const int v = quarter * 32 + lane;
-        if (warp < 12) {
-            for (int t0c = 0; t0c < 64; t0c += 32) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_O + t0c, x);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (write_o && t0c + j < np) O[(tok0 + t0p + t0c + j) * DV + v] = __float2bfloat16_rn(x[j]);
+        raw_issued = 1;
+        bool ok = true, scan_ok = true;
+        if (warp >= 4) scan_ok = scan(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int t0 = c * C, n = min(C, T - t0);
+            const int pb = c & 1;   // P, T and Kb buffer of this chunk
+            // ---- W1: the scan of chunk c (warps 4-7) has finished ----
+            ok = group_and(BAR_WY, scan_ok);
+            if (!ok) break;
+            raw_done = c + 1;
+            const bool exact = sExact[c & 3] != 0;
+            // ---- W3: Kh and Qg are rebuilt once the state group has consumed those of
+            //      chunk c-1 (H3) ----
+            if (c > 0) {
+                ok = group_and(BAR_WY, wtid != 0 || wait(bar_h3, (uint32_t)((c - 1) & 1)));
+                if (!ok) break;
             }
-        } else {
-            for (int d0 = 0; d0 < DK; d0 += 32) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_S + d0, x);
-                tmem_wait_ld();
-                if (!exactp) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
-                    tmem_st32(tmem + lane_base + TM_S + d0, x);
-                }
-                st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
-                if (last && STp) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
-                }
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-    };
-
-    Waiter Wm{bar_mma, 0u}, Wr{bar_raw, 0u};
-    bool ok = true, exact_prev = false;
-    int t0_prev = 0, n_prev = 0;
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int t0 = c * C, n = min(C, T - t0);
-        float *egc = sEGC + (c & 1) * 128;
-        // ===== P1: cumulative log-decay, then operands =====
-        if (!Wr.all()) { ok = false; break; }
-        raw_done = c + 1;
-        if (tid == 0 && c + 2 < nchunks) prefetch_inputs(c + 2);
-        if (!vec_g) {
-            if (tid < 64) sGs[tid] = (tid < n) ? a.g[tok0 + t0 + tid] : 0.f;
-            __syncthreads();
-        }
-        // gamma: each thread scans 16 tokens of one key channel, then adds the totals of
-        // the earlier quarters of the chunk.  Tokens past the end contribute zero.
-        const int sd = tid & 127, sq = tid >> 7;
-        {
-            float acc = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = sq * 16 + i;
-                const float g = (t < n) ? (vec_g ? sGam[t * DK + sd] : sGs[t]) : 0.f;
-                acc += g;
-                sGam[t * DK + sd] = acc;
-            }
-            sTot[sq * 128 + sd] = acc;
-        }
-        __syncthreads();
-        bool big = false;
-        {
-            float off = 0.f;
-#pragma unroll
-            for (int u = 0; u < 3; ++u)
-                if (u < sq) off += sTot[u * 128 + sd];
-            float gm = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int t = sq * 16 + i;
-                gm = sGam[t * DK + sd] + off;
-                sGam[t * DK + sd] = gm;
-                big |= fabsf(gm) > kFastLimit;
-            }
-            if (sq == 3) {
-                sGC[sd] = gm;
-                egc[sd] = __expf(gm);
-            }
-        }
-        const bool exact = __syncthreads_or(big);   // also publishes gamma, gamma_C
-
-        {
-            // operands: thread (tg, cg) owns tokens 2 tg, 2 tg + 1, channels 8 cg .. 8 cg + 7
-            const int tg = tid >> 4, cg = tid & 15;
+            const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
+            {
+                // thread (tg, cg) owns tokens 4 tg .. 4 tg + 3, channels 8 cg .. 8 cg + 7
+                const int tg = wtid >> 4, cg = wtid & 15;
 #pragma unroll 1
-            for (int i = 0; i < 2; ++i) {
-                const int t = tg * 2 + i;
-                const bool in = t < n;
-                const uint32_t ro = (uint32_t)(t * DK * 2 + cg * 16);
-                const uint4 z = make_uint4(0, 0, 0, 0);
-                const uint4 uq = in ? *reinterpret_cast<const uint4 *>(sm + RAW_Q + ro) : z;
-                const uint4 uk = in ? *reinterpret_cast<const uint4 *>(sm + RAW_K + ro) : z;
-                const uint4 uv = in ? *reinterpret_cast<const uint4 *>(sm + RAW_V + ro) : z;
-                const float4 g0 = *reinterpret_cast<const float4 *>(sGam + t * DK + cg * 8);
-                const float4 g1 = *reinterpret_cast<const float4 *>(sGam + t * DK + cg * 8 + 4);
-                const float gam[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                float fq[8], fk[8], fv[8], fb[8], fw[8];
-                bf16x8_to_f32(uq, fq);
-                bf16x8_to_f32(uk, fk);
-                bf16x8_to_f32(uv, fv);
-                if (gdn2) {
-                    const uint4 ub = in ? *reinterpret_cast<const uint4 *>(sm + RAW_B + ro) : z;
-                    const uint4 uw = in ? *reinterpret_cast<const uint4 *>(sm + RAW_W + ro) : z;
-                    bf16x8_to_f32(ub, fb);
-                    bf16x8_to_f32(uw, fw);
-                } else {
-                    const float beta = in ? __bfloat162float(Bg[tok0 + t0 + t]) : 0.f;
+                for (int i = 0; i < 4; ++i) {
+                    const int t = tg * 4 + i;
+                    const bool in = t < n;
+                    const uint32_t ro = (uint32_t)(t * DK * 2 + cg * 16);
+                    const uint4 uq = sel(in, *reinterpret_cast<const uint4 *>(sm + RAW_Q + ro));
+                    const uint4 uk = sel(in, *reinterpret_cast<const uint4 *>(sm + RAW_K + ro));
+                    const float4 g0 = *reinterpret_cast<const float4 *>(sGam + t * DK + cg * 8);
+                    const float4 g1 = *reinterpret_cast<const float4 *>(sGam + t * DK + cg * 8 + 4);
+                    const float gm[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                    float fq[8], fk[8], fb[8];
+                    bf16x8_to_f32(uq, fq);
+                    bf16x8_to_f32(uk, fk);
+                    if (gdn2) {
+                        bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + RAW_B + ro)), fb);
+                    } else {
+                        const float bt = __bfloat162float(Bg[tok0 + t0 + min(t, n - 1)]);
+                        const float beta = in ? bt : 0.f;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) fb[j] = fw[j] = beta;
+                        for (int j = 0; j < 8; ++j) fb[j] = beta;
+                    }
+                    float kh[8], qg[8], kb[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float e = __expf(gm[j]);
+                        kh[j] = fb[j] * fk[j] * e;
+                        qg[j] = fq[j] * e;
+                    }
+                    if (exact) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(sGC[cg * 8 + j] - gm[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(-gm[j]);
+                    }
+                    st_chunk(sbase + OFF_QK + tile_chunk(128, t, cg), kh);
+                    st_chunk(sbase + OFF_QK + tile_chunk(128, 64 + t, cg), qg);
+                    st_chunk(kb_tile + tile_chunk(64, t, cg), kb);
                 }
-                float kh[8], qg[8], kb[8], wv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float e = __expf(gam[j]);
-                    kh[j] = fb[j] * fk[j] * e;
-                    qg[j] = fq[j] * e;
-                    wv[j] = transfer ? 0.f : fw[j] * fv[j];
-                }
-                if (exact) {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(sGC[cg * 8 + j] - gam[j]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(-gam[j]);
-                }
-                st_chunk(sbase + OFF_QK + tile_chunk(128, t, cg), kh);
-                st_chunk(sbase + OFF_QK + tile_chunk(128, 64 + t, cg), qg);
-                st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
-                st_chunk(sbase + OFF_WV + tile_chunk(64, t, cg), wv);
             }
-        }
-        fence_async_smem();
-        __syncthreads();
-
-        // ===== P2: [A;P] = [Kh;Qg] Kb^T | previous chunk's outputs and state (warps 8-15) =====
-        if (!exact && tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, false, false);
+            fence_async_smem();
+            group_sync(BAR_WY);
+            if (wtid == 0) mbar_arrive(bar_h1);   // H1: operands of chunk c built
+            // the raw inputs are dead on the fast path: the next chunk's travel from now on
+            if (!exact && c + 1 < nchunks) {
+                raw_issued = c + 2;
+                issue_raw(c + 1);
+            }
+            // ---- W4: [A; P] = [Kh; Qg] Kb^T ----
+            if (!exact) {
+                if (wtid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(128, 64, false, false, false);
 #pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s),
-                         desc_kmajor(sbase + OFF_KB, 64, 0, s), id, s > 0);
-            mma_commit(bar_mma);
-        }
-        if (warp >= 8 && c > 0)
-            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((c - 1) & 1) * 128, false);
-        if (!exact) {
-            if (!Wm.all()) { ok = false; break; }
-        } else {
-            tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-        }
-
-        // ===== P3: A (fp32, strictly lower) and P (bf16, lower incl.) =====
-        if (!exact) {
-            if (warp < 8) {
-                const int r = quarter * 32 + lane, j0 = (warp >> 2) * 32;   // row of [A; P], columns
+                    for (int s = 0; s < DK / 16; ++s)
+                        mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s),
+                                 desc_kmajor(kb_tile, 64, 0, s), id, s > 0);
+                    mma_commit(bar_wy);
+                }
+                ++mma_wy;
+                ok = group_and(BAR_WY, wtid != 0 || wait(bar_wy, (uint32_t)((mma_wy - 1) & 1)));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            // ---- W5: this chunk's P and T buffers were chunk c-2's: wait until it finished ----
+            if (c > 1) {
+                ok = group_and(BAR_WY, wtid != 0 || wait(bar_h4 + 8 * pb, (uint32_t)(((c - 2) >> 1) & 1)));
+                if (!ok) break;
+            }
+            const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
+            // ---- W6: A (fp32, strictly lower) and P (bf16, lower incl.) ----
+            if (!exact) {
+                const int r = quarter * 32 + lane, j0 = (warp >> 2) * 32;   // row of [A; P]
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_AP + j0, x);
                 tmem_wait_ld();
@@ -436,164 +522,228 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                         float f[8];
 #pragma unroll
                         for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
-                        st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+                        st_chunk(p_tile + tile_chunk(64, t, j0 / 8 + h), f);
                     }
                 }
-            }
-        } else {
-            // exact per-pair decays (strong-decay chunks only), from the staged raw inputs
-            float av[8], pv[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int p = tid + u * kThreads, i = p >> 6, j = p & 63;
-                float sa = 0.f, sp = 0.f;
-                if (j <= i && i < n) {
-                    const __nv_bfloat16 *qi = (const __nv_bfloat16 *)(sm + RAW_Q) + i * DK;
-                    const __nv_bfloat16 *ki = (const __nv_bfloat16 *)(sm + RAW_K) + i * DK;
-                    const __nv_bfloat16 *kj = (const __nv_bfloat16 *)(sm + RAW_K) + j * DK;
-                    const __nv_bfloat16 *bi = (const __nv_bfloat16 *)(sm + RAW_B) + i * DK;
-                    const float bs = gdn2 ? 0.f : __bfloat162float(Bg[tok0 + t0 + i]);
-                    for (int d = 0; d < DK; ++d) {
-                        const float dec = __expf(sGam[i * DK + d] - sGam[j * DK + d]);
-                        const float kjd = __bfloat162float(kj[d]) * dec;
-                        const float bid = gdn2 ? __bfloat162float(bi[d]) : bs;
-                        sa = fmaf(bid * __bfloat162float(ki[d]), kjd, sa);
-                        sp = fmaf(__bfloat162float(qi[d]), kjd, sp);
+            } else {
+                // exact per-pair decays (strong-decay chunks only), from the staged raw inputs
+#pragma unroll 1
+                for (int u = 0; u < 16; ++u) {
+                    const int p = wtid + u * 256, i = p >> 6, j = p & 63;
+                    float sa = 0.f, sp2 = 0.f;
+                    if (j <= i && i < n) {
+                        const __nv_bfloat16 *qi = (const __nv_bfloat16 *)(sm + RAW_Q) + i * DK;
+                        const __nv_bfloat16 *ki = (const __nv_bfloat16 *)(sm + RAW_K) + i * DK;
+                        const __nv_bfloat16 *kj = (const __nv_bfloat16 *)(sm + RAW_K) + j * DK;
+                        const __nv_bfloat16 *bi = (const __nv_bfloat16 *)(sm + RAW_B) + i * DK;
+                        const float bs = gdn2 ? 0.f : __bfloat162float(Bg[tok0 + t0 + i]);
+                        for (int d = 0; d < DK; ++d) {
+                            const float dec = __expf(sGam[i * DK + d] - sGam[j * DK + d]);
+                            const float kjd = __bfloat162float(kj[d]) * dec;
+                            const float bid = gdn2 ? __bfloat162float(bi[d]) : bs;
+                            sa = fmaf(bid * __bfloat162float(ki[d]), kjd, sa);
+                            sp2 = fmaf(__bfloat162float(qi[d]), kjd, sp2);
+                        }
                     }
+                    sA32[i * kAS + j] = (j < i) ? sa : 0.f;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + (p_tile - sbase) + tile_off(64, i, j)) =
+                        __float2bfloat16_rn(sp2);
                 }
-                av[u] = (j < i) ? sa : 0.f;
-                pv[u] = sp;
             }
-            __syncthreads();   // raw b is read above and overlaps the A scratch
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int p = tid + u * kThreads, i = p >> 6, j = p & 63;
-                sA32[i * kAS + j] = av[u];
-                *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_P + tile_off(64, i, j)) = __float2bfloat16_rn(pv[u]);
+            group_sync(BAR_WY);
+            if (exact && c + 1 < nchunks) {   // raw inputs read above: now the next chunk's
+                raw_issued = c + 2;
+                issue_raw(c + 1);
+            }
+            // ---- W7: T = (I + A)^-1 by warps 0-3, straight into the bf16 tile, while
+            //      warps 4-7 scan the next chunk's log-decay ----
+            if (warp < 4) {
+                tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{}, TileOut{t_tile});
+                fence_async_smem();
+                Bar128{}();
+                if (wtid == 0) mbar_arrive(bar_h2 + 8 * pb);   // H2: T and P of chunk c ready
+            } else if (c + 1 < nchunks) {
+                scan_ok = scan(c + 1);
             }
         }
-        __syncthreads();
-
-        // ===== P4: T = (I + A)^-1 =====
-        if (warp < 4) tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // the staging area is free again: the next chunk's raw inputs travel from now on
-        if (c + 1 < nchunks) {
-            raw_issued = c + 2;
-            if (tid == 0) issue_raw(c + 1);
-        }
-
-        // ===== P5: W^T = Kh^T T^T,  U^T = WV^T T^T,  O^T = S^T Qg^T =====
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, true, false, false);
-#pragma unroll
-            for (int s = 0; s < C / 16; ++s) {
-                mma_bf16(tmem + TM_W, desc_mnmajor(sbase + OFF_QK, 128, 0, s),
-                         desc_kmajor(sbase + OFF_T, 64, 0, s), id, s > 0);
-                mma_bf16(tmem + TM_E, desc_mnmajor(sbase + OFF_WV, 64, 0, s),
-                         desc_kmajor(sbase + OFF_T, 64, 0, s), id, s > 0);
-            }
-            const uint32_t ido = idesc_bf16(128, 64, false, false, false);
-#pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                mma_bf16_ts(tmem + TM_O, tmem + TM_SB + s * 8, desc_kmajor(sbase + OFF_QK, 128, 64, s),
-                            ido, s > 0);
-            mma_commit(bar_mma);
-        }
-        if (!Wm.all()) { ok = false; break; }
-
-        // ===== P6: W^T -> bf16 operand (MN-major B); exact chunks pre-scale the state =====
-        if (warp < 8) {
-            const int d = quarter * 32 + lane, t0c = (warp >> 2) * 32;
+        if (!ok) sAbort[0] = 1;
+    } else {
+        // =========================================================== state group (8-15)
+        const int stid = tid - 256;   // 0 .. 255
+        const int half = (warp - 8) >> 2;
+        const int v = quarter * 32 + lane;   // value channel = TMEM lane
+        const int j0 = half * 32;            // this thread's token columns of X, E and O
+        bool ok = true;
+        // initial state -> TMEM: fp32 S^T and its bf16 operand copy
+        for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
             float x[32];
-            tmem_ld32(tmem + lane_base + TM_W + t0c, x);
-            tmem_wait_ld();
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                float f[8];
+            for (int j = 0; j < 32; ++j)
+                x[j] = transfer ? (d0 + j == v ? 1.f : 0.f) : (S0p ? S0p[(size_t)(d0 + j) * DV + v] : 0.f);
+            tmem_st32(tmem + lane_base + TM_S + d0, x);
+            st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
+        }
+        if (stid == 0 && nchunks > 1) prefetch_inputs(1);
+        tmem_wait_st();
+        tc_fence_before();
+        group_sync(BAR_ST);
+        for (int c = 0; c < nchunks; ++c) {
+            const int t0 = c * C, n = min(C, T - t0);
+            const int pb = c & 1;
+            const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
+            const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
+            const float *egc = sEGC + (c & 3) * 128;
+            // (w.v)^T for this thread's lane and token columns, read from global memory
+            // before the wait for the operands.  Rows past the end are clamped to the last
+            // row (so every load is in bounds and none is conditional) and give zero.
+            float wvt[32];
+            {
+                __nv_bfloat16 vv[32], ww[32];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = x[q8 * 8 + j];
-                st_chunk(sbase + OFF_WT + tile_chunk(128, d, t0c / 8 + q8), f);
+                for (int j = 0; j < 32; ++j) {
+                    const int t = min(j0 + j, n - 1);
+                    const size_t ej = (tok0 + t0 + t) * DV + v;
+                    vv[j] = V[ej];
+                    ww[j] = gdn2 ? Wg[ej] : Bg[tok0 + t0 + t];
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const bool in = j0 + j < n && !transfer;
+                    wvt[j] = in ? __bfloat162float(ww[j]) * __bfloat162float(vv[j]) : 0.f;
+                }
             }
-        } else if (exact) {
-            const int dlo = ((warp - 8) >> 2) * 64;
-            for (int d0 = dlo; d0 < dlo + 64; d0 += 32) {
+            // ---- S1: operands of chunk c (H1); [X | O] = S^T [Kh; Qg]^T ----
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_h1, (uint32_t)(c & 1)));
+            if (!ok) break;
+            const bool exact = sExact[c & 3] != 0;
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128, false, false, false);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    mma_bf16_ts(tmem + TM_XO, tmem + TM_SB + s * 8, desc_kmajor(sbase + OFF_QK, 128, 0, s),
+                                id, s > 0);
+                mma_commit(bar_st);
+                if (c + 2 < nchunks) prefetch_inputs(c + 2);
+            }
+            ++mma_st;
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            // ---- S2: R^T = (w.v)^T - X -> bf16 in TMEM; exact chunks pre-scale S ----
+            {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_XO + j0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) x[j] = wvt[j] - x[j];
+                st_tmem_bf16(tmem + lane_base + TM_XB + j0 / 2, x);
+            }
+            if (exact) {
+                // strong-decay chunk: the state is scaled before its update
+                for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_base + TM_S + d0, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
+                    tmem_st32(tmem + lane_base + TM_S + d0, x);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            group_sync(BAR_ST);
+            if (stid == 0) mbar_arrive(bar_h3);   // H3: Kh, Qg of chunk c consumed
+            // ---- S3: T and P of chunk c (H2); E^T = R^T T^T ----
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_h2 + 8 * pb, (uint32_t)((c >> 1) & 1)));
+            if (!ok) break;
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)
+                    mma_bf16_ts(tmem + TM_XO, tmem + TM_XB + s * 8, desc_kmajor(t_tile, 64, 0, s), id, s > 0);
+                mma_commit(bar_st);
+            }
+            ++mma_st;
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            // ---- S4: E^T -> bf16 in TMEM ----
+            {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_XO + j0, x);
+                tmem_wait_ld();
+                st_tmem_bf16(tmem + lane_base + TM_XB + j0 / 2, x);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            group_sync(BAR_ST);
+            // ---- S5: O^T += E^T P^T,  S^T += E^T Kb (or K_end) ----
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t ido = idesc_bf16(128, 64, false, false, false);
+                const uint32_t ids = idesc_bf16(128, 128, false, true, false);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s) {
+                    mma_bf16_ts(tmem + TM_XO + 64, tmem + TM_XB + s * 8, desc_kmajor(p_tile, 64, 0, s), ido, 1u);
+                    mma_bf16_ts(tmem + TM_S, tmem + TM_XB + s * 8, desc_mnmajor(kb_tile, 64, 0, s), ids, 1u);
+                }
+                mma_commit(bar_st);
+            }
+            ++mma_st;
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            // ---- S6: output rows [j0, j0 + 32); state columns [64 half, +64) scaled, kept
+            //      in fp32 and as the bf16 operand ----
+            {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_XO + 64 + j0, x);
+                tmem_wait_ld();
+                if (write_o) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (j0 + j < n) O[(tok0 + t0 + j0 + j) * DV + v] = __float2bfloat16_rn(x[j]);
+                }
+            }
+            const bool last = (c == nchunks - 1);
+            for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_S + d0, x);
                 tmem_wait_ld();
+                if (!exact) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
-                tmem_st32(tmem + lane_base + TM_S + d0, x);
+                    for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
+                    tmem_st32(tmem + lane_base + TM_S + d0, x);
+                }
+                st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
+                if (last && STp) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
+                }
             }
             tmem_wait_st();
+            tc_fence_before();
+            group_sync(BAR_ST);
+            if (stid == 0) mbar_arrive(bar_h4 + 8 * pb);   // H4: chunk c finished
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ===== P7: E^T = U^T - S^T W^T =====
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id = idesc_bf16(128, 64, false, true, true);
-#pragma unroll
-            for (int s = 0; s < DK / 16; ++s)
-                mma_bf16_ts(tmem + TM_E, tmem + TM_SB + s * 8, desc_mnmajor(sbase + OFF_WT, 128, 0, s),
-                            id, 1u);
-            mma_commit(bar_mma);
-        }
-        if (!Wm.all()) { ok = false; break; }
-
-        // ===== P8: E^T -> bf16 operand in TMEM =====
-        {
-            const int t0c = (warp >> 2) * 16;
-            float x[16];
-            tmem_ld16(tmem + lane_base + TM_E + t0c, x);
-            tmem_wait_ld();
-            uint32_t pk[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) pk[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
-            tmem_st8(tmem + lane_base + TM_EB + t0c / 2, pk);
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ===== P9: O^T += E^T P^T,  S^T += E^T Kb (or K_end) =====
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t ido = idesc_bf16(128, 64, false, false, false);
-            const uint32_t ids = idesc_bf16(128, 128, false, true, false);
-#pragma unroll
-            for (int s = 0; s < C / 16; ++s) {
-                mma_bf16_ts(tmem + TM_O, tmem + TM_EB + s * 8, desc_kmajor(sbase + OFF_P, 64, 0, s),
-                            ido, 1u);
-                mma_bf16_ts(tmem + TM_S, tmem + TM_EB + s * 8, desc_mnmajor(sbase + OFF_KB, 64, 0, s),
-                            ids, 1u);
-            }
-            mma_commit(bar_mma);
-        }
-        if (!Wm.all()) { ok = false; break; }
-        exact_prev = exact;
-        t0_prev = t0;
-        n_prev = n;
+        if (!ok) sAbort[0] = 1;
     }
 
-    if (ok && nchunks > 0) {
-        // ===== P10 of the last chunk: output rows, final state =====
-        if (warp >= 8)
-            finish_chunk(t0_prev, n_prev, exact_prev, sEGC + ((nchunks - 1) & 1) * 128, true);
-        tc_fence_before();
-        __syncthreads();
-    }
-    if (!ok) {
-        if (tid == 0) atomicExch(&g_tc_error, 1);
-        // drain: committed tensor-core work and an outstanding raw copy (bounded waits)
-        if (tid == 0) mma_commit(bar_mma);
-        mbar_wait(bar_mma, Wm.phase, kWaitLimit);
-        if (raw_issued > raw_done) mbar_wait(bar_raw, (uint32_t)(raw_done & 1), kWaitLimit);
+    __syncthreads();
+    if (sAbort[0]) {
+        // drain: committed tensor-core work of both groups and an outstanding raw copy
+        if (tid == 0) {
+            atomicExch(&g_tc_error, 1);
+            mma_commit(bar_wy);
+            drain_commits(bar_wy, mma_wy + 1);
+            if (raw_issued > raw_done) mbar_wait(bar_raw, (uint32_t)(raw_done & 1), kWaitLimit);
+        }
+        if (tid == 256) {
+            mma_commit(bar_st);
+            drain_commits(bar_st, mma_st + 1);
+        }
     }
     __syncthreads();
     tc_fence_after();
