@@ -72,8 +72,7 @@ constexpr int OFF_QK = (OFF_X + 4 * 16 * tri::XLD * 4 + 1023) / 1024 * 1024;
 constexpr int OFF_KB = OFF_QK + 32768;          // Kb bf16 [2][64 t][128 d] 32 KB
 constexpr int OFF_P = OFF_KB + 32768;           // P  bf16 [2][64 t][64 j]  16 KB
 constexpr int OFF_T = OFF_P + 16384;            // T  bf16 [2][64 t][64 j]  16 KB
-constexpr int OFF_TOT = OFF_T + 16384;          // scan: quarter totals fp32 [4][128]
-constexpr int OFF_GS = OFF_TOT + 2048;          // scalar g_log of the chunk (GDN) fp32 [64]
+constexpr int OFF_GS = OFF_T + 16384;           // scalar g_log of the chunk (GDN) fp32 [64]
 constexpr int OFF_GC = OFF_GS + 256;            // gamma_C fp32 [128]
 constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [4][128], slot c % 4
 constexpr int OFF_FLAG = OFF_EGC + 2048;        // exact flags [4] (slot c % 4), abort flag
@@ -101,6 +100,13 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
         f[2 * i] = x.x;
         f[2 * i + 1] = x.y;
     }
+}
+
+// 1/x to within an ulp or two (PTX rcp.approx); x is a normal number here
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 // v where in, else zero (a staged row past the end of the input holds stale data)
@@ -207,6 +213,64 @@ __device__ __forceinline__ void drain_commits(uint32_t bar, int n) {
     if (n >= 1) mbar_wait(bar, (uint32_t)((n - 1) & 1), kWaitLimit);
 }
 
+// Exact path, strong-decay chunks only: A (fp32, strictly lower) and P (bf16 tile, lower
+// incl.) from per-pair decays exp(gamma_i - gamma_j), computed from the staged raw q, k, b
+// and gamma on CUDA cores by the 256 threads of the WY group.  beta: the scalar b of the
+// chunk's tokens (tied modes), or NULL when b is a per-channel vector staged with q and k.
+// Kept out of line: it is rarely run and would otherwise crowd the instruction cache.
+__device__ __noinline__ void exact_ap(unsigned char *sm, float *sA32, uint32_t p_off, const float *sGam,
+                                      const __nv_bfloat16 *beta, int n, int wtid) {
+#pragma unroll 1
+    for (int u = 0; u < 16; ++u) {
+        const int p = wtid + u * 256, i = p >> 6, j = p & 63;
+        float sa = 0.f, sp = 0.f;
+        if (j <= i && i < n) {
+            const __nv_bfloat16 *qi = (const __nv_bfloat16 *)(sm + RAW_Q) + i * DK;
+            const __nv_bfloat16 *ki = (const __nv_bfloat16 *)(sm + RAW_K) + i * DK;
+            const __nv_bfloat16 *kj = (const __nv_bfloat16 *)(sm + RAW_K) + j * DK;
+            const __nv_bfloat16 *bi = (const __nv_bfloat16 *)(sm + RAW_B) + i * DK;
+            const float bs = beta ? __bfloat162float(beta[i]) : 0.f;
+#pragma unroll 2
+            for (int d = 0; d < DK; ++d) {
+                const float dec = __expf(sGam[i * DK + d] - sGam[j * DK + d]);
+                const float kjd = __bfloat162float(kj[d]) * dec;
+                const float bid = beta ? bs : __bfloat162float(bi[d]);
+                sa = fmaf(bid * __bfloat162float(ki[d]), kjd, sa);
+                sp = fmaf(__bfloat162float(qi[d]), kjd, sp);
+            }
+        }
+        sA32[i * kAS + j] = (j < i) ? sa : 0.f;
+        *reinterpret_cast<__nv_bfloat16 *>(sm + p_off + tile_off(64, i, j)) = __float2bfloat16_rn(sp);
+    }
+}
+
+// Exact path: gamma of key channel d over the chunk's n tokens (zero contribution past the
+// end) from the g_log in global memory, stride apart, into column d of the gamma tile
+// (strong-decay chunks only; out of line like exact_ap).
+__device__ __noinline__ void exact_gamma(float *sGam, const float *g, int stride, int n, int d) {
+    float acc = 0.f;
+#pragma unroll 1
+    for (int t = 0; t < C; ++t) {
+        if (t < n) acc += g[(size_t)t * stride];
+        sGam[t * DK + d] = acc;
+    }
+}
+
+// Exact path: S^T columns [d_begin, d_begin + 64) scaled by exp(gamma_C) in TMEM, before the
+// state update (strong-decay chunks only; out of line like exact_ap).
+__device__ __noinline__ void prescale_state(uint32_t taddr, const float *egc, int d_begin) {
+#pragma unroll 1
+    for (int d0 = d_begin; d0 < d_begin + 64; d0 += 32) {
+        float x[32];
+        tmem_ld32(taddr + d0, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
+        tmem_st32(taddr + d0, x);
+    }
+    tmem_wait_st();
+}
+
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -241,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     float *sT32 = reinterpret_cast<float *>(sm + OFF_T32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
     float *sGam = reinterpret_cast<float *>(sm + RAW_G);
-    float *sTot = reinterpret_cast<float *>(sm + OFF_TOT);
     float *sGs = reinterpret_cast<float *>(sm + OFF_GS);
     float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
     float *sEGC = reinterpret_cast<float *>(sm + OFF_EGC);
@@ -336,96 +399,55 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             }
         };
         // Cumulative log-decay of chunk c by warps 4-7 (they run it while warps 0-3 invert
-        // the chunk before).  Waits for the chunk's raw inputs; thread (p, h) scans key
-        // channels 2p, 2p+1 over the quarters 2h, 2h+1 of the chunk (16 tokens each) in
-        // registers, then adds the totals of the earlier quarters.  Tokens past the end
-        // contribute zero.  Leaves gamma in place of the raw g_log, gamma_C, exp(gamma_C)
-        // and the exact-path flag; false if the wait failed.
+        // the chunk before).  Waits for the chunk's raw inputs; thread d scans key channel d
+        // (tokens past the end contribute zero) and leaves e^gamma in place of the raw g_log.
+        // A chunk with |gamma| > 60 somewhere takes the exact path, which needs gamma itself:
+        // then the scan is redone from the g_log in global memory (rare).  Also writes
+        // gamma_C, exp(gamma_C) and the exact-path flag.  False if the wait failed.
         auto scan = [&](int c) -> bool {
-            const int st = wtid - 128;   // 0 .. 127
+            const int d = wtid - 128;   // 0 .. 127
             const int t0 = c * C, n = min(C, T - t0);
-            if (!bar128_and(4, st != 0 || wait(bar_raw, (uint32_t)(c & 1)))) return false;
+            if (!bar128_and(4, d != 0 || wait(bar_raw, (uint32_t)(c & 1)))) return false;
             if (!vec_g) {
-                if (st < 64) sGs[st] = (st < n) ? a.g[tok0 + t0 + st] : 0.f;
+                if (d < 64) sGs[d] = (d < n) ? a.g[tok0 + t0 + d] : 0.f;
                 bar128_sync(4);
             }
-            const int sp = st & 63, h = st >> 6;
+            float acc = 0.f, mx = 0.f;
+#pragma unroll 1
+            for (int b = 0; b < C; b += 16) {
+                float x[16];
 #pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const int q = 2 * h + qq;
-                float2 gv[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int t = q * 16 + i;
-                    if (vec_g) {
-                        gv[i] = *reinterpret_cast<const float2 *>(sGam + t * DK + 2 * sp);
-                    } else {
-                        const float x = sGs[t];
-                        gv[i] = make_float2(x, x);
-                    }
-                }
-                float2 acc = make_float2(0.f, 0.f);
+                for (int i = 0; i < 16; ++i) x[i] = vec_g ? sGam[(b + i) * DK + d] : sGs[b + i];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const bool in = q * 16 + i < n;
-                    acc.x += in ? gv[i].x : 0.f;
-                    acc.y += in ? gv[i].y : 0.f;
-                    *reinterpret_cast<float2 *>(sGam + (q * 16 + i) * DK + 2 * sp) = acc;
+                    acc += (b + i < n) ? x[i] : 0.f;
+                    mx = fmaxf(mx, fabsf(acc));
+                    x[i] = __expf(acc);
                 }
-                reinterpret_cast<float2 *>(sTot)[q * 64 + sp] = acc;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sGam[(b + i) * DK + d] = x[i];
             }
-            bar128_sync(4);
-            bool big = false;
-#pragma unroll
-            for (int qq = 0; qq < 2; ++qq) {
-                const int q = 2 * h + qq;
-                float2 off = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int u = 0; u < 3; ++u) {
-                    if (u < q) {
-                        const float2 x = reinterpret_cast<const float2 *>(sTot)[u * 64 + sp];
-                        off.x += x.x;
-                        off.y += x.y;
-                    }
-                }
-                float2 gm = off;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float2 *gp = reinterpret_cast<float2 *>(sGam + (q * 16 + i) * DK + 2 * sp);
-                    gm = *gp;
-                    gm.x += off.x;
-                    gm.y += off.y;
-                    big |= fmaxf(fabsf(gm.x), fabsf(gm.y)) > kFastLimit;
-                    *gp = gm;
-                }
-                if (q == 3) {
-                    *reinterpret_cast<float2 *>(sGC + 2 * sp) = gm;
-                    *reinterpret_cast<float2 *>(sEGC + (c & 3) * 128 + 2 * sp) =
-                        make_float2(__expf(gm.x), __expf(gm.y));
-                }
-            }
-            const bool any = bar128_or(4, big);
-            if (st == 0) sExact[c & 3] = any ? 1 : 0;
+            const bool any = bar128_or(4, mx > kFastLimit);
+            if (any) exact_gamma(sGam, vec_g ? a.g + (tok0 + t0) * DK + d : a.g + tok0 + t0, vec_g ? DK : 1, n, d);
+            sGC[d] = acc;
+            sEGC[(c & 3) * 128 + d] = __expf(acc);
+            if (d == 0) sExact[c & 3] = any ? 1 : 0;
             return true;
         };
         issue_raw(0);
         raw_issued = 1;
         bool ok = true, scan_ok = true;
-        if (warp >= 4) scan_ok = scan(0);
-        for (int c = 0; c < nchunks; ++c) {
+        // iteration c = -1 only scans chunk 0 (one call site keeps one copy of the scan)
+        for (int c = -1; c < nchunks; ++c) {
+          if (c >= 0) {
             const int t0 = c * C, n = min(C, T - t0);
             const int pb = c & 1;   // P, T and Kb buffer of this chunk
-            // ---- W1: the scan of chunk c (warps 4-7) has finished ----
-            ok = group_and(BAR_WY, scan_ok);
+            // ---- W1: the scan of chunk c (warps 4-7) has finished, and the state group has
+            //      consumed Kh and Qg of chunk c-1 (H3), so they may be rebuilt ----
+            ok = group_and(BAR_WY, scan_ok && (c == 0 || wtid != 0 || wait(bar_h3, (uint32_t)((c - 1) & 1))));
             if (!ok) break;
             raw_done = c + 1;
             const bool exact = sExact[c & 3] != 0;
-            // ---- W3: Kh and Qg are rebuilt once the state group has consumed those of
-            //      chunk c-1 (H3) ----
-            if (c > 0) {
-                ok = group_and(BAR_WY, wtid != 0 || wait(bar_h3, (uint32_t)((c - 1) & 1)));
-                if (!ok) break;
-            }
             const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
             {
                 // thread (tg, cg) owns tokens 4 tg .. 4 tg + 3, channels 8 cg .. 8 cg + 7
@@ -451,19 +473,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
 #pragma unroll
                         for (int j = 0; j < 8; ++j) fb[j] = beta;
                     }
+                    // gm holds e^gamma on the fast path, gamma on the exact path
                     float kh[8], qg[8], kb[8];
+                    if (!exact) {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float e = __expf(gm[j]);
-                        kh[j] = fb[j] * fk[j] * e;
-                        qg[j] = fq[j] * e;
-                    }
-                    if (exact) {
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(sGC[cg * 8 + j] - gm[j]);
+                        for (int j = 0; j < 8; ++j) {
+                            kh[j] = fb[j] * fk[j] * gm[j];
+                            qg[j] = fq[j] * gm[j];
+                            kb[j] = fk[j] * rcp_approx(gm[j]);
+                        }
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) kb[j] = fk[j] * __expf(-gm[j]);
+                        for (int j = 0; j < 8; ++j) {
+                            const float e = __expf(gm[j]);
+                            kh[j] = fb[j] * fk[j] * e;
+                            qg[j] = fq[j] * e;
+                            kb[j] = fk[j] * __expf(sGC[cg * 8 + j] - gm[j]);
+                        }
                     }
                     st_chunk(sbase + OFF_QK + tile_chunk(128, t, cg), kh);
                     st_chunk(sbase + OFF_QK + tile_chunk(128, 64 + t, cg), qg);
@@ -478,7 +504,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 raw_issued = c + 2;
                 issue_raw(c + 1);
             }
-            // ---- W4: [A; P] = [Kh; Qg] Kb^T ----
+            // ---- W4: [A; P] = [Kh; Qg] Kb^T; this chunk's P and T buffers were chunk c-2's,
+            //      so that chunk must have finished (H4) ----
             if (!exact) {
                 if (wtid == 0) {
                     tc_fence_after();
@@ -490,15 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     mma_commit(bar_wy);
                 }
                 ++mma_wy;
-                ok = group_and(BAR_WY, wtid != 0 || wait(bar_wy, (uint32_t)((mma_wy - 1) & 1)));
-                if (!ok) break;
-                tc_fence_after();
             }
-            // ---- W5: this chunk's P and T buffers were chunk c-2's: wait until it finished ----
-            if (c > 1) {
-                ok = group_and(BAR_WY, wtid != 0 || wait(bar_h4 + 8 * pb, (uint32_t)(((c - 2) >> 1) & 1)));
-                if (!ok) break;
-            }
+            ok = group_and(BAR_WY, wtid != 0 ||
+                                       ((exact || wait(bar_wy, (uint32_t)((mma_wy - 1) & 1))) &&
+                                        (c < 2 || wait(bar_h4 + 8 * pb, (uint32_t)(((c - 2) >> 1) & 1)))));
+            if (!ok) break;
+            tc_fence_after();
             const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
             // ---- W6: A (fp32, strictly lower) and P (bf16, lower incl.) ----
             if (!exact) {
@@ -526,29 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     }
                 }
             } else {
-                // exact per-pair decays (strong-decay chunks only), from the staged raw inputs
-#pragma unroll 1
-                for (int u = 0; u < 16; ++u) {
-                    const int p = wtid + u * 256, i = p >> 6, j = p & 63;
-                    float sa = 0.f, sp2 = 0.f;
-                    if (j <= i && i < n) {
-                        const __nv_bfloat16 *qi = (const __nv_bfloat16 *)(sm + RAW_Q) + i * DK;
-                        const __nv_bfloat16 *ki = (const __nv_bfloat16 *)(sm + RAW_K) + i * DK;
-                        const __nv_bfloat16 *kj = (const __nv_bfloat16 *)(sm + RAW_K) + j * DK;
-                        const __nv_bfloat16 *bi = (const __nv_bfloat16 *)(sm + RAW_B) + i * DK;
-                        const float bs = gdn2 ? 0.f : __bfloat162float(Bg[tok0 + t0 + i]);
-                        for (int d = 0; d < DK; ++d) {
-                            const float dec = __expf(sGam[i * DK + d] - sGam[j * DK + d]);
-                            const float kjd = __bfloat162float(kj[d]) * dec;
-                            const float bid = gdn2 ? __bfloat162float(bi[d]) : bs;
-                            sa = fmaf(bid * __bfloat162float(ki[d]), kjd, sa);
-                            sp2 = fmaf(__bfloat162float(qi[d]), kjd, sp2);
-                        }
-                    }
-                    sA32[i * kAS + j] = (j < i) ? sa : 0.f;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + (p_tile - sbase) + tile_off(64, i, j)) =
-                        __float2bfloat16_rn(sp2);
-                }
+                exact_ap(sm, sA32, p_tile - sbase, sGam, gdn2 ? nullptr : Bg + tok0 + t0, n, wtid);
             }
             group_sync(BAR_WY);
             if (exact && c + 1 < nchunks) {   // raw inputs read above: now the next chunk's
@@ -562,9 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 fence_async_smem();
                 Bar128{}();
                 if (wtid == 0) mbar_arrive(bar_h2 + 8 * pb);   // H2: T and P of chunk c ready
-            } else if (c + 1 < nchunks) {
-                scan_ok = scan(c + 1);
             }
+          }
+          if (warp >= 4 && c + 1 < nchunks) scan_ok = scan(c + 1);
         }
         if (!ok) sAbort[0] = 1;
     } else {
@@ -594,22 +596,39 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
             const float *egc = sEGC + (c & 3) * 128;
             // (w.v)^T for this thread's lane and token columns, read from global memory
-            // before the wait for the operands.  Rows past the end are clamped to the last
-            // row (so every load is in bounds and none is conditional) and give zero.
+            // before the wait for the operands; tokens past the end give zero
             float wvt[32];
             {
-                __nv_bfloat16 vv[32], ww[32];
+                const int last = transfer ? -1 : min(31, n - 1 - j0);   // last token column in range
+                const __nv_bfloat16 *vp = V + (tok0 + t0 + j0) * DV + v;
+                const __nv_bfloat16 *wp = gdn2 ? Wg + (tok0 + t0 + j0) * DV + v : Bg + tok0 + t0 + j0;
+                const int ws = gdn2 ? DV : 1;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int t = min(j0 + j, n - 1);
-                    const size_t ej = (tok0 + t0 + t) * DV + v;
-                    vv[j] = V[ej];
-                    ww[j] = gdn2 ? Wg[ej] : Bg[tok0 + t0 + t];
-                }
+                for (int h = 0; h < 32; h += 16) {   // two halves of 16 columns bound the registers
+                    __nv_bfloat16 vv[16], ww[16];
+                    if (last == 31) {
+                        // whole columns: fixed offsets from one base address, all loads in flight
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const bool in = j0 + j < n && !transfer;
-                    wvt[j] = in ? __bfloat162float(ww[j]) * __bfloat162float(vv[j]) : 0.f;
+                        for (int j = 0; j < 16; ++j) {
+                            vv[j] = vp[(h + j) * DV];
+                            ww[j] = wp[(h + j) * ws];
+                        }
+                    } else if (last >= 0) {
+                        // ragged end: rows past the end re-read the last row and give zero
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jj = min(h + j, last);
+                            vv[j] = vp[jj * DV];
+                            ww[j] = wp[jj * ws];
+                        }
+                    } else {
+                        // no row of these columns is in range (or a transition-matrix run)
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) vv[j] = ww[j] = __float2bfloat16_rn(0.f);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        wvt[h + j] = (h + j <= last) ? __bfloat162float(ww[j]) * __bfloat162float(vv[j]) : 0.f;
                 }
             }
             // ---- S1: operands of chunk c (H1); [X | O] = S^T [Kh; Qg]^T ----
@@ -639,17 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 for (int j = 0; j < 32; ++j) x[j] = wvt[j] - x[j];
                 st_tmem_bf16(tmem + lane_base + TM_XB + j0 / 2, x);
             }
-            if (exact) {
-                // strong-decay chunk: the state is scaled before its update
-                for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
-                    float x[32];
-                    tmem_ld32(tmem + lane_base + TM_S + d0, x);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) x[j] *= egc[d0 + j];
-                    tmem_st32(tmem + lane_base + TM_S + d0, x);
-                }
-            }
+            if (exact) prescale_state(tmem + lane_base + TM_S, egc, half * 64);   // strong decay
             tmem_wait_st();
             tc_fence_before();
             group_sync(BAR_ST);
