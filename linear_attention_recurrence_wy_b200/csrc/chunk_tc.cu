@@ -711,12 +711,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 tmem_ld32(tmem + lane_base + TM_XO + 64 + j0, x);
                 tmem_wait_ld();
                 if (write_o) {
+                    __nv_bfloat16 *op = O + (tok0 + t0 + j0) * DV + v;
+                    const int lim = n - j0;
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (j0 + j < n) O[(tok0 + t0 + j0 + j) * DV + v] = __float2bfloat16_rn(x[j]);
+                        if (j < lim) op[j * DV] = __float2bfloat16_rn(x[j]);
                 }
             }
-            const bool last = (c == nchunks - 1);
             for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_S + d0, x);
@@ -727,15 +728,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     tmem_st32(tmem + lane_base + TM_S + d0, x);
                 }
                 st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
-                if (last && STp) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
-                }
             }
             tmem_wait_st();
             tc_fence_before();
             group_sync(BAR_ST);
             if (stid == 0) mbar_arrive(bar_h4 + 8 * pb);   // H4: chunk c finished
+        }
+        // end state: S^T columns [64 half, +64) of this thread's lane, from TMEM
+        if (ok && STp) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 16) {
+                float x[16];
+                tmem_ld16(tmem + lane_base + TM_S + d0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) STp[(size_t)(d0 + j) * DV + v] = x[j];
+            }
         }
         if (!ok) sAbort[0] = 1;
     }
