@@ -420,7 +420,7 @@ def run_ours(args, rank, world, local):
 # keyed by workload and by a digest of the kernel's sources at capture time (a changed
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
-    ("gdn2_t4k", "chunk_tc"): (953.813248e6 + 124.982528e6, "b9da433a"),
+    ("gdn2_t4k", "chunk_tc"): (948.232192e6 + 125.164544e6, "4f526893"),
     ("decode", "decode"): (275.789312e6 + 211.644416e6, "938c1bac"),
 }
 
