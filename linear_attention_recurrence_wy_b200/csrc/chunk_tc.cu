@@ -377,22 +377,23 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         // ============================================================== WY group (0-7)
         const int wtid = tid;   // 0 .. 255
         // raw q, k, b, g_log of chunk c -> staging, one bulk copy per tensor, issued by
-        // lane 0 of warps 0-3 (issuing a bulk copy takes the issuing thread a while)
+        // lane 0 of warps 4-7 (issuing a bulk copy takes the issuing thread a while; warp 0
+        // issues the MMAs)
         auto issue_raw = [&](int c) {
-            if (lane != 0 || warp >= 4) return;
+            if (lane != 0 || warp < 4) return;
             const int t0 = c * C, n = min(C, T - t0);
             const size_t e = (tok0 + t0) * DK;
             const uint32_t row16 = (uint32_t)n * DK * 2;
             fence_async_smem();
-            if (warp == 0) {
+            if (warp == 4) {
                 uint32_t bytes = 2 * row16;
                 if (gdn2) bytes += row16;
                 if (vec_g) bytes += 2 * row16;
                 mbar_arrive_expect_tx(bar_raw, bytes);
                 bulk_g2s(sbase + RAW_Q, Q + e, row16, bar_raw);
-            } else if (warp == 1) {
+            } else if (warp == 5) {
                 bulk_g2s(sbase + RAW_K, K + e, row16, bar_raw);
-            } else if (warp == 2) {
+            } else if (warp == 6) {
                 if (gdn2) bulk_g2s(sbase + RAW_B, Bg + e, row16, bar_raw);
             } else if (vec_g) {
                 bulk_g2s(sbase + RAW_G, a.g + e, 2 * row16, bar_raw);
@@ -498,14 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             }
             fence_async_smem();
             group_sync(BAR_WY);
-            if (wtid == 0) mbar_arrive(bar_h1);   // H1: operands of chunk c built
-            // the raw inputs are dead on the fast path: the next chunk's travel from now on
-            if (!exact && c + 1 < nchunks) {
-                raw_issued = c + 2;
-                issue_raw(c + 1);
-            }
-            // ---- W4: [A; P] = [Kh; Qg] Kb^T; this chunk's P and T buffers were chunk c-2's,
-            //      so that chunk must have finished (H4) ----
+            // ---- W4: [A; P] = [Kh; Qg] Kb^T, issued before the state group may queue its own
+            //      MMAs (H1); this chunk's P and T buffers were chunk c-2's, so that chunk must
+            //      have finished (H4) ----
             if (!exact) {
                 if (wtid == 0) {
                     tc_fence_after();
@@ -517,6 +513,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     mma_commit(bar_wy);
                 }
                 ++mma_wy;
+            }
+            if (wtid == 0) mbar_arrive(bar_h1);   // H1: operands of chunk c built
+            // the raw inputs are dead on the fast path: the next chunk's travel from now on
+            if (!exact && c + 1 < nchunks) {
+                raw_issued = c + 2;
+                issue_raw(c + 1);
             }
             ok = group_and(BAR_WY, wtid != 0 ||
                                        ((exact || wait(bar_wy, (uint32_t)((mma_wy - 1) & 1))) &&
