@@ -171,9 +171,9 @@ gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const 
  * gdr_last_device_error -- read and clear the device-side error word.
  *
  * Synchronises `stream`, then returns GDR_ERR_TIMEOUT if a bounded wait inside a
- * tensor-core kernel gave up since the last call (the kernel then skipped its
- * remaining work and released its tensor memory), GDR_ERR_CUDA if the stream
- * reports a CUDA error, else GDR_OK.
+ * tensor-core kernel or the streaming decode kernel gave up since the last call
+ * (the kernel then skipped its remaining work, drained its own copies and released
+ * its tensor memory), GDR_ERR_CUDA if the stream reports a CUDA error, else GDR_OK.
  */
 gdr_status_t gdr_last_device_error(void *stream);
 

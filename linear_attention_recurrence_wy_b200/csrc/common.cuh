@@ -45,6 +45,8 @@ __device__ __forceinline__ void st_elem(void *p, size_t i, int dtype, float x) {
 // Launch wrappers (one per kernel family); each returns GDR_OK or GDR_ERR_CUDA.
 gdr_status_t launch_chunk_simt(const ChunkArgs &a, cudaStream_t s);
 gdr_status_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// Reads and zeroes the device error word of the streaming decode kernel's bounded waits.
+cudaError_t decode_read_and_clear_error(int *err);
 gdr_status_t launch_state_copy(const ChunkArgs &a, cudaStream_t s);
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);
 

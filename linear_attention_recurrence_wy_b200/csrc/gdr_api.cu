@@ -182,9 +182,10 @@ extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void
 extern "C" gdr_status_t gdr_last_device_error(void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_CUDA;
-    int err = 0;
+    int err = 0, derr = 0;
     if (chunk_tc_read_and_clear_error(&err) != cudaSuccess) return GDR_ERR_CUDA;
-    return err ? GDR_ERR_TIMEOUT : GDR_OK;
+    if (decode_read_and_clear_error(&derr) != cudaSuccess) return GDR_ERR_CUDA;
+    return (err || derr) ? GDR_ERR_TIMEOUT : GDR_OK;
 }
 
 extern "C" const char *gdr_status_string(gdr_status_t status) {

@@ -38,6 +38,26 @@ def test_decode_small(cuda_ok, dtype, mode, dk, dv):
     assert_close("S", np64(S), S_ref, "f32" if dtype == "f32" else dtype)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+def test_decode_many_heads(cuda_ok, dtype, mode):
+    """More heads than SMs at d = 128: every CTA of the streaming kernel cycles its state
+    buffers several times (1177 heads, not a multiple of the SM count), two steps in a row."""
+    N, H, d = 107, 11, 128
+    dd = workload.make_small(N, H, 2, d, d, mode=mode, dtype=dtype, seed=77, s0_std=0.2)
+    S0 = torch.randn(N, H, d, d, generator=torch.Generator().manual_seed(78)) * 0.2
+    step = lambda t: [None if dd[k] is None else dd[k][:, :, t].contiguous() for k in ("q", "k", "v", "g", "b", "w")]
+    S = S0.cuda()
+    Sr = S0.double().numpy()
+    for t in range(2):
+        args = step(t)
+        o = gdr.decode_step(*[None if a is None else a.cuda() for a in args], S, mode=mode)
+        o_ref, Sr = oracle.decode(*args, S=Sr, mode=mode)
+        torch.cuda.synchronize()
+        assert_close(f"o step {t}", np64(o), o_ref, dtype)
+    assert_close("S", np64(S), Sr, "f32" if dtype == "f32" else dtype)
+
+
 def test_decode_workload_1000_steps(cuda_ok):
     cfg = workload.DECODE
     pool = workload.make_decode_pool(cfg)
