@@ -278,7 +278,7 @@ def run_ours(args, rank, world, local):
         d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in pool.items()}
         S = d["S0"].clone()
         P = wl["pool"]
-        n_inner = wl["steps"]
+        n_inner = args.decode_steps or wl["steps"]
 
         def step():
             for s in range(n_inner):
@@ -387,7 +387,7 @@ def run_ours(args, rank, world, local):
         return
     if name == "decode":
         launch_ms = kern_ms / launches_per_step
-        kname = "gdr decode_kernel"
+        kname = "gdr decode_stream_kernel" if wl["dk"] == wl["dv"] == 128 else "gdr decode_kernel"
     else:
         # one step = the whole forward; with a sequence split it is three launches
         # (state pass, combine, output pass) and the step is the unit of the roofline
@@ -420,8 +420,8 @@ def run_ours(args, rank, world, local):
 # keyed by workload and by a digest of the kernel's sources at capture time (a changed
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
-    ("gdn2_t4k", "chunk_tc"): (948.232192e6 + 125.164544e6, "4f526893"),
-    ("decode", "decode"): (275.789312e6 + 211.644416e6, "938c1bac"),
+    ("gdn2_t4k", "chunk_tc"): (948.236288e6 + 126.146048e6, "28ac1924"),
+    ("decode", "decode"): (275.810304e6 + 212.322560e6, "6e1ae928"),
 }
 
 
@@ -464,6 +464,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-cpu-s", type=float, default=15.0)
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="decode steps per bench step (default: the workload's 1000); fewer keep an "
+                         "ncu capture's launch count small")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch of the dominant kernel, if captured for this build")
     args = ap.parse_args()
