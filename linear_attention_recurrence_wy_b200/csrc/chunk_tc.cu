@@ -73,7 +73,8 @@ constexpr int OFF_KB = OFF_QK + 32768;          // Kb bf16 [2][64 t][128 d] 32 K
 constexpr int OFF_P = OFF_KB + 32768;           // P  bf16 [2][64 t][64 j]  16 KB
 constexpr int OFF_T = OFF_P + 16384;            // T  bf16 [2][64 t][64 j]  16 KB
 constexpr int OFF_GS = OFF_T + 16384;           // scalar g_log of the chunk (GDN) fp32 [64]
-constexpr int OFF_GC = OFF_GS + 256;            // gamma_C fp32 [128]
+constexpr int OFF_BETA = OFF_GS + 256;          // scalar beta of the chunk (KDA, GDN) fp32 [64]
+constexpr int OFF_GC = OFF_BETA + 256;          // gamma_C fp32 [128]
 constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [4][128], slot c % 4
 constexpr int OFF_FLAG = OFF_EGC + 2048;        // exact flags [4] (slot c % 4), abort flag
 constexpr int OFF_BAR = OFF_FLAG + 64;          // mbarriers + TMEM slot
@@ -306,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
     float *sGam = reinterpret_cast<float *>(sm + RAW_G);
     float *sGs = reinterpret_cast<float *>(sm + OFF_GS);
+    float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
     float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
     float *sEGC = reinterpret_cast<float *>(sm + OFF_EGC);
     volatile int *sExact = reinterpret_cast<volatile int *>(sm + OFF_FLAG);   // [4]
@@ -408,11 +410,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         auto scan = [&](int c) -> bool {
             const int d = wtid - 128;   // 0 .. 127
             const int t0 = c * C, n = min(C, T - t0);
+            // scalar gates of the tied modes (they need no staging copy): GDN's g_log by
+            // threads 0-63, beta by threads 64-127 for the operand build
+            if (!vec_g && d < 64) sGs[d] = (d < n) ? a.g[tok0 + t0 + d] : 0.f;
+            if (!gdn2 && d >= 64) sBeta[d - 64] = (d - 64 < n) ? __bfloat162float(Bg[tok0 + t0 + d - 64]) : 0.f;
             if (!bar128_and(4, d != 0 || wait(bar_raw, (uint32_t)(c & 1)))) return false;
-            if (!vec_g) {
-                if (d < 64) sGs[d] = (d < n) ? a.g[tok0 + t0 + d] : 0.f;
-                bar128_sync(4);
-            }
             float acc = 0.f, mx = 0.f;
 #pragma unroll 1
             for (int b = 0; b < C; b += 16) {
@@ -469,8 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     if (gdn2) {
                         bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + RAW_B + ro)), fb);
                     } else {
-                        const float bt = __bfloat162float(Bg[tok0 + t0 + min(t, n - 1)]);
-                        const float beta = in ? bt : 0.f;
+                        const float beta = sBeta[t];   // zero past the end
 #pragma unroll
                         for (int j = 0; j < 8; ++j) fb[j] = beta;
                     }
