@@ -411,6 +411,9 @@ def run_ours(args, rank, world, local):
             "data": "synthetic", "config": config_of(name, world), "roofline": roof,
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "wall_total_ms": total_ms}
+    if name != "decode":
+        # the same throughput for a whole layer of H heads: B*T / step time
+        line["layer_tokens_per_s"] = value / wl.H
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(name, target_cpu_s=args.ref_cpu_s)
     print(json.dumps(line), flush=True)

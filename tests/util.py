@@ -30,16 +30,29 @@ def max_abs(x, ref):
     return float(np.max(np.abs(x - ref))) if x.size else 0.0
 
 
+def worst_head(x, ref, metric):
+    """Worst per-(sequence, head) error over the two leading axes (reported beside the
+    whole-tensor figure the tolerance applies to); None below three dimensions."""
+    if x.ndim < 3 or x.size == 0:
+        return None
+    xs = x.reshape(x.shape[0] * x.shape[1], -1)
+    rs = ref.reshape(ref.shape[0] * ref.shape[1], -1)
+    return max(metric(a, b) for a, b in zip(xs, rs))
+
+
 def assert_close(name, x, ref, dtype):
     x, ref = np.asarray(x, np.float64), np.asarray(ref, np.float64)
     assert x.shape == ref.shape, (name, x.shape, ref.shape)
     assert np.all(np.isfinite(x)), f"{name}: non-finite values"
     if dtype in ("f32", torch.float32):
-        err = max_abs(x, ref)
-        assert err <= TOL_F32_MAXABS, f"{name}: max abs err {err:.3e} > {TOL_F32_MAXABS}"
+        metric, tol, what = max_abs, TOL_F32_MAXABS, "max abs"
     else:
-        err = rel_l2(x, ref)
-        assert err <= TOL_BF16_RELL2, f"{name}: rel L2 err {err:.3e} > {TOL_BF16_RELL2}"
+        metric, tol, what = rel_l2, TOL_BF16_RELL2, "rel L2"
+    err = metric(x, ref)
+    worst = worst_head(x, ref, metric)
+    report = f"{name}: {what} err {err:.3e}" + ("" if worst is None else f" (worst head {worst:.3e})")
+    print(report)
+    assert err <= tol, f"{report} > {tol}"
     return err
 
 
