@@ -22,7 +22,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gdr_oracle.c")
 _LIB = os.path.join(_HERE, "libgdr_oracle.so")
-_MODE = {"gdn2": 0, "kda": 1, "gdn": 2}
+_MODE = {"gdn2": 0, "kda": 1, "gdn": 2, "bonly": 3, "wonly": 4}
 _lib = None
 
 
@@ -86,7 +86,8 @@ def fwd(q, k, v, g, b, w=None, S0=None, mode="gdn2", nthreads=None):
 
 def decode(q, k, v, g, b, w=None, S=None, mode="gdn2", nthreads=None):
     """One-token step.  q,k [N,H,dk]; v [N,H,dv]; g [N,H,dk] (gdn: [N,H]);
-    b [N,H,dk] (kda/gdn: beta [N,H]); S [N,H,dk,dv].  Returns (o, S_new)."""
+    b [N,H,dk] (kda/gdn: beta [N,H]; wonly: [N,H]); w [N,H,dv] (bonly: [N,H]);
+    S [N,H,dk,dv].  Returns (o, S_new)."""
     lib = _load()
     q, k, v, g, b, w = map(_f64, (q, k, v, g, b, w))
     S = np.array(_f64(S), copy=True)

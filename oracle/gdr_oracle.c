@@ -27,10 +27,15 @@
  *     mode 2 (GDN): additionally a scalar decay g_t, i.e.
  *                   S_t = alpha_t (I - beta_t k k^T) S_{t-1} + beta_t k v^T,
  *                   alpha_t = exp(g_t).
+ *   Gate-ablation variants (Gated DeltaNet-2 Review §5, "Gate ablation" table), the
+ *   same update with one gate a per-token scalar times the all-ones vector:
+ *     mode 3 (b-only): channel erase b_t [dk], scalar write w_t.
+ *     mode 4 (w-only): scalar erase b_t, channel write w_t [dv].
  *
  * Layouts (row-major): q,k,b [B,H,T,dk]; v,w,o [B,H,T,dv]; g [B,H,T,dk]
- * (mode 2: [B,H,T]); beta (modes 1,2) is passed in b as [B,H,T]; S0, S_T
- * [B,H,dk,dv].  S0 == NULL means a zero initial state; S_T == NULL skips it.
+ * (mode 2: [B,H,T]); beta (modes 1,2) is passed in b as [B,H,T]; the scalar gate of
+ * modes 3 and 4 (w, resp. b) is [B,H,T]; S0, S_T [B,H,dk,dv].  S0 == NULL means a zero
+ * initial state; S_T == NULL skips it.
  * Sequence-heads are distributed over `nthreads` POSIX threads.
  */
 #include <math.h>
@@ -45,7 +50,12 @@ typedef struct {
     int lo, hi; /* [lo, hi) range of sequence-head indices */
 } job_t;
 
-/* One recurrence step on state S (dk x dv); writes o (dv). */
+/* elements of b and w per token, by mode */
+static int b_width(int mode, int dk) { return (mode == 0 || mode == 3) ? dk : 1; }
+static int w_width(int mode, int dv) { return (mode == 0 || mode == 4) ? dv : (mode == 3 ? 1 : 0); }
+
+/* One recurrence step on state S (dk x dv); writes o (dv).  b holds b_width values, w
+ * w_width values (NULL when 0: the write gate is then beta = b[0]). */
 static void step(double *S, const double *q, const double *k, const double *v,
                  const double *g, const double *b, const double *w,
                  int dk, int dv, int mode, double *o, double *r, double *u) {
@@ -58,12 +68,15 @@ static void step(double *S, const double *q, const double *k, const double *v,
     /* r = S^T (b . k) */
     for (int j = 0; j < dv; ++j) r[j] = 0.0;
     for (int i = 0; i < dk; ++i) {
-        double bk = (mode == 0 ? b[i] : b[0]) * k[i];
+        double bk = (mode == 0 || mode == 3 ? b[i] : b[0]) * k[i];
         const double *row = S + (size_t)i * dv;
         for (int j = 0; j < dv; ++j) r[j] += row[j] * bk;
     }
     /* u = w . v - r */
-    for (int j = 0; j < dv; ++j) u[j] = (mode == 0 ? w[j] : b[0]) * v[j] - r[j];
+    for (int j = 0; j < dv; ++j) {
+        double wj = (mode == 0 || mode == 4) ? w[j] : (mode == 3 ? w[0] : b[0]);
+        u[j] = wj * v[j] - r[j];
+    }
     /* S <- S + k u^T */
     for (int i = 0; i < dk; ++i) {
         double *row = S + (size_t)i * dv;
@@ -84,14 +97,14 @@ static void *run_fwd(void *arg) {
     double *r = (double *)malloc(sizeof(double) * dv);
     double *u = (double *)malloc(sizeof(double) * dv);
     const int gw = (J->mode == 2) ? 1 : dk;   /* g elements per token */
-    const int bw = (J->mode == 0) ? dk : 1;   /* b elements per token */
+    const int bw = b_width(J->mode, dk), ww = w_width(J->mode, dv);
     for (int bh = J->lo; bh < J->hi; ++bh) {
         if (J->S0) memcpy(S, J->S0 + (size_t)bh * dk * dv, sizeof(double) * (size_t)dk * dv);
         else memset(S, 0, sizeof(double) * (size_t)dk * dv);
         for (int t = 0; t < T; ++t) {
             size_t tok = (size_t)bh * T + t;
             step(S, J->q + tok * dk, J->k + tok * dk, J->v + tok * dv, J->g + tok * gw,
-                 J->b + tok * bw, J->mode == 0 ? J->w + tok * dv : NULL, dk, dv, J->mode,
+                 J->b + tok * bw, ww ? J->w + tok * ww : NULL, dk, dv, J->mode,
                  J->o + tok * dv, r, u);
         }
         if (J->ST) memcpy(J->ST + (size_t)bh * dk * dv, S, sizeof(double) * (size_t)dk * dv);
@@ -124,7 +137,7 @@ int gdr_oracle_fwd(const double *q, const double *k, const double *v, const doub
                    double *ST, int B, int H, int T, int dk, int dv, int mode, int nthreads) {
     if (!q || !k || !v || !g || !b || !o || B < 0 || H < 0 || T < 0 || dk < 1 || dv < 1)
         return -1;
-    if (mode < 0 || mode > 2 || (mode == 0 && !w)) return -1;
+    if (mode < 0 || mode > 4 || (w_width(mode, dv) && !w)) return -1;
     job_t J = {q, k, v, g, b, w, S0, o, ST, B, H, T, dk, dv, mode, 0, 0};
     if (T == 0) { /* nothing to read out; S_T = S0 */
         if (ST) {
@@ -142,12 +155,12 @@ static void *run_decode(void *arg) {
     double *r = (double *)malloc(sizeof(double) * dv);
     double *u = (double *)malloc(sizeof(double) * dv);
     const int gw = (J->mode == 2) ? 1 : dk;
-    const int bw = (J->mode == 0) ? dk : 1;
+    const int bw = b_width(J->mode, dk), ww = w_width(J->mode, dv);
     for (int nh = J->lo; nh < J->hi; ++nh) {
         double *S = J->ST + (size_t)nh * dk * dv;
         step(S, J->q + (size_t)nh * dk, J->k + (size_t)nh * dk, J->v + (size_t)nh * dv,
              J->g + (size_t)nh * gw, J->b + (size_t)nh * bw,
-             J->mode == 0 ? J->w + (size_t)nh * dv : NULL, dk, dv, J->mode,
+             ww ? J->w + (size_t)nh * ww : NULL, dk, dv, J->mode,
              J->o + (size_t)nh * dv, r, u);
     }
     free(r); free(u);
@@ -160,7 +173,7 @@ int gdr_oracle_decode(const double *q, const double *k, const double *v, const d
                       int N, int H, int dk, int dv, int mode, int nthreads) {
     if (!q || !k || !v || !g || !b || !S || !o || N < 0 || H < 0 || dk < 1 || dv < 1)
         return -1;
-    if (mode < 0 || mode > 2 || (mode == 0 && !w)) return -1;
+    if (mode < 0 || mode > 4 || (w_width(mode, dv) && !w)) return -1;
     job_t J = {q, k, v, g, b, w, NULL, o, S, N, H, 1, dk, dv, mode, 0, 0};
     return launch(J, N * H, nthreads, run_decode);
 }

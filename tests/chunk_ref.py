@@ -37,6 +37,10 @@ def expand_gates(g, b, w, mode, dk, dv):
     """Full per-channel gates from a mode's tied parameters."""
     if mode == "gdn2":
         return g, b, w
+    if mode == "bonly":    # channel erase, one write scalar per token
+        return g, b, np.repeat(w[..., None], dv, axis=-1)
+    if mode == "wonly":    # one erase scalar per token, channel write
+        return g, np.repeat(b[..., None], dk, axis=-1), w
     beta = b
     bb = np.repeat(beta[..., None], dk, axis=-1)
     ww = np.repeat(beta[..., None], dv, axis=-1)

@@ -47,7 +47,7 @@ def test_exact_rational_examples():
 
 
 # 2. chunkwise WY rederivation agrees with the sequential recurrence
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 @pytest.mark.parametrize("C", [16, 32, 64])
 @pytest.mark.parametrize("T", [1, 17, 64, 65, 130])
 def test_chunkwise_rederivation(mode, C, T):
@@ -91,6 +91,40 @@ def test_tied_reductions():
                 S = at * (np.eye(dk) - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, vt)
                 np.testing.assert_allclose(o_gdn[bi, hi, t], S.T @ qt, rtol=1e-11, atol=1e-12)
             np.testing.assert_allclose(S_gdn[bi, hi], S, rtol=1e-11, atol=1e-12)
+
+
+# 3b. gate-ablation variants (Gated DeltaNet-2 Review §5, "Gate ablation"): b-only is
+#     GDN-2 with the write gate w_t * 1, w-only is GDN-2 with the erase gate b_t * 1; the
+#     expanded erase range b in [0, 2] keeps the chunkwise form exact.
+def test_gate_ablation_variants():
+    dk, dv = 8, 6
+    d = rnd_inputs(31, 2, 2, 37, dk, dv, mode="bonly")
+    w_full = np.repeat(d["w"].double().numpy()[..., None], dv, -1)
+    o1, S1 = run_oracle(d)
+    o2, S2 = oracle.fwd(d["q"], d["k"], d["v"], d["g"], d["b"], w_full, d["S0"], mode="gdn2")
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(S1, S2, rtol=1e-13, atol=1e-14)
+    # a write gate that varies over channels must matter: the scalar is not a channel read
+    w_ch = w_full.copy()
+    w_ch[..., 0] *= 0.5
+    o3, _ = oracle.fwd(d["q"], d["k"], d["v"], d["g"], d["b"], w_ch, d["S0"], mode="gdn2")
+    assert np.max(np.abs(o3 - o1)) > 1e-3
+
+    d = rnd_inputs(32, 2, 2, 37, dk, dv, mode="wonly")
+    b_full = np.repeat(d["b"].double().numpy()[..., None], dk, -1)
+    o1, S1 = run_oracle(d)
+    o2, S2 = oracle.fwd(d["q"], d["k"], d["v"], d["g"], b_full, d["w"], d["S0"], mode="gdn2")
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(S1, S2, rtol=1e-13, atol=1e-14)
+
+    d = workload.make_small(2, 2, 70, 12, 10, mode="gdn2", dtype="f32", seed=33, g_scale=0.5,
+                            s0_std=0.3, b_range=2.0)
+    assert float(d["b"].max()) > 1.0                  # the expanded range is in use
+    o, ST = run_oracle(d)
+    o2, ST2 = chunk_ref.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"],
+                                  mode="gdn2", C=32)
+    np.testing.assert_allclose(o, o2, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(ST, ST2, rtol=1e-10, atol=1e-11)
 
 
 # 4. beta = 0: nothing is erased or written; the state only decays (closed form)
@@ -155,7 +189,7 @@ def test_bruteforce_matrix_form():
 
 
 # 8. the decode step repeated T times equals the forward; state hand-off is exact
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 def test_decode_steps_equal_forward_and_split(mode):
     d = rnd_inputs(8, 2, 2, 21, 8, 8, mode=mode)
     o, ST = run_oracle(d)

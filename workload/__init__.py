@@ -10,12 +10,12 @@ Layouts (row-major, contiguous):
   q, k          [B, H, T, dk]
   v             [B, H, T, dv]
   g_log         [B, H, T, dk] fp32   (GDN mode: [B, H, T])
-  b             [B, H, T, dk]        (KDA / GDN modes: beta, [B, H, T])
-  w             [B, H, T, dv]        (KDA / GDN modes: None)
+  b             [B, H, T, dk]        (KDA / GDN modes: beta, [B, H, T]; w-only: [B, H, T])
+  w             [B, H, T, dv]        (KDA / GDN modes: None; b-only: [B, H, T])
   S0            [B, H, dk, dv] fp32 or None
 q, k, v, b, w are rounded to the workload's dtype (fp32 or bf16); g_log and S0
 are always fp32.  Draw order from one torch CPU generator: q, k, v, g, b (or
-beta), w, S0, then any extra tied-mode beta.
+beta), w, S0, then any extra tied-mode beta or variant scalar gate.
 """
 from __future__ import annotations
 
@@ -25,7 +25,7 @@ from typing import Optional
 
 import torch
 
-MODES = ("gdn2", "kda", "gdn")
+MODES = ("gdn2", "kda", "gdn", "bonly", "wonly")
 
 
 @dataclass(frozen=True)
@@ -38,7 +38,7 @@ class Workload:
     dv: int
     chunk: int
     dtype: str            # "f32" or "bf16": dtype of q, k, v, b, w, o
-    mode: str             # "gdn2", "kda" or "gdn"
+    mode: str             # "gdn2", "kda" or "gdn" (the variants derive from "gdn2")
     seed: int
     g_scale: float = 0.1  # g_log = -softplus(N(0,1)) * g_scale
     q_scale: bool = False # multiply q by dk**-0.5 after normalisation
@@ -84,11 +84,15 @@ def _l2norm(x: torch.Tensor, eps: float = 1e-6) -> torch.Tensor:
     return x * torch.rsqrt((x * x).sum(-1, keepdim=True) + eps)
 
 
-def make_inputs(wl: Workload, mode: Optional[str] = None, B: Optional[int] = None):
+def make_inputs(wl: Workload, mode: Optional[str] = None, B: Optional[int] = None,
+                b_range: float = 1.0):
     """Draw one workload's inputs on the CPU.  Returns a dict of torch tensors.
 
     `mode` overrides the workload's mode (the tied KDA variant of the long
-    context workload uses the same q, k, v, g and draws beta after w).
+    context workload uses the same q, k, v, g and draws beta after S0; the b-only
+    and w-only gate-ablation variants of a GDN-2 workload draw their scalar gate
+    there too).  `b_range` scales the erase gate: 2 gives the expanded erase range
+    b in [0, 2] of the same ablation.
     `B` draws only the first B sequences' worth of shapes (used by sharded
     runs; the draw is then a different sample)."""
     mode = mode or wl.mode
@@ -121,6 +125,11 @@ def make_inputs(wl: Workload, mode: Optional[str] = None, B: Optional[int] = Non
         # tied variant on the same q, k, v, g: b = w = beta * 1
         b = torch.sigmoid(randn(Bn, H, T))
         w = None
+    elif mode == "bonly":
+        w = torch.sigmoid(randn(Bn, H, T))   # scalar write gate
+    elif mode == "wonly":
+        b = torch.sigmoid(randn(Bn, H, T))   # scalar erase gate
+    b = b * b_range
     out = dict(q=q.to(dt).contiguous(), k=k.to(dt).contiguous(), v=v.to(dt).contiguous(),
                g=g.contiguous(), b=b.to(dt).contiguous(),
                w=None if w is None else w.to(dt).contiguous(),
@@ -129,12 +138,12 @@ def make_inputs(wl: Workload, mode: Optional[str] = None, B: Optional[int] = Non
 
 
 def make_small(B, H, T, dk, dv, mode="gdn2", dtype="f32", seed=0, g_scale=1.0,
-               s0_std=0.0, g_const=None):
+               s0_std=0.0, g_const=None, b_range=1.0):
     """Inputs for a small parity case of arbitrary shape."""
     wl = Workload("small", B=B, H=H, T=T, dk=dk, dv=dv, chunk=64, dtype=dtype,
                   mode="gdn" if mode == "gdn" else "gdn2", seed=seed,
                   g_scale=g_scale, s0_std=s0_std)
-    d = make_inputs(wl, mode=mode)
+    d = make_inputs(wl, mode=mode, b_range=b_range)
     if g_const is not None:
         d["g"] = torch.full_like(d["g"], float(g_const))
     return d
