@@ -11,7 +11,11 @@
  * g_t in R^{dk} (fp32), erase gate b_t in [0,1]^{dk} and write gate w_t in [0,1]^{dv}.
  * The tied modes are the reductions named on the same Q3: KDA (b = w = beta * 1) and
  * Gated DeltaNet (additionally a scalar decay, S_t = alpha_t (I - beta_t k k^T)
- * S_{t-1} + beta_t k v^T with alpha_t = exp(g_t)).
+ * S_{t-1} + beta_t k v^T with alpha_t = exp(g_t)).  The gate-ablation variants of the
+ * Gated DeltaNet-2 Review (§5, "Gate ablation") keep one gate channel-wise and make the
+ * other a per-token scalar: b-only (channel erase b, scalar write w) and w-only (scalar
+ * erase b, channel write w).  The "expanded erase range" variant of the same table is
+ * b in [0, 2], which every mode accepts as input values.
  *
  * Common conventions
  *   - Every pointer is a DEVICE pointer on the current CUDA device; the caller owns
@@ -23,8 +27,8 @@
  *   - Layouts are row-major and contiguous:
  *       q, k   [B, H, T, dk]          v, o   [B, H, T, dv]
  *       g_log  [B, H, T, dk] fp32     (GDR_MODE_GDN: [B, H, T])
- *       b      [B, H, T, dk]          (KDA, GDN: beta [B, H, T])
- *       w      [B, H, T, dv]          (KDA, GDN: ignored, may be NULL)
+ *       b      [B, H, T, dk]          (KDA, GDN: beta [B, H, T]; w-only: [B, H, T])
+ *       w      [B, H, T, dv]          (KDA, GDN: ignored, may be NULL; b-only: [B, H, T])
  *       S0,S_T [B, H, dk, dv] fp32
  *   - q, k, v, b, w, o have the element type `dtype`; g_log and states are fp32.
  *   - Every pointer must be 16-byte aligned (GDR_ERR_ALIGN otherwise).
@@ -55,7 +59,9 @@ typedef enum {
 typedef enum {
     GDR_MODE_GDN2 = 0,     /* Gated DeltaNet-2: g [dk], b [dk], w [dv] per token */
     GDR_MODE_KDA = 1,      /* KDA: g [dk], beta per token in b; w ignored */
-    GDR_MODE_GDN = 2       /* Gated DeltaNet: scalar g, beta per token in b; w ignored */
+    GDR_MODE_GDN = 2,      /* Gated DeltaNet: scalar g, beta per token in b; w ignored */
+    GDR_MODE_BONLY = 3,    /* b-only variant: g [dk], b [dk], scalar write w per token */
+    GDR_MODE_WONLY = 4     /* w-only variant: g [dk], scalar erase b per token, w [dv] */
 } gdr_mode_t;
 
 typedef enum {

@@ -20,7 +20,7 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdr.so")
-MODES = {"gdn2": 0, "kda": 1, "gdn": 2}
+MODES = {"gdn2": 0, "kda": 1, "gdn": 2, "bonly": 3, "wonly": 4}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 _lib = None
 
@@ -119,8 +119,15 @@ def _check(t, name, shape, dtype, device):
 
 
 def _gate_shapes(mode, lead, dk, dv):
+    """Shapes of g, b and w (None: w unused) for a mode."""
+    if mode not in MODES:
+        raise ValueError(f"unknown mode {mode!r}")
     if mode == "gdn2":
         return (*lead, dk), (*lead, dk), (*lead, dv)
+    if mode == "bonly":
+        return (*lead, dk), (*lead, dk), tuple(lead)
+    if mode == "wonly":
+        return (*lead, dk), tuple(lead), (*lead, dv)
     if mode == "kda":
         return (*lead, dk), tuple(lead), None
     return tuple(lead), tuple(lead), None
@@ -129,7 +136,8 @@ def _gate_shapes(mode, lead, dk, dv):
 def chunk_fwd(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, o=None, S_T=None,
               return_state=True):
     """Chunkwise forward.  q,k [B,H,T,dk], v [B,H,T,dv] (fp32 or bf16, CUDA), g fp32,
-    b (beta for kda/gdn), w (gdn2 only), S0 fp32 [B,H,dk,dv] or None.
+    b (beta for kda/gdn, a scalar erase gate for wonly), w (gdn2, bonly: scalar, wonly),
+    S0 fp32 [B,H,dk,dv] or None.
     Returns (o, S_T) with S_T None when return_state is False."""
     B, H, T, dk = q.shape
     dv = v.shape[-1]
@@ -142,7 +150,7 @@ def chunk_fwd(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, o=None, 
     _check(v, "v", (B, H, T, dv), dt, dev)
     _check(g, "g", gshape, torch.float32, dev)
     _check(b, "b", bshape, dt, dev)
-    if mode == "gdn2":
+    if wshape is not None:
         _check(w, "w", wshape, dt, dev)
     if S0 is not None:
         _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
@@ -151,7 +159,7 @@ def chunk_fwd(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, o=None, 
     if S_T is None and return_state:
         S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
     rc = gdr_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
-                       _ptr(w) if mode == "gdn2" else None, _ptr(S0), _ptr(o), _ptr(S_T),
+                       _ptr(w) if wshape is not None else None, _ptr(S0), _ptr(o), _ptr(S_T),
                        B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], _stream())
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd")
@@ -179,14 +187,14 @@ def chunk_fwd_split(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, ns
                                 (v, "v", (B, H, T, dv), dt), (g, "g", gshape, torch.float32),
                                 (b, "b", bshape, dt)):
         _check(t, name, shape, tdt, q.device)
-    if mode == "gdn2":
+    if wshape is not None:
         _check(w, "w", wshape, dt, q.device)
     if o is None:
         o = torch.empty(B, H, T, dv, dtype=dt, device=q.device)
     if S_T is None and return_state:
         S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     rc = gdr_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
-                             _ptr(w) if mode == "gdn2" else None, _ptr(S0), _ptr(o), _ptr(S_T),
+                             _ptr(w) if wshape is not None else None, _ptr(S0), _ptr(o), _ptr(S_T),
                              B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], nseg,
                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream())
     if rc != 0:
@@ -220,13 +228,13 @@ def decode_step(q, k, v, g, b, w, S, *, mode="gdn2", o=None):
     _check(v, "v", (N, H, dv), dt, dev)
     _check(g, "g", gshape, torch.float32, dev)
     _check(b, "b", bshape, dt, dev)
-    if mode == "gdn2":
+    if wshape is not None:
         _check(w, "w", wshape, dt, dev)
     _check(S, "S", (N, H, dk, dv), torch.float32, dev)
     if o is None:
         o = torch.empty(N, H, dv, dtype=dt, device=dev)
     rc = gdr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
-                         _ptr(w) if mode == "gdn2" else None, _ptr(S), _ptr(o),
+                         _ptr(w) if wshape is not None else None, _ptr(S), _ptr(o),
                          N, H, dk, dv, MODES[mode], DTYPES[dt], _stream())
     if rc != 0:
         raise GdrError(rc, "gdr_decode_step")

@@ -68,8 +68,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
                 const size_t tk = tok0 + c0 + t;
                 kv = ld_elem(a.k, tk * dk + d, a.dtype);
                 qv = ld_elem(a.q, tk * dk + d, a.dtype);
-                bv = (a.mode == GDR_MODE_GDN2) ? ld_elem(a.b, tk * dk + d, a.dtype)
-                                               : ld_elem(a.b, tk, a.dtype);
+                bv = mode_b_vec(a.mode) ? ld_elem(a.b, tk * dk + d, a.dtype) : ld_elem(a.b, tk, a.dtype);
                 gv = (a.mode == GDR_MODE_GDN) ? a.g[tk] : a.g[tk * dk + d];
             }
             kk[idx] = kv;
@@ -83,8 +82,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
             if (t < n) {
                 const size_t tk = tok0 + c0 + t;
                 const float vv = ld_elem(a.v, tk * dv + v0 + j, a.dtype);
-                const float ww = (a.mode == GDR_MODE_GDN2) ? ld_elem(a.w, tk * dv + v0 + j, a.dtype)
-                                                           : ld_elem(a.b, tk, a.dtype);
+                const float ww = mode_w_vec(a.mode) ? ld_elem(a.w, tk * dv + v0 + j, a.dtype)
+                                 : ld_elem(a.mode == GDR_MODE_BONLY ? a.w : a.b, tk, a.dtype);
                 x = ww * vv;
             }
             Vs[idx] = x;

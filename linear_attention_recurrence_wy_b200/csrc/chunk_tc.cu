@@ -324,7 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
     const __nv_bfloat16 *Wg = (const __nv_bfloat16 *)a.w;
     __nv_bfloat16 *O = (__nv_bfloat16 *)a.o;
-    const bool gdn2 = (mode == GDR_MODE_GDN2), vec_g = (mode != GDR_MODE_GDN);
+    // gate shapes: per-channel erase b (GDN-2, b-only), per-channel write w (GDN-2, w-only),
+    // per-channel decay (all but GDN); a scalar write gate is w itself (b-only) or beta
+    const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
+    const __nv_bfloat16 *Wsc = mode == GDR_MODE_BONLY ? Wg : Bg;
 
     if (tid == 0) {
         for (int i = 0; i < NBAR; ++i) mbar_init(bar_wy + 8 * i, 1);
@@ -365,10 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         prefetch_l2(Q + e, n * DK * 2);
         prefetch_l2(K + e, n * DK * 2);
         prefetch_l2(V + e, n * DV * 2);
-        if (gdn2) {
-            prefetch_l2(Bg + e, n * DK * 2);
-            prefetch_l2(Wg + e, n * DV * 2);
-        }
+        if (vec_b) prefetch_l2(Bg + e, n * DK * 2);
+        if (vec_w) prefetch_l2(Wg + e, n * DV * 2);
         if (vec_g) prefetch_l2(a.g + e, n * DK * 4);
     };
 
@@ -389,14 +390,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             fence_async_smem();
             if (warp == 4) {
                 uint32_t bytes = 2 * row16;
-                if (gdn2) bytes += row16;
+                if (vec_b) bytes += row16;
                 if (vec_g) bytes += 2 * row16;
                 mbar_arrive_expect_tx(bar_raw, bytes);
                 bulk_g2s(sbase + RAW_Q, Q + e, row16, bar_raw);
             } else if (warp == 5) {
                 bulk_g2s(sbase + RAW_K, K + e, row16, bar_raw);
             } else if (warp == 6) {
-                if (gdn2) bulk_g2s(sbase + RAW_B, Bg + e, row16, bar_raw);
+                if (vec_b) bulk_g2s(sbase + RAW_B, Bg + e, row16, bar_raw);
             } else if (vec_g) {
                 bulk_g2s(sbase + RAW_G, a.g + e, 2 * row16, bar_raw);
             }
@@ -410,10 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         auto scan = [&](int c) -> bool {
             const int d = wtid - 128;   // 0 .. 127
             const int t0 = c * C, n = min(C, T - t0);
-            // scalar gates of the tied modes (they need no staging copy): GDN's g_log by
-            // threads 0-63, beta by threads 64-127 for the operand build
+            // scalar gates (they need no staging copy): GDN's g_log by threads 0-63, a
+            // scalar erase gate (beta, or w-only's b) by threads 64-127 for the operand build
             if (!vec_g && d < 64) sGs[d] = (d < n) ? a.g[tok0 + t0 + d] : 0.f;
-            if (!gdn2 && d >= 64) sBeta[d - 64] = (d - 64 < n) ? __bfloat162float(Bg[tok0 + t0 + d - 64]) : 0.f;
+            if (!vec_b && d >= 64) sBeta[d - 64] = (d - 64 < n) ? __bfloat162float(Bg[tok0 + t0 + d - 64]) : 0.f;
             if (!bar128_and(4, d != 0 || wait(bar_raw, (uint32_t)(c & 1)))) return false;
             float acc = 0.f, mx = 0.f;
 #pragma unroll 1
@@ -468,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     float fq[8], fk[8], fb[8];
                     bf16x8_to_f32(uq, fq);
                     bf16x8_to_f32(uk, fk);
-                    if (gdn2) {
+                    if (vec_b) {
                         bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + RAW_B + ro)), fb);
                     } else {
                         const float beta = sBeta[t];   // zero past the end
@@ -553,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     }
                 }
             } else {
-                exact_ap(sm, sA32, p_tile - sbase, sGam, gdn2 ? nullptr : Bg + tok0 + t0, n, wtid);
+                exact_ap(sm, sA32, p_tile - sbase, sGam, vec_b ? nullptr : Bg + tok0 + t0, n, wtid);
             }
             group_sync(BAR_WY);
             if (exact && c + 1 < nchunks) {   // raw inputs read above: now the next chunk's
@@ -604,8 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             {
                 const int last = transfer ? -1 : min(31, n - 1 - j0);   // last token column in range
                 const __nv_bfloat16 *vp = V + (tok0 + t0 + j0) * DV + v;
-                const __nv_bfloat16 *wp = gdn2 ? Wg + (tok0 + t0 + j0) * DV + v : Bg + tok0 + t0 + j0;
-                const int ws = gdn2 ? DV : 1;
+                const __nv_bfloat16 *wp = vec_w ? Wg + (tok0 + t0 + j0) * DV + v : Wsc + tok0 + t0 + j0;
+                const int ws = vec_w ? DV : 1;
 #pragma unroll
                 for (int h = 0; h < 32; h += 16) {   // two halves of 16 columns bound the registers
                     __nv_bfloat16 vv[16], ww[16];

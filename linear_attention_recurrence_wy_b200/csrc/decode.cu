@@ -54,8 +54,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
     for (int i = tid; i < DK; i += kThreads) {
         const size_t e = (size_t)nh * DK + i;
         const float kv = ld_elem(a.k, e, a.dtype);
-        const float bv = (a.mode == GDR_MODE_GDN2) ? ld_elem(a.b, e, a.dtype)
-                                                   : ld_elem(a.b, nh, a.dtype);
+        const float bv = mode_b_vec(a.mode) ? ld_elem(a.b, e, a.dtype) : ld_elem(a.b, nh, a.dtype);
         const float gv = (a.mode == GDR_MODE_GDN) ? a.g[nh] : a.g[e];
         s_q[i] = ld_elem(a.q, e, a.dtype);
         s_k[i] = kv;
@@ -64,8 +63,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(DecodeArgs a) {
     }
     for (int j = tid; j < DV; j += kThreads) {
         const size_t e = (size_t)nh * DV + j;
-        const float wv = (a.mode == GDR_MODE_GDN2) ? ld_elem(a.w, e, a.dtype)
-                                                   : ld_elem(a.b, nh, a.dtype);
+        const float wv = mode_w_vec(a.mode) ? ld_elem(a.w, e, a.dtype)
+                         : ld_elem(a.mode == GDR_MODE_BONLY ? a.w : a.b, nh, a.dtype);
         s_wv[j] = wv * ld_elem(a.v, e, a.dtype);
     }
     __syncthreads();
@@ -165,7 +164,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
     const int tid = threadIdx.x, cg = tid & 31, r0 = tid >> 5;   // columns 4 cg .., rows r0 + 8 p
     const int NH = a.N * a.H, G = gridDim.x;
     const int iters = blockIdx.x < NH ? (NH - 1 - blockIdx.x) / G + 1 : 0;
-    const bool bf = a.dtype == GDR_BF16, gdn2 = a.mode == GDR_MODE_GDN2, vec_g = a.mode != GDR_MODE_GDN;
+    const bool bf = a.dtype == GDR_BF16, vec_g = mode_g_vec(a.mode);
+    const bool vec_b = mode_b_vec(a.mode), vec_w = mode_w_vec(a.mode);
+    const void *wsrc = a.mode == GDR_MODE_BONLY ? a.w : a.b;   // scalar write gate, when not vec_w
     const int esz = bf ? 2 : 4;   // bytes per element of q, k, v, b, w
     float *red_r = reinterpret_cast<float *>(sm + SO_RED), *red_o = red_r + 8 * (SD + 1);
     float *s_q = reinterpret_cast<float *>(sm + SO_ROW), *s_k = s_q + SD, *s_bk = s_k + SD;
@@ -175,9 +176,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
     const uint32_t bar_full = sbase + SO_MISC + 8;   // [kBufs] mbarriers, 8-byte aligned
 
     // per-head vectors of iteration i -> vector buffer i & 1 by 16-byte asynchronous copies;
-    // the scalar gates of the tied modes are loaded into registers here (thread 255) and
+    // scalar gates (erase, write, decay) are loaded into registers here (thread 255) and
     // stored by put_scalars once the head before no longer needs the buffer
-    float pend_b = 0.f, pend_g = 0.f;
+    float pend_b = 0.f, pend_w = 0.f, pend_g = 0.f;
     auto fetch_vectors = [&](int i) {
         const int h = blockIdx.x + i * G;
         unsigned char *vb = sm + SO_VEC + (i & 1) * kVecBytes;
@@ -189,8 +190,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
             int pieces = per;
             if (slot == 0) src = (const unsigned char *)a.q + (size_t)h * SD * esz;
             else if (slot == 1) src = (const unsigned char *)a.k + (size_t)h * SD * esz;
-            else if (slot == 2) src = gdn2 ? (const unsigned char *)a.b + (size_t)h * SD * esz : nullptr;
-            else if (slot == 3) src = gdn2 ? (const unsigned char *)a.w + (size_t)h * SD * esz : nullptr;
+            else if (slot == 2) src = vec_b ? (const unsigned char *)a.b + (size_t)h * SD * esz : nullptr;
+            else if (slot == 3) src = vec_w ? (const unsigned char *)a.w + (size_t)h * SD * esz : nullptr;
             else if (slot == 4) src = (const unsigned char *)a.v + (size_t)h * SD * esz;
             else { src = vec_g ? (const unsigned char *)(a.g + (size_t)h * SD) : nullptr; pieces = SD * 4 / 16; }
             if (src && piece < pieces)
@@ -198,14 +199,16 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
         }
         cp_async_commit();
         if (tid == kStreamThreads - 1) {
-            if (!gdn2) pend_b = ld_elem(a.b, h, a.dtype);
+            if (!vec_b) pend_b = ld_elem(a.b, h, a.dtype);
+            if (!vec_w) pend_w = ld_elem(wsrc, h, a.dtype);
             if (!vec_g) pend_g = a.g[h];
         }
     };
     auto put_scalars = [&](int i) {   // thread 255, after fetch_vectors(i)
         float *vb = reinterpret_cast<float *>(sm + SO_VEC + (i & 1) * kVecBytes);
-        if (!gdn2) vb[2 * kVecSlot / 4] = pend_b;   // scalar beta in slot 2
-        if (!vec_g) vb[5 * kVecSlot / 4] = pend_g;  // scalar g_log in slot 5
+        if (!vec_b) vb[2 * kVecSlot / 4] = pend_b;   // scalar erase gate in slot 2
+        if (!vec_w) vb[3 * kVecSlot / 4] = pend_w;   // scalar write gate in slot 3
+        if (!vec_g) vb[5 * kVecSlot / 4] = pend_g;   // scalar g_log in slot 5
     };
     // bounded wait on a state buffer; gives up early once another thread has aborted
     auto wait_full = [&](int i) -> bool {
@@ -254,13 +257,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
                           : reinterpret_cast<const float *>(vb + slot * kVecSlot)[j];
             };
             const float kv = vec(1, tid);
-            const float bv = gdn2 ? vec(2, tid) : reinterpret_cast<const float *>(vb + 2 * kVecSlot)[0];
+            const float bv = vec_b ? vec(2, tid) : reinterpret_cast<const float *>(vb + 2 * kVecSlot)[0];
             const float gv = reinterpret_cast<const float *>(vb + 5 * kVecSlot)[vec_g ? tid : 0];
             s_q[tid] = vec(0, tid);
             s_k[tid] = kv;
             s_bk[tid] = bv * kv;
             s_a[tid] = __expf(gv);
-            const float wv = gdn2 ? vec(3, tid) : bv;
+            const float wv = vec_w ? vec(3, tid) : reinterpret_cast<const float *>(vb + 3 * kVecSlot)[0];
             s_wv[tid] = wv * vec(4, tid);
         }
         ok = __syncthreads_and(tid != 0 || wait_full(i));

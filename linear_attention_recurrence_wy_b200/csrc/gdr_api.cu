@@ -17,7 +17,7 @@ bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 gdr_status_t check_common(int mode, int dtype, int n0, int H, int dk, int dv) {
-    if (mode < GDR_MODE_GDN2 || mode > GDR_MODE_GDN) return GDR_ERR_MODE;
+    if (mode < GDR_MODE_GDN2 || mode > GDR_MODE_WONLY) return GDR_ERR_MODE;
     if (dtype != GDR_F32 && dtype != GDR_BF16) return GDR_ERR_DTYPE;
     if (n0 < 0 || H < 0 || !dim_ok(dk) || !dim_ok(dv)) return GDR_ERR_DIM;
     return GDR_OK;
@@ -33,7 +33,7 @@ gdr_status_t check_chunk(const void *q, const void *k, const void *v, const floa
     if ((int64_t)B * H > INT32_MAX / 64) return GDR_ERR_DIM;
     if ((int64_t)B * H * T > 0) {
         if (!q || !k || !v || !g_log || !b || !o) return GDR_ERR_NULL;
-        if (mode == GDR_MODE_GDN2 && !w) return GDR_ERR_NULL;
+        if (mode_uses_w(mode) && !w) return GDR_ERR_NULL;
     }
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g_log) || !aligned16(b) ||
         !aligned16(w) || !aligned16(S0) || !aligned16(o) || !aligned16(S_T))
@@ -44,7 +44,7 @@ gdr_status_t check_chunk(const void *q, const void *k, const void *v, const floa
 ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_log, const void *b,
                     const void *w, const float *S0, void *o, float *S_T, int B, int H, int T,
                     int dk, int dv, int chunk, int mode, int dtype) {
-    ChunkArgs a{q, k, v, b, mode == GDR_MODE_GDN2 ? w : nullptr, g_log, S0, o, S_T,
+    ChunkArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, o, S_T,
                 B, H, T, dk, dv, chunk, mode, dtype,
                 1, T, 0, nullptr, nullptr, nullptr};
     return a;
@@ -74,7 +74,7 @@ extern "C" gdr_status_t gdr_chunk_fwd(const void *q, const void *k, const void *
     const bool work = (int64_t)B * H * T > 0;
     if (work) {
         if (!q || !k || !v || !g_log || !b || !o) return GDR_ERR_NULL;
-        if (mode == GDR_MODE_GDN2 && !w) return GDR_ERR_NULL;
+        if (mode_uses_w(mode) && !w) return GDR_ERR_NULL;
     }
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g_log) || !aligned16(b) ||
         !aligned16(w) || !aligned16(S0) || !aligned16(o) || !aligned16(S_T))
@@ -170,11 +170,11 @@ extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void
     if ((int64_t)N * H > INT32_MAX) return GDR_ERR_DIM;
     if ((int64_t)N * H == 0) return GDR_OK;
     if (!q || !k || !v || !g_log || !b || !S || !o) return GDR_ERR_NULL;
-    if (mode == GDR_MODE_GDN2 && !w) return GDR_ERR_NULL;
+    if (mode_uses_w(mode) && !w) return GDR_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g_log) || !aligned16(b) ||
         !aligned16(w) || !aligned16(S) || !aligned16(o))
         return GDR_ERR_ALIGN;
-    DecodeArgs a{q, k, v, b, mode == GDR_MODE_GDN2 ? w : nullptr, g_log, S, o,
+    DecodeArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S, o,
                  N, H, dk, dv, (int)mode, (int)dtype};
     return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -59,7 +59,7 @@ def call_dec(q=A, k=A, v=A, g=A, b=A, w=A, S=A, o=A, N=1, H=1, dk=64, dv=64, mod
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(mode=3), MODE), (dict(mode=-1), MODE), (dict(dtype=2), DTYPE),
+    (dict(mode=5), MODE), (dict(mode=-1), MODE), (dict(dtype=2), DTYPE),
     (dict(dk=48), DIM), (dict(dv=256), DIM), (dict(chunk=128), DIM), (dict(chunk=8), DIM),
     (dict(B=-1), DIM), (dict(T=-1), DIM), (dict(H=-2), DIM),
     (dict(q=None), NULL), (dict(k=None), NULL), (dict(v=None), NULL), (dict(g=None), NULL),
@@ -76,6 +76,9 @@ def test_chunk_fwd_tied_modes_do_not_need_w(L):
     assert call_fwd(w=None, mode=1, B=0) == OK
     assert call_fwd(w=None, mode=2, B=0) == OK
     assert call_fwd(w=None, mode=0, B=1) == NULL
+    # the b-only and w-only variants carry a w (scalar, resp. per channel)
+    assert call_fwd(w=None, mode=3, B=1) == NULL
+    assert call_fwd(w=None, mode=4, B=1) == NULL
 
 
 def test_chunk_fwd_empty_batch_is_a_no_op(L):

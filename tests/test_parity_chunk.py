@@ -26,7 +26,7 @@ def check_case(d_cpu, chunk, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 @pytest.mark.parametrize("T", [1, 17, 64, 65, 200])
 def test_small_shapes_modes(cuda_ok, dtype, mode, T):
     d = workload.make_small(2, 3, T, 64, 64, mode=mode, dtype=dtype, seed=T, g_scale=0.5,
@@ -104,7 +104,7 @@ def test_in_place_state_and_split_sequence(cuda_ok):
     assert_close("S split", np64(S), np64(S_full), "f32")
 
 
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 def test_decode_steps_equal_chunk_forward(cuda_ok, mode):
     d_cpu = workload.make_small(2, 2, 40, 64, 64, mode=mode, dtype="f32", seed=11, s0_std=0.1)
     d = to_dev(d_cpu)
@@ -116,6 +116,18 @@ def test_decode_steps_equal_chunk_forward(cuda_ok, mode):
         assert_close(f"o[{t}]", np64(o_t), np64(o_full[:, :, t]), "f32")
     torch.cuda.synchronize()
     assert_close("S", np64(S), np64(S_full), "f32")
+
+
+# ---- gate-ablation variants on the tensor-core path (dk = dv = 128, bf16) --------------
+@pytest.mark.parametrize("mode,b_range", [("bonly", 1.0), ("wonly", 1.0), ("gdn2", 2.0),
+                                          ("bonly", 2.0)])
+@pytest.mark.parametrize("T", [65, 200])
+def test_variants_tensor_core(cuda_ok, mode, b_range, T):
+    """b-only, w-only and the expanded erase range b in [0, 2] (Gated DeltaNet-2 Review,
+    gate ablation) through the tcgen05 kernel."""
+    d = workload.make_small(2, 2, T, 128, 128, mode=mode, dtype="bf16", seed=T + 3, g_scale=0.1,
+                            s0_std=0.05, b_range=b_range)
+    check_case(d, 64, "bf16")
 
 
 # ---- the measured workloads, at full size; sampled sequence-heads vs the oracle ----------

@@ -20,7 +20,7 @@ def pool_step(pool, p, sel=None):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32), (16, 128), (32, 16)])
 def test_decode_small(cuda_ok, dtype, mode, dk, dv):
     torch.manual_seed(dk * dv)
@@ -39,7 +39,7 @@ def test_decode_small(cuda_ok, dtype, mode, dk, dv):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 def test_decode_many_heads(cuda_ok, dtype, mode):
     """More heads than SMs at d = 128: every CTA of the streaming kernel cycles its state
     buffers several times (1177 heads, not a multiple of the SM count), two steps in a row."""

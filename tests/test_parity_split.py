@@ -17,7 +17,7 @@ def split_fwd(d, nseg, S0=None, S_T=None):
                                d["S0"] if S0 is None else S0, mode=d["mode"], nseg=nseg, S_T=S_T)
 
 
-@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn"])
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 @pytest.mark.parametrize("nseg,T", [(2, 200), (3, 640), (5, 1000), (8, 1000), (64, 1000)])
 def test_split_matches_oracle(cuda_ok, mode, nseg, T):
     d_cpu = workload.make_small(1, 3, T, 128, 128, mode=mode, dtype="bf16", seed=nseg + T,
