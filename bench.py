@@ -8,6 +8,7 @@ head), inputs resident in HBM.  Workloads (synthetic, seeded; workload/):
   gdn2_t4k   (default) B=8, H=16, T=4096, dk=dv=128, chunk 64, bf16, Gated DeltaNet-2
   gdn_t2k    B=4, H=16, T=2048, Gated DeltaNet (scalar gates)
   gdn2_t16k  B=1, H=16, T=16384;  gdn2_t16k_kda: the tied KDA mode on the same inputs
+  gdn2_t4k_bonly / gdn2_t4k_wonly: the b-only / w-only gate-ablation variants of gdn2_t4k
   decode     256 sequences x 16 heads, one token per step, state in place
 Metric: token-heads/s (tokens/s per head-layer) = B*H*T / step time (decode:
 step-heads/s).  With N ranks every rank runs its own copy of the workload on its
@@ -45,6 +46,10 @@ def chunk_bytes(wl: workload.Workload, mode: str) -> float:
     per_tok = (2 * dk + dv) * e + dv * e               # q, k, v in; o out
     if mode == "gdn2":
         per_tok += dk * 4 + dk * e + dv * e             # g [dk] fp32, b [dk], w [dv]
+    elif mode == "bonly":
+        per_tok += dk * 4 + dk * e + e                  # g [dk], b [dk], scalar w
+    elif mode == "wonly":
+        per_tok += dk * 4 + e + dv * e                  # g [dk], scalar b, w [dv]
     elif mode == "kda":
         per_tok += dk * 4 + e                           # g [dk], beta
     else:
@@ -170,8 +175,9 @@ def rank_workload(name: str, rank: int):
         cfg["seed"] = cfg["seed"] + 1000 * rank
         return cfg, "gdn2"
     base, mode = name, None
-    if name.endswith("_kda"):
-        base, mode = name[:-4], "kda"
+    for m in ("kda", "bonly", "wonly"):
+        if name.endswith("_" + m):
+            base, mode = name[:-len(m) - 1], m
     wl = workload.CONFIGS[base]
     if rank:
         from dataclasses import replace
@@ -463,7 +469,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gdn2_t4k",
-                    choices=["gdn2_t4k", "gdn_t2k", "gdn2_t16k", "gdn2_t16k_kda", "gdn2_tiny", "decode"])
+                    choices=["gdn2_t4k", "gdn_t2k", "gdn2_t16k", "gdn2_t16k_kda", "gdn2_tiny", "decode",
+                             "gdn2_t4k_bonly", "gdn2_t4k_wonly"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-cpu-s", type=float, default=15.0)
