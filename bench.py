@@ -9,6 +9,8 @@ head), inputs resident in HBM.  Workloads (synthetic, seeded; workload/):
   gdn_t2k    B=4, H=16, T=2048, Gated DeltaNet (scalar gates)
   gdn2_t16k  B=1, H=16, T=16384;  gdn2_t16k_kda: the tied KDA mode on the same inputs
   gdn2_t4k_bonly / gdn2_t4k_wonly: the b-only / w-only gate-ablation variants of gdn2_t4k
+  mixer_t4k  the T=4K shape through gdr_mixer_fwd: raw token-major projections in, the
+             RMSNorm-SiLU-gated output out (activations and epilogue fused in the kernel)
   decode     256 sequences x 16 heads, one token per step, state in place
 Metric: token-heads/s (tokens/s per head-layer) = B*H*T / step time (decode:
 step-heads/s).  With N ranks every rank runs its own copy of the workload on its
@@ -63,6 +65,15 @@ def chunk_flops(wl: workload.Workload) -> float:
     (A, P, W, U, W S, Q S, P E, K^T E; the triangular inverse is not counted)."""
     d = max(wl.dk, wl.dv)
     return wl.units * (6.0 * wl.dk * wl.dv + 10.0 * wl.chunk * d)
+
+
+def mixer_bytes(cfg) -> float:
+    """Raw projections read once (q, k, v, xb, xw, z bf16; xg fp32), y written once, S0 read
+    and S_T written once per head."""
+    dk, dv = cfg["dk"], cfg["dv"]
+    per_tok = (2 * dk + dv) * 2 + dk * 4 + dk * 2 + dv * 2 + dv * 2 + dv * 2
+    per_head = (2 if cfg["s0_std"] > 0 else 1) * dk * dv * 4
+    return cfg["B"] * cfg["H"] * (cfg["T"] * per_tok + per_head)
 
 
 def decode_bytes(cfg) -> float:
@@ -174,6 +185,10 @@ def rank_workload(name: str, rank: int):
         cfg = dict(workload.DECODE)
         cfg["seed"] = cfg["seed"] + 1000 * rank
         return cfg, "gdn2"
+    if name == "mixer_t4k":
+        cfg = dict(workload.MIXER)
+        cfg["seed"] = cfg["seed"] + 1000 * rank
+        return cfg, cfg["mode"]
     base, mode = name, None
     for m in ("kda", "bonly", "wonly"):
         if name.endswith("_" + m):
@@ -205,6 +220,23 @@ def cpu_oracle_sample(name, target_cpu_s=15.0):
         dt = time.perf_counter() - t0
         return dict(value=steps * n_heads / dt, unit="step-heads/s", cores=cores, kind="oracle",
                     sample=f"{steps} decode steps of 16 sequences x {cfg['H']} heads (of 256 x {cfg['H']})")
+    if name == "mixer_t4k":
+        from oracle import mixer
+        c = workload.MIXER
+        d = workload.make_mixer_inputs(1, 1, c["T"], c["dk"], c["dv"], mode=c["mode"], layout=c["layout"],
+                                       seed=c["seed"], xg_shift=c["xg_shift"], s0_std=c["s0_std"])
+        t0 = time.perf_counter()
+        mixer.mixer_fwd(d["q"], d["k"], d["v"], d["xg"], d["xb"], d["xw"], d["z"], d["weight"], d["S0"],
+                        mode=c["mode"], token_major=True)
+        t_head = time.perf_counter() - t0
+        n = max(1, min(c["B"] * c["H"], int(target_cpu_s / max(t_head, 1e-3))))
+        t0 = time.perf_counter()
+        for _ in range(n):
+            mixer.mixer_fwd(d["q"], d["k"], d["v"], d["xg"], d["xb"], d["xw"], d["z"], d["weight"], d["S0"],
+                            mode=c["mode"], token_major=True)
+        dt = time.perf_counter() - t0
+        return dict(value=n * c["T"] / dt, unit="token-heads/s", cores=1, kind="oracle",
+                    sample=f"{n} sequence-heads x T={c['T']} of mixer_t4k, one after another")
     wl, mode = rank_workload(name, 0)
     T = wl.T
     small = workload.Workload("sample", B=1, H=1, T=T, dk=wl.dk, dv=wl.dv, chunk=wl.chunk,
@@ -253,6 +285,8 @@ def run_reference(args, rank, world):
 def metric_name(name):
     if name == "decode":
         return "decode step-heads/s (256 seqs x 16 heads, dk=dv=128); % HBM roofline"
+    if name == "mixer_t4k":
+        return "token-mixer fwd tokens/s per head·layer at T=4K (fused prologue/epilogue); % HBM roofline"
     return "chunked fwd tokens/s per head·layer at T=4K; % tensor-pipe / HBM roofline"
 
 
@@ -262,6 +296,11 @@ def config_of(name, world):
         return {"workload": "gdn2_decode", "N": c["N"], "H": c["H"], "dk": c["dk"], "dv": c["dv"],
                 "mode": "gdn2", "state": "fp32 in place", "inputs": "bf16",
                 "l2": "state 537 MB per step > L2", "parallelism": f"replicas{world}"}
+    if name == "mixer_t4k":
+        c = workload.MIXER
+        return {"workload": name, "B": c["B"], "H": c["H"], "T": c["T"], "dk": c["dk"], "dv": c["dv"],
+                "chunk": c["chunk"], "mode": c["mode"], "layout": "[B,T,H,D]", "inputs": "bf16 raw projections",
+                "state": "fp32", "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
     wl, mode = rank_workload(name, 0)
     return {"workload": name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk, "dv": wl.dv,
             "chunk": wl.chunk, "mode": mode, "inputs": wl.dtype, "state": "fp32",
@@ -279,7 +318,25 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     flush = None
 
-    if name == "decode":
+    if name == "mixer_t4k":
+        c = wl
+        inp = workload.make_mixer_inputs(c["B"], c["H"], c["T"], c["dk"], c["dv"], mode=c["mode"],
+                                         layout=c["layout"], seed=c["seed"], xg_shift=c["xg_shift"],
+                                         s0_std=c["s0_std"])
+        d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
+        y = torch.empty(c["B"], c["T"], c["H"], c["dv"], dtype=torch.bfloat16, device=dev)
+        ST = torch.empty(c["B"], c["H"], c["dk"], c["dv"], dtype=torch.float32, device=dev)
+
+        def fwd():
+            gdr.mixer_fwd(d["q"], d["k"], d["v"], d["xg"], d["xb"], d["xw"], d["z"], d["weight"], d["S0"],
+                          mode=c["mode"], layout=c["layout"], y=y, S_T=ST)
+        step = fwd
+        units = c["B"] * c["H"] * c["T"]
+        bytes_per_launch = mixer_bytes(c)
+        launches_per_step = 1
+        unit = "token-heads/s"
+        nseg = 1
+    elif name == "decode":
         pool = workload.make_decode_pool(wl)
         d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in pool.items()}
         S = d["S0"].clone()
@@ -365,7 +422,30 @@ def run_ours(args, rank, world, local):
 
     # end to end through the public API with host buffers (pinned), copies inside
     e2e = None
-    if not args.no_e2e and name != "decode":
+    if not args.no_e2e and name == "mixer_t4k":
+        c = wl
+        hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v))
+        outh = (torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
+                torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True))
+        d2h = sum(x.numel() * x.element_size() for x in outh)
+        n_e2e = max(1, min(args.steps, 5))
+        call = lambda: gdr.mixer_fwd_host(hin["q"], hin["k"], hin["v"], hin["xg"], hin["xb"], hin["xw"],
+                                          hin["z"], hin["weight"], hin["S0"], mode=c["mode"],
+                                          layout=c["layout"], device=dev, out=outh)
+        call()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+        e2e = {"value": units * world / (e2e_ms * 1e-3), "unit": unit,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    elif not args.no_e2e and name != "decode":
         hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
         h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v))
         outh = (torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
@@ -394,6 +474,9 @@ def run_ours(args, rank, world, local):
     if name == "decode":
         launch_ms = kern_ms / launches_per_step
         kname = "gdr decode_stream_kernel" if wl["dk"] == wl["dv"] == 128 else "gdr decode_kernel"
+    elif name == "mixer_t4k":
+        launch_ms = kern_ms
+        kname = "gdr chunk_tc_kernel<mixer> (tcgen05, fused prologue/epilogue)"
     else:
         # one step = the whole forward; with a sequence split it is three launches
         # (state pass, combine, output pass) and the step is the unit of the roofline
@@ -404,7 +487,7 @@ def run_ours(args, rank, world, local):
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic_for(name, kname), "peak_source": f"{peak_src} hbm_gbs",
             "kernel": kname}
-    if name != "decode":
+    if name not in ("decode", "mixer_t4k"):
         fl = chunk_flops(wl)
         roof["tensor_context"] = {"flops_per_launch": fl,
                                   "achieved_tflops": fl / (launch_ms * 1e-3) / 1e12,
@@ -413,13 +496,13 @@ def run_ours(args, rank, world, local):
     line = {"metric": metric_name(name), "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if (name == "decode" or wl.dtype == "bf16") else "f32",
+            "dtype": "bf16" if (name in ("decode", "mixer_t4k") or wl.dtype == "bf16") else "f32",
             "data": "synthetic", "config": config_of(name, world), "roofline": roof,
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "wall_total_ms": total_ms}
     if name != "decode":
         # the same throughput for a whole layer of H heads: B*T / step time
-        line["layer_tokens_per_s"] = value / wl.H
+        line["layer_tokens_per_s"] = value / (wl["H"] if name == "mixer_t4k" else wl.H)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(name, target_cpu_s=args.ref_cpu_s)
     print(json.dumps(line), flush=True)
@@ -431,6 +514,7 @@ def run_ours(args, rank, world, local):
 TRAFFIC = {
     ("gdn2_t4k", "chunk_tc"): (948.236288e6 + 126.146048e6, "28ac1924"),
     ("decode", "decode"): (275.810304e6 + 212.322560e6, "6e1ae928"),
+    ("mixer_t4k", "chunk_tc"): (1088.785e6 + 126.118144e6, "cc136a80"),
 }
 
 
@@ -470,7 +554,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gdn2_t4k",
                     choices=["gdn2_t4k", "gdn_t2k", "gdn2_t16k", "gdn2_t16k_kda", "gdn2_tiny", "decode",
-                             "gdn2_t4k_bonly", "gdn2_t4k_wonly"])
+                             "gdn2_t4k_bonly", "gdn2_t4k_wonly", "mixer_t4k"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-cpu-s", type=float, default=15.0)

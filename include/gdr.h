@@ -53,7 +53,8 @@ typedef enum {
     GDR_ERR_ALIGN = -5,    /* a pointer is not 16-byte aligned */
     GDR_ERR_CUDA = -6,     /* a CUDA launch or attribute call failed */
     GDR_ERR_TIMEOUT = -7,  /* a bounded device-side wait gave up (tensor-core path) */
-    GDR_ERR_WORKSPACE = -8 /* workspace missing, misaligned or smaller than required */
+    GDR_ERR_WORKSPACE = -8,/* workspace missing, misaligned or smaller than required */
+    GDR_ERR_VALUE = -9     /* a scalar argument is out of range (eps, b_range, layout) */
 } gdr_status_t;
 
 typedef enum {
@@ -68,6 +69,12 @@ typedef enum {
     GDR_F32 = 0,           /* q, k, v, b, w, o are float */
     GDR_BF16 = 1           /* q, k, v, b, w, o are bfloat16 */
 } gdr_dtype_t;
+
+typedef enum {
+    GDR_LAYOUT_BHTD = 0,   /* head-major:  [B, H, T, D] (scalar gates [B, H, T]) */
+    GDR_LAYOUT_BTHD = 1    /* token-major: [B, T, H, D] (scalar gates [B, T, H]), as the
+                              projections of a token-mixer block produce them */
+} gdr_layout_t;
 
 /*
  * gdr_chunk_fwd -- chunkwise-parallel forward over whole sequences.
@@ -172,6 +179,48 @@ gdr_status_t gdr_chunk_fwd_split_noalloc(const void *q, const void *k, const voi
 gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v, const float *g_log,
                              const void *b, const void *w, float *S, void *o, int N, int H,
                              int dk, int dv, gdr_mode_t mode, gdr_dtype_t dtype, void *stream);
+
+/*
+ * gdr_mixer_fwd -- the recurrence inside its token-mixer block, fused into one kernel.
+ *
+ * The block around the recurrence (Gated DeltaNet-2 Review §4-3, engineering notes):
+ * the q and k paths end in an L2 normalisation, the decay branch is a log-decay
+ * projection kept in fp32, the erase and write gates are their own projections through
+ * a sigmoid, and the recurrent output is RMS-normalised and multiplied by a SiLU output
+ * gate.  This call takes the raw projections and returns the gated output:
+ *
+ *     q_t <- q_t / sqrt(|q_t|^2 + 1e-6)        k_t <- k_t / sqrt(|k_t|^2 + 1e-6)
+ *     g_t  = -softplus(xg_t)                    (natural-log decay, <= 0)
+ *     b_t  = b_range * sigmoid(xb_t)            w_t = sigmoid(xw_t)
+ *     o_t  = the forward of gdr_chunk_fwd on (q, k, v, g, b, w) from S0
+ *     y_t  = o_t / sqrt(mean_v o_t[v]^2 + eps) * norm_weight * z_t * sigmoid(z_t)
+ *
+ * In the tied modes (KDA, GDN) xb holds the raw beta, beta = b_range * sigmoid(xb) is
+ * both gates, and xw is ignored (may be NULL).  b-only: xw [.., T] is the raw scalar
+ * write gate; w-only: xb [.., T] is the raw scalar erase gate.  b_range = 2 is the
+ * expanded erase range b in [0, 2]; the write gate is never scaled except as beta.
+ *
+ *   layout       GDR_LAYOUT_BHTD: every per-token tensor is [B, H, T, D] (scalar gates
+ *                [B, H, T]); GDR_LAYOUT_BTHD: [B, T, H, D] (scalar gates [B, T, H]).
+ *                q, k, xb (per channel) have D = dk; v, xw (per channel), z, y have
+ *                D = dv; xg has D = dk (GDN: a scalar).
+ *   xg           fp32 pre-activation decay.  q, k, v, xb, xw, z, y: bf16.
+ *   norm_weight  fp32 [dv], shared by the heads.
+ *   S0, S_T      fp32 [B, H, dk, dv] as in gdr_chunk_fwd (NULL: zero / not written).
+ *   eps          > 0 and finite; b_range >= 0 and finite (else GDR_ERR_VALUE).
+ *   y            must not overlap any input.
+ *
+ * Supported: dtype GDR_BF16, dk = dv = 128, chunk = 64 (the tcgen05 kernel); other
+ * sizes return GDR_ERR_DIM, GDR_F32 returns GDR_ERR_DTYPE.  Every pointer 16-byte
+ * aligned.  T == 0 writes S_T = S0 (or zeros).  Asynchronous on `stream`; validation
+ * first, as for every entry point.
+ */
+gdr_status_t gdr_mixer_fwd(const void *q, const void *k, const void *v, const float *xg,
+                           const void *xb, const void *xw, const void *z,
+                           const float *norm_weight, const float *S0, void *y, float *S_T,
+                           int B, int H, int T, int dk, int dv, int chunk, gdr_mode_t mode,
+                           gdr_dtype_t dtype, gdr_layout_t layout, float b_range, float eps,
+                           void *stream);
 
 /*
  * gdr_last_device_error -- read and clear the device-side error word.

@@ -7,9 +7,9 @@ PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raise
 
 Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
 gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
-gdr_decode_step,
-gdr_last_device_error, gdr_status_string.
-Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, decode_step.
+gdr_mixer_fwd, gdr_decode_step, gdr_last_device_error, gdr_status_string.
+Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
+decode_step.
 """
 from __future__ import annotations
 
@@ -22,6 +22,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgdr.so")
 MODES = {"gdn2": 0, "kda": 1, "gdn": 2, "bonly": 3, "wonly": 4}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+LAYOUTS = {"bhtd": 0, "bthd": 1}
 _lib = None
 
 
@@ -50,6 +51,8 @@ def lib():
         L.gdr_chunk_fwd_split_segments.restype = ci
         L.gdr_chunk_fwd_split_workspace.argtypes = [ci] * 5
         L.gdr_chunk_fwd_split_workspace.restype = ctypes.c_ulonglong
+        L.gdr_mixer_fwd.argtypes = [vp] * 11 + [ci] * 9 + [ctypes.c_float] * 2 + [vp]
+        L.gdr_mixer_fwd.restype = ci
         L.gdr_decode_step.argtypes = [vp] * 8 + [ci] * 6 + [vp]
         L.gdr_decode_step.restype = ci
         L.gdr_last_device_error.argtypes = [vp]
@@ -84,6 +87,12 @@ def gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, dtype):
 
 def gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg):
     return lib().gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg)
+
+
+def gdr_mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0, y, S_T, B, H, T, dk, dv, chunk, mode,
+                  dtype, layout, b_range, eps, stream):
+    return lib().gdr_mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0, y, S_T, B, H, T, dk, dv,
+                               chunk, mode, dtype, layout, b_range, eps, stream)
 
 
 def gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, stream):
@@ -214,6 +223,63 @@ def chunk_fwd_host(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, dev
         out = (torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True),
                torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True))
     out[0].copy_(o_d, non_blocking=True)
+    out[1].copy_(S_d, non_blocking=True)
+    return out
+
+
+def mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0=None, *, mode="gdn2", layout="bhtd",
+              b_range=1.0, eps=1e-5, chunk=64, y=None, S_T=None, return_state=True):
+    """The recurrence inside its token-mixer block (gdr_mixer_fwd): raw projections in,
+    gated output out.  layout "bhtd": q, k, xb [B,H,T,dk], v, xw, z [B,H,T,dv] (scalar
+    gates [B,H,T]); "bthd": [B,T,H,d] (scalar gates [B,T,H]).  bf16 except xg (fp32) and
+    norm_weight (fp32 [dv]).  Returns (y, S_T) with y in the input layout."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"unknown layout {layout!r}")
+    if layout == "bhtd":
+        B, H, T, dk = q.shape
+        lead = (B, H, T)
+    else:
+        B, T, H, dk = q.shape
+        lead = (B, T, H)
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    if dt not in DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    gshape, bshape, wshape = _gate_shapes(mode, lead, dk, dv)
+    for t, name, shape, tdt in ((q, "q", (*lead, dk), dt), (k, "k", (*lead, dk), dt),
+                                (v, "v", (*lead, dv), dt), (xg, "xg", gshape, torch.float32),
+                                (xb, "xb", bshape, dt), (z, "z", (*lead, dv), dt),
+                                (norm_weight, "norm_weight", (dv,), torch.float32)):
+        _check(t, name, shape, tdt, dev)
+    if wshape is not None:
+        _check(xw, "xw", wshape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if y is None:
+        y = torch.empty(*lead, dv, dtype=dt, device=dev)
+    if S_T is None and return_state:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    rc = gdr_mixer_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(xg), _ptr(xb),
+                       _ptr(xw) if wshape is not None else None, _ptr(z), _ptr(norm_weight),
+                       _ptr(S0), _ptr(y), _ptr(S_T), B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt],
+                       LAYOUTS[layout], float(b_range), float(eps), _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_mixer_fwd")
+    return y, S_T
+
+
+def mixer_fwd_host(q, k, v, xg, xb, xw, z, norm_weight, S0=None, *, mode="gdn2", layout="bhtd",
+                   b_range=1.0, eps=1e-5, device="cuda", out=None):
+    """mixer_fwd end to end from host tensors (pinned host memory is copied
+    asynchronously); y and S_T come back into host tensors (`out` to reuse them)."""
+    nb = q.is_pinned()
+    to = lambda t: None if t is None else t.to(device, non_blocking=nb)
+    y_d, S_d = mixer_fwd(to(q), to(k), to(v), to(xg), to(xb), to(xw), to(z), to(norm_weight), to(S0),
+                         mode=mode, layout=layout, b_range=b_range, eps=eps)
+    if out is None:
+        out = (torch.empty(y_d.shape, dtype=y_d.dtype, pin_memory=True),
+               torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True))
+    out[0].copy_(y_d, non_blocking=True)
     out[1].copy_(S_d, non_blocking=True)
     return out
 

@@ -36,10 +36,27 @@
 // chunks ahead of the state group.  The next chunk's raw inputs are copied as soon as
 // the operands are built (fast path) or A and P are formed (exact path).
 //
+// Token mixer (kMixer instantiation; Gated DeltaNet-2 Review §4-3, engineering notes): the
+// same pipeline on the block's raw projections.  The scan turns the decay projection into
+// e^gamma as a running product of sigmoid(-x) (= e^-softplus(x)); the operand build
+// L2-normalises q and k per token (16 lanes per token, shuffles) and applies b's sigmoid;
+// the state group applies w's sigmoid and, after the state update, the output gate
+// y = o rsqrt(mean_v o^2 + eps) weight z sigmoid(z): the sum of squares over the value
+// channels is one MMA of the squared outputs against a ones operand in TMEM, and y leaves
+// through the chunk's free K-bar tile by one TMA tensor store.  Either layout, [B,H,T,D]
+// or the projections' [B,T,H,D] (then the raw q, k, b, g chunks arrive by TMA tensor copies).
+//
 // Every wait on an mbarrier is bounded.  On expiry a thread raises a CTA-wide abort flag;
 // both groups leave their loops at their next wait, the kernel records the failure in
 // g_tc_error, waits (bounded) for its own bulk copies and tensor-core work, frees its
 // TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <string.h>
+
+#include <mutex>
+
 #include "chunk_tc.cuh"
 #include "tc_util.cuh"
 #include "tri_inverse.cuh"
@@ -56,6 +73,7 @@ constexpr int C = 64, DK = 128, DV = 128;
 constexpr int kThreads = 512;
 constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kFastLimit = 60.f;
+constexpr float kFastProd = 8.7565108e-27f;   // e^-60: the same limit on e^gamma
 constexpr int kAS = tri::LD;   // fp32 row stride of the A / T scratch
 
 // shared memory map (byte offsets from a 1024-aligned base)
@@ -77,7 +95,8 @@ constexpr int OFF_BETA = OFF_GS + 256;          // scalar beta of the chunk (KDA
 constexpr int OFF_GC = OFF_BETA + 256;          // gamma_C fp32 [128]
 constexpr int OFF_EGC = OFF_GC + 512;           // exp(gamma_C) fp32 [4][128], slot c % 4
 constexpr int OFF_FLAG = OFF_EGC + 2048;        // exact flags [4] (slot c % 4), abort flag
-constexpr int OFF_BAR = OFF_FLAG + 64;          // mbarriers + TMEM slot
+constexpr int OFF_RQ = OFF_FLAG + 64;           // mixer: 1/||q_t||, 1/||k_t|| of the chunk [2][64]
+constexpr int OFF_BAR = OFF_RQ + 512;           // mbarriers + TMEM slot
 constexpr int NBAR = 9;
 constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 8 + 1024;   // + alignment slack
 
@@ -87,6 +106,8 @@ constexpr uint32_t TM_XO = 128;  // [X, then E^T | O^T] fp32                  64
 constexpr uint32_t TM_AP = 256;  // [A; P] fp32                                 64
 constexpr uint32_t TM_SB = 320;  // S^T bf16 (packed)                           64
 constexpr uint32_t TM_XB = 384;  // R^T, then E^T bf16 (packed)                 32
+constexpr uint32_t TM_ONES = 448; // mixer: bf16 ones, the A operand of the output's
+                                  // sum of squares over value channels        64
 constexpr uint32_t TM_COLS = 512;
 
 // named barriers (0 is __syncthreads; 1 is warps 0-3, the inverse's; 4 is warps 4-7, the scan's)
@@ -189,6 +210,22 @@ __device__ __forceinline__ void mbar_arrive(uint32_t saddr) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr) : "memory");
 }
 
+// ---- token-mixer activations (Gated DeltaNet-2 Review §4-3, engineering notes) ----------
+// log(1 + e^x) = max(x, 0) + log(1 + e^-|x|): the decay branch, g = -softplus(x)
+__device__ __forceinline__ float softplus_f(float x) {
+    return fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x)));
+}
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// The gates (b, w, beta and the SiLU of z) through one tanh: sigmoid(x) = (1 + tanh(x/2)) / 2,
+// with PTX tanh.approx (about 2^-11 relative error, below the bf16 rounding of the operands
+// these gates scale).  The decay keeps the exp-based form: its factors multiply up over a chunk.
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float sigmoid_gate(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
+
 // Final values of T (from the inverse) straight into the bf16 operand tile.
 struct TileOut {
     uint32_t tile;   // shared address of the T tile ([64 t][64 j], 128-byte swizzled)
@@ -217,10 +254,13 @@ __device__ __forceinline__ void drain_commits(uint32_t bar, int n) {
 // Exact path, strong-decay chunks only: A (fp32, strictly lower) and P (bf16 tile, lower
 // incl.) from per-pair decays exp(gamma_i - gamma_j), computed from the staged raw q, k, b
 // and gamma on CUDA cores by the 256 threads of the WY group.  beta: the scalar b of the
-// chunk's tokens (tied modes), or NULL when b is a per-channel vector staged with q and k.
+// chunk's tokens in shared memory (tied modes, w-only), or NULL when b is a per-channel
+// vector staged with q and k.  Mixer: rq, rk hold the tokens' 1/||q||, 1/||k|| (else
+// NULL) and b_act > 0 makes a per-channel b = b_act * sigmoid(raw b).
 // Kept out of line: it is rarely run and would otherwise crowd the instruction cache.
 __device__ __noinline__ void exact_ap(unsigned char *sm, float *sA32, uint32_t p_off, const float *sGam,
-                                      const __nv_bfloat16 *beta, int n, int wtid) {
+                                      const float *beta, const float *rq, const float *rk, float b_act,
+                                      int n, int wtid) {
 #pragma unroll 1
     for (int u = 0; u < 16; ++u) {
         const int p = wtid + u * 256, i = p >> 6, j = p & 63;
@@ -230,14 +270,19 @@ __device__ __noinline__ void exact_ap(unsigned char *sm, float *sA32, uint32_t p
             const __nv_bfloat16 *ki = (const __nv_bfloat16 *)(sm + RAW_K) + i * DK;
             const __nv_bfloat16 *kj = (const __nv_bfloat16 *)(sm + RAW_K) + j * DK;
             const __nv_bfloat16 *bi = (const __nv_bfloat16 *)(sm + RAW_B) + i * DK;
-            const float bs = beta ? __bfloat162float(beta[i]) : 0.f;
+            const float bs = beta ? beta[i] : 0.f;
 #pragma unroll 2
             for (int d = 0; d < DK; ++d) {
                 const float dec = __expf(sGam[i * DK + d] - sGam[j * DK + d]);
                 const float kjd = __bfloat162float(kj[d]) * dec;
-                const float bid = beta ? bs : __bfloat162float(bi[d]);
+                float bid = beta ? bs : __bfloat162float(bi[d]);
+                if (!beta && b_act > 0.f) bid = b_act * sigmoid_gate(bid);
                 sa = fmaf(bid * __bfloat162float(ki[d]), kjd, sa);
                 sp = fmaf(__bfloat162float(qi[d]), kjd, sp);
+            }
+            if (rq) {
+                sa *= rk[i] * rk[j];
+                sp *= rq[i] * rk[j];
             }
         }
         sA32[i * kAS + j] = (j < i) ? sa : 0.f;
@@ -247,12 +292,16 @@ __device__ __noinline__ void exact_ap(unsigned char *sm, float *sA32, uint32_t p
 
 // Exact path: gamma of key channel d over the chunk's n tokens (zero contribution past the
 // end) from the g_log in global memory, stride apart, into column d of the gamma tile
-// (strong-decay chunks only; out of line like exact_ap).
-__device__ __noinline__ void exact_gamma(float *sGam, const float *g, int stride, int n, int d) {
+// (strong-decay chunks only; out of line like exact_ap).  act: the mixer's raw decay
+// projection, g = -softplus(raw).
+__device__ __noinline__ void exact_gamma(float *sGam, const float *g, size_t stride, int n, int d, bool act) {
     float acc = 0.f;
 #pragma unroll 1
     for (int t = 0; t < C; ++t) {
-        if (t < n) acc += g[(size_t)t * stride];
+        if (t < n) {
+            const float x = g[(size_t)t * stride];
+            acc += act ? -softplus_f(x) : x;
+        }
         sGam[t * DK + d] = acc;
     }
 }
@@ -272,7 +321,20 @@ __device__ __noinline__ void prescale_state(uint32_t taddr, const float *egc, in
     tmem_wait_st();
 }
 
-__global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
+// Tensor maps of the mixer (one box = one chunk of one head, rows dense in shared memory).
+// Token-major inputs [B, T, H, D]: dims {D, H, T, B}, box {D, 1, 64, 1}; the raw chunk
+// inputs then arrive by one tiled copy per tensor (rows past the end of a sequence are
+// zero-filled), and v, w, z are prefetched to L2 by box.  y, the mixer's output, is
+// written by one tiled store per chunk in either layout (head-major: dims {D, T, H, B},
+// box {D, 64, 1, 1}); rows past the end are clipped.
+struct TokenMaps {
+    CUtensorMap q, k, b, g, v, w, z, y;
+};
+
+// kMixer: the token-mixer instantiation (activations on load, output epilogue, either
+// layout; ChunkArgs::mixer).  The plain instantiation is the recurrence alone on [B,H,T,D].
+template <bool kMixer>
+__global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, const __grid_constant__ TokenMaps tm) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
@@ -288,7 +350,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     const int t_begin = seg * a.seg_len;
     const int T = min(a.seg_len, a.T - t_begin);              // tokens of this segment
     const int mode = a.mode;
-    const size_t tok0 = (size_t)bh * a.T + t_begin;
+    // token t of this segment is row tok0 + t * ts of every [.., D] input
+    const int ts = kMixer ? a.tstride : 1;
+    size_t tok0 = (size_t)bh * a.T + t_begin;
+    if (kMixer && ts != 1) tok0 = ((size_t)(bh / a.H) * a.T + t_begin) * a.H + bh % a.H;
+    const int hc = bh % a.H, bc = bh / a.H;   // tensor-map coordinates of this head
     const int nchunks = (T + C - 1) / C;
     const size_t sidx = ((size_t)bh * a.nseg + seg) * DK * DV;
     const float *S0p = nullptr;        // initial state (NULL: zero, unless the identity)
@@ -310,6 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
     float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
     float *sEGC = reinterpret_cast<float *>(sm + OFF_EGC);
+    float *sRq = reinterpret_cast<float *>(sm + OFF_RQ), *sRk = sRq + 64;
     volatile int *sExact = reinterpret_cast<volatile int *>(sm + OFF_FLAG);   // [4]
     volatile int *sAbort = reinterpret_cast<volatile int *>(sm + OFF_FLAG + 16);
     const uint32_t bar_wy = sbase + OFF_BAR;     // the WY group's MMA commits
@@ -324,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
     const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
     const __nv_bfloat16 *Wg = (const __nv_bfloat16 *)a.w;
     __nv_bfloat16 *O = (__nv_bfloat16 *)a.o;
+    const __nv_bfloat16 *Z = (const __nv_bfloat16 *)a.z;
     // gate shapes: per-channel erase b (GDN-2, b-only), per-channel write w (GDN-2, w-only),
     // per-channel decay (all but GDN); a scalar write gate is w itself (b-only) or beta
     const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
@@ -361,8 +429,20 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         return false;
     };
 
-    // L2 prefetch of chunk c's inputs (issued by the state group's first thread)
+    // L2 prefetch of chunk c's inputs (issued by the state group's first thread; contiguous
+    // chunks only)
     auto prefetch_inputs = [&](int c) {
+        if (kMixer && ts != 1) {
+            const int tt = t_begin + c * C;
+            tma_prefetch_4d(&tm.q, 0, hc, tt, bc);
+            tma_prefetch_4d(&tm.k, 0, hc, tt, bc);
+            tma_prefetch_4d(&tm.v, 0, hc, tt, bc);
+            tma_prefetch_4d(&tm.z, 0, hc, tt, bc);
+            if (vec_b) tma_prefetch_4d(&tm.b, 0, hc, tt, bc);
+            if (vec_w) tma_prefetch_4d(&tm.w, 0, hc, tt, bc);
+            if (vec_g) tma_prefetch_4d(&tm.g, 0, hc, tt, bc);
+            return;
+        }
         const int t0 = c * C, n = min(C, T - t0);
         const size_t e = (tok0 + t0) * DK;
         prefetch_l2(Q + e, n * DK * 2);
@@ -371,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         if (vec_b) prefetch_l2(Bg + e, n * DK * 2);
         if (vec_w) prefetch_l2(Wg + e, n * DV * 2);
         if (vec_g) prefetch_l2(a.g + e, n * DK * 4);
+        if (kMixer) prefetch_l2(Z + e, n * DV * 2);
     };
 
     int raw_issued = 0, raw_done = 0;   // raw copies (WY group)
@@ -383,6 +464,28 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         // lane 0 of warps 4-7 (issuing a bulk copy takes the issuing thread a while; warp 0
         // issues the MMAs)
         auto issue_raw = [&](int c) {
+            if (kMixer && ts != 1) {
+                // token-major: one tiled tensor copy per tensor; a box is always whole
+                // (64 rows, zero-filled past the end), so its bytes are counted whole
+                if (lane != 0 || warp < 4) return;
+                const int tt = t_begin + c * C;
+                constexpr uint32_t box16 = C * DK * 2;
+                fence_async_smem();
+                if (warp == 4) {
+                    uint32_t bytes = 2 * box16;
+                    if (vec_b) bytes += box16;
+                    if (vec_g) bytes += 2 * box16;
+                    mbar_arrive_expect_tx(bar_raw, bytes);
+                    tma_load_4d(sbase + RAW_Q, &tm.q, 0, hc, tt, bc, bar_raw);
+                } else if (warp == 5) {
+                    tma_load_4d(sbase + RAW_K, &tm.k, 0, hc, tt, bc, bar_raw);
+                } else if (warp == 6) {
+                    if (vec_b) tma_load_4d(sbase + RAW_B, &tm.b, 0, hc, tt, bc, bar_raw);
+                } else if (vec_g) {
+                    tma_load_4d(sbase + RAW_G, &tm.g, 0, hc, tt, bc, bar_raw);
+                }
+                return;
+            }
             if (lane != 0 || warp < 4) return;
             const int t0 = c * C, n = min(C, T - t0);
             const size_t e = (tok0 + t0) * DK;
@@ -413,9 +516,46 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             const int t0 = c * C, n = min(C, T - t0);
             // scalar gates (they need no staging copy): GDN's g_log by threads 0-63, a
             // scalar erase gate (beta, or w-only's b) by threads 64-127 for the operand build
-            if (!vec_g && d < 64) sGs[d] = (d < n) ? a.g[tok0 + t0 + d] : 0.f;
-            if (!vec_b && d >= 64) sBeta[d - 64] = (d - 64 < n) ? __bfloat162float(Bg[tok0 + t0 + d - 64]) : 0.f;
+            if (!vec_g && d < 64) {
+                const float x = (d < n) ? a.g[tok0 + (size_t)(t0 + d) * ts] : 0.f;
+                sGs[d] = kMixer ? sigmoid_f(-x) : x;   // mixer: the decay factor e^g itself
+            }
+            if (!vec_b && d >= 64) {
+                const float x = (d - 64 < n) ? __bfloat162float(Bg[tok0 + (size_t)(t0 + d - 64) * ts]) : 0.f;
+                sBeta[d - 64] = (kMixer && d - 64 < n) ? a.b_range * sigmoid_gate(x) : x;
+            }
             if (!bar128_and(4, d != 0 || wait(bar_raw, (uint32_t)(c & 1)))) return false;
+            if (kMixer) {
+                // g = -softplus(raw) <= 0, so e^g = sigmoid(-raw) and e^gamma is the running
+                // product of those factors (no logarithm per token); |gamma| peaks at the
+                // chunk's last token, where the fast-path limit is checked
+                float prod = 1.f;
+#pragma unroll 1
+                for (int b = 0; b < C; b += 16) {
+                    float x[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] = vec_g ? sGam[(b + i) * DK + d] : sGs[b + i];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float e = vec_g ? sigmoid_f(-x[i]) : x[i];
+                        prod *= (b + i < n) ? e : 1.f;
+                        x[i] = prod;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) sGam[(b + i) * DK + d] = x[i];
+                }
+                const bool any = bar128_or(4, !(prod >= kFastProd));
+                float gc = 0.f;
+                if (any) {
+                    exact_gamma(sGam, vec_g ? a.g + (tok0 + (size_t)t0 * ts) * DK + d : a.g + tok0 + (size_t)t0 * ts,
+                                vec_g ? (size_t)DK * ts : (size_t)ts, n, d, true);
+                    gc = sGam[(C - 1) * DK + d];
+                }
+                sGC[d] = gc;
+                sEGC[(c & 3) * 128 + d] = any ? __expf(gc) : prod;
+                if (d == 0) sExact[c & 3] = any ? 1 : 0;
+                return true;
+            }
             float acc = 0.f, mx = 0.f;
 #pragma unroll 1
             for (int b = 0; b < C; b += 16) {
@@ -432,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 for (int i = 0; i < 16; ++i) sGam[(b + i) * DK + d] = x[i];
             }
             const bool any = bar128_or(4, mx > kFastLimit);
-            if (any) exact_gamma(sGam, vec_g ? a.g + (tok0 + t0) * DK + d : a.g + tok0 + t0, vec_g ? DK : 1, n, d);
+            if (any) exact_gamma(sGam, vec_g ? a.g + (tok0 + t0) * DK + d : a.g + tok0 + t0, vec_g ? DK : 1, n, d, false);
             sGC[d] = acc;
             sEGC[(c & 3) * 128 + d] = __expf(acc);
             if (d == 0) sExact[c & 3] = any ? 1 : 0;
@@ -469,8 +609,37 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     float fq[8], fk[8], fb[8];
                     bf16x8_to_f32(uq, fq);
                     bf16x8_to_f32(uk, fk);
+                    if (kMixer) {
+                        // L2 norms of q_t and k_t: the 16 threads of token t are 16
+                        // consecutive lanes (tokens past the end are zero and stay zero)
+                        float sq = 0.f, sk = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            sq = fmaf(fq[j], fq[j], sq);
+                            sk = fmaf(fk[j], fk[j], sk);
+                        }
+#pragma unroll
+                        for (int o = 1; o < 16; o <<= 1) {
+                            sq += __shfl_xor_sync(0xffffffffu, sq, o);
+                            sk += __shfl_xor_sync(0xffffffffu, sk, o);
+                        }
+                        const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            fq[j] *= rq;
+                            fk[j] *= rk;
+                        }
+                        if (cg == 0) {
+                            sRq[t] = rq;
+                            sRk[t] = rk;
+                        }
+                    }
                     if (vec_b) {
                         bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + RAW_B + ro)), fb);
+                        if (kMixer) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) fb[j] = a.b_range * sigmoid_gate(fb[j]);
+                        }
                     } else {
                         const float beta = sBeta[t];   // zero past the end
 #pragma unroll
@@ -554,7 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                     }
                 }
             } else {
-                exact_ap(sm, sA32, p_tile - sbase, sGam, vec_b ? nullptr : Bg + tok0 + t0, n, wtid);
+                exact_ap(sm, sA32, p_tile - sbase, sGam, vec_b ? nullptr : sBeta, kMixer ? sRq : nullptr,
+                         kMixer ? sRk : nullptr, (kMixer && vec_b) ? a.b_range : 0.f, n, wtid);
             }
             group_sync(BAR_WY);
             if (exact && c + 1 < nchunks) {   // raw inputs read above: now the next chunk's
@@ -579,6 +749,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
         const int half = (warp - 8) >> 2;
         const int v = quarter * 32 + lane;   // value channel = TMEM lane
         const int j0 = half * 32;            // this thread's token columns of X, E and O
+        const size_t vs = (size_t)DV * ts;   // elements between consecutive tokens of v, w, z, o
+        // mixer: RMSNorm weight of this value channel; the write gate's activation scale
+        // (the tied modes write with beta = b_range * sigmoid(b))
+        const float nwv = kMixer ? a.nw[v] : 0.f;
+        const float wact = (mode == GDR_MODE_KDA || mode == GDR_MODE_GDN) ? a.b_range : 1.f;
         bool ok = true;
         // initial state -> TMEM: fp32 S^T and its bf16 operand copy
         for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
@@ -588,6 +763,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 x[j] = transfer ? (d0 + j == v ? 1.f : 0.f) : (S0p ? S0p[(size_t)(d0 + j) * DV + v] : 0.f);
             tmem_st32(tmem + lane_base + TM_S + d0, x);
             st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
+        }
+        if (kMixer) {
+            float ones[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ones[j] = __uint_as_float(0x3F803F80u);   // bf16 pair (1, 1)
+            tmem_st32(tmem + lane_base + TM_ONES + half * 32, ones);
         }
         if (stid == 0 && nchunks > 1) prefetch_inputs(1);
         tmem_wait_st();
@@ -602,11 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             // (w.v)^T for this thread's lane and token columns, read from global memory
             // before the wait for the operands; tokens past the end give zero
             float wvt[32];
+            uint32_t zp[16];   // mixer: the output gate z of the same lane and tokens, bf16 pairs
             {
                 const int last = transfer ? -1 : min(31, n - 1 - j0);   // last token column in range
-                const __nv_bfloat16 *vp = V + (tok0 + t0 + j0) * DV + v;
-                const __nv_bfloat16 *wp = vec_w ? Wg + (tok0 + t0 + j0) * DV + v : Wsc + tok0 + t0 + j0;
-                const int ws = vec_w ? DV : 1;
+                const size_t row = tok0 + (size_t)(t0 + j0) * ts;
+                const __nv_bfloat16 *vp = V + row * DV + v;
+                const __nv_bfloat16 *wp = vec_w ? Wg + row * DV + v : Wsc + row;
+                const size_t ws = vec_w ? vs : (size_t)ts;
 #pragma unroll
                 for (int h = 0; h < 32; h += 16) {   // two halves of 16 columns bound the registers
                     __nv_bfloat16 vv[16], ww[16];
@@ -614,7 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                         // whole columns: fixed offsets from one base address, all loads in flight
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            vv[j] = vp[(h + j) * DV];
+                            vv[j] = vp[(h + j) * vs];
                             ww[j] = wp[(h + j) * ws];
                         }
                     } else if (last >= 0) {
@@ -622,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int jj = min(h + j, last);
-                            vv[j] = vp[jj * DV];
+                            vv[j] = vp[jj * vs];
                             ww[j] = wp[jj * ws];
                         }
                     } else {
@@ -631,8 +814,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                         for (int j = 0; j < 16; ++j) vv[j] = ww[j] = __float2bfloat16_rn(0.f);
                     }
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        wvt[h + j] = (h + j <= last) ? __bfloat162float(ww[j]) * __bfloat162float(vv[j]) : 0.f;
+                    for (int j = 0; j < 16; ++j) {
+                        float wf = __bfloat162float(ww[j]);
+                        if (kMixer) wf = wact * sigmoid_gate(wf);
+                        wvt[h + j] = (h + j <= last) ? wf * __bfloat162float(vv[j]) : 0.f;
+                    }
+                }
+                if (kMixer && write_o) {
+                    // loaded here, while the group waits for the operands, and kept packed
+                    const __nv_bfloat16 *zq = Z + row * DV + v;
+                    unsigned short zb[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        zb[j] = last >= 0 ? __bfloat16_as_ushort(zq[min(j, last) * vs]) : (unsigned short)0;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) zp[j] = (uint32_t)zb[2 * j] | ((uint32_t)zb[2 * j + 1] << 16);
                 }
             }
             // ---- S1: operands of chunk c (H1); [X | O] = S^T [Kh; Qg]^T ----
@@ -666,7 +862,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             tmem_wait_st();
             tc_fence_before();
             group_sync(BAR_ST);
-            if (stid == 0) mbar_arrive(bar_h3);   // H3: Kh, Qg of chunk c consumed
+            if (stid == 0) {
+                // the previous chunk's output store has read its tile (a K-bar buffer the
+                // WY group may rebuild once H3 has arrived)
+                if (kMixer) bulk_wait_read_all();
+                mbar_arrive(bar_h3);   // H3: Kh, Qg of chunk c consumed
+            }
             // ---- S3: T and P of chunk c (H2); E^T = R^T T^T ----
             ok = group_and(BAR_ST, stid != 0 || wait(bar_h2 + 8 * pb, (uint32_t)((c >> 1) & 1)));
             if (!ok) break;
@@ -710,17 +911,40 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             tc_fence_after();
             // ---- S6: output rows [j0, j0 + 32); state columns [64 half, +64) scaled, kept
             //      in fp32 and as the bf16 operand ----
-            {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_XO + 64 + j0, x);
-                tmem_wait_ld();
-                if (write_o) {
-                    __nv_bfloat16 *op = O + (tok0 + t0 + j0) * DV + v;
-                    const int lim = n - j0;
+            float xo[32];
+            tmem_ld32(tmem + lane_base + TM_XO + 64 + j0, xo);
+            tmem_wait_ld();
+            if (!kMixer && write_o) {
+                __nv_bfloat16 *op = O + (tok0 + (size_t)(t0 + j0) * ts) * DV + v;
+                const int lim = n - j0;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (j < lim) op[j * DV] = __float2bfloat16_rn(x[j]);
+                for (int j = 0; j < 32; ++j)
+                    if (j < lim) op[j * vs] = __float2bfloat16_rn(xo[j]);
+            }
+            if (kMixer && write_o) {
+                // RMSNorm of the output over the 128 value channels (one per TMEM lane): the
+                // squares go to this chunk's K-bar buffer (free once S5 has completed) as a
+                // bf16 [v][t] tile, and one MMA against a ones A operand writes sum_v o^2 of
+                // every token into every lane; it runs while the state is rescaled below
+                uint32_t sq[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sq[j] = pack_bf16(xo[2 * j] * xo[2 * j], xo[2 * j + 1] * xo[2 * j + 1]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    st_shared_v4(kb_tile + tile_chunk(128, v, j0 / 8 + q), sq[4 * q], sq[4 * q + 1], sq[4 * q + 2],
+                                 sq[4 * q + 3]);
+                fence_async_smem();
+                tc_fence_before();
+                group_sync(BAR_ST);
+                if (stid == 0) {
+                    tc_fence_after();
+                    const uint32_t id = idesc_bf16(128, 64, false, true, false);
+#pragma unroll
+                    for (int s = 0; s < DV / 16; ++s)
+                        mma_bf16_ts(tmem + TM_XO, tmem + TM_ONES + s * 8, desc_mnmajor(kb_tile, 128, 0, s), id, s > 0);
+                    mma_commit(bar_st);
                 }
+                ++mma_st;
             }
             for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
                 float x[32];
@@ -734,6 +958,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
                 st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, x);
             }
             tmem_wait_st();
+            if (kMixer && write_o) {
+                // y = o * rsqrt(mean_v o^2 + eps) * weight_v * z * sigmoid(z)
+                ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+                if (!ok) break;
+                tc_fence_after();
+                float ss[32];
+                tmem_ld32(tmem + lane_base + TM_XO + j0, ss);
+                tmem_wait_ld();
+                // every lane holds the same 32 sums: lane j takes token j's rsqrt, the rest by shuffle
+                float mine = ss[0];
+#pragma unroll
+                for (int j = 1; j < 32; ++j) mine = lane == j ? ss[j] : mine;
+                const float rstd = rsqrtf(fmaf(mine, 1.f / 128.f, a.eps));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float zf = __uint_as_float((j & 1) ? (zp[j >> 1] & 0xFFFF0000u) : (zp[j >> 1] << 16));
+                    xo[j] *= __shfl_sync(0xffffffffu, rstd, j) * nwv * (zf * sigmoid_gate(zf));
+                }
+                // y rows -> this chunk's K-bar buffer (the sum MMA has read it), row-major
+                // [64 t][128 v]; one tiled store writes the chunk (rows past the end clipped)
+                unsigned short *yt = reinterpret_cast<unsigned short *>(sm + (kb_tile - sbase));
+#pragma unroll
+                for (int j = 0; j < 32; ++j) yt[(j0 + j) * DV + v] = __bfloat16_as_ushort(__float2bfloat16_rn(xo[j]));
+                fence_async_smem();
+                group_sync(BAR_ST);
+                if (stid == 0) {
+                    const int tt = t_begin + t0;
+                    if (ts != 1) tma_store_4d(&tm.y, kb_tile, 0, hc, tt, bc);
+                    else tma_store_4d(&tm.y, kb_tile, 0, tt, hc, bc);
+                    bulk_commit();
+                }
+            }
             tc_fence_before();
             group_sync(BAR_ST);
             if (stid == 0) mbar_arrive(bar_h4 + 8 * pb);   // H4: chunk c finished
@@ -751,6 +1007,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a) {
             }
         }
         if (!ok) sAbort[0] = 1;
+        if (kMixer && stid == 0) bulk_wait_all();   // the last output store has landed
     }
 
     __syncthreads();
@@ -778,13 +1035,85 @@ bool chunk_tc_supported(const ChunkArgs &a) {
     return a.dtype == GDR_BF16 && a.dk == DK && a.dv == DV && a.chunk == C;
 }
 
+namespace {
+
+// cuTensorMapEncodeTiled from the driver, looked up once (no link against libcuda)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Map of a token-major [B, T, H, D] tensor (D = 128 elements of esize bytes): dims
+// {D, H, T, B}, box {D, 1, C, 1}, no swizzle, zero fill out of range.
+bool encode_token_major(CUtensorMap *m, const void *base, int B, int T, int H, CUtensorMapDataType dt,
+                        int esize) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)DK, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)DK * esize, (cuuint64_t)H * DK * esize,
+                                   (cuuint64_t)T * H * DK * esize};
+    const cuuint32_t box[4] = {(cuuint32_t)DK, 1, (cuuint32_t)C, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Map of a head-major [B, H, T, D] tensor: dims {D, T, H, B}, box {D, C, 1, 1}.
+bool encode_head_major(CUtensorMap *m, const void *base, int B, int T, int H, CUtensorMapDataType dt,
+                       int esize) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)DK, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)DK * esize, (cuuint64_t)T * DK * esize,
+                                   (cuuint64_t)H * T * DK * esize};
+    const cuuint32_t box[4] = {(cuuint32_t)DK, (cuuint32_t)C, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 gdr_status_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-    if (cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
+    static_assert(DK == DV, "one box shape serves every per-channel tensor");
+    auto kern = a.mixer ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
+    TokenMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    if (a.mixer && a.tstride != 1) {
+        const auto BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        bool ok = encode_token_major(&tm.q, a.q, a.B, a.T, a.H, BF, 2) &&
+                  encode_token_major(&tm.k, a.k, a.B, a.T, a.H, BF, 2) &&
+                  encode_token_major(&tm.v, a.v, a.B, a.T, a.H, BF, 2) &&
+                  encode_token_major(&tm.z, a.z, a.B, a.T, a.H, BF, 2);
+        if (ok && mode_b_vec(a.mode)) ok = encode_token_major(&tm.b, a.b, a.B, a.T, a.H, BF, 2);
+        if (ok && mode_w_vec(a.mode)) ok = encode_token_major(&tm.w, a.w, a.B, a.T, a.H, BF, 2);
+        if (ok && mode_g_vec(a.mode))
+            ok = encode_token_major(&tm.g, a.g, a.B, a.T, a.H, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4);
+        if (!ok) return GDR_ERR_CUDA;
+    }
+    if (a.mixer) {
+        const bool ok = a.tstride != 1
+                            ? encode_token_major(&tm.y, a.o, a.B, a.T, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2)
+                            : encode_head_major(&tm.y, a.o, a.B, a.T, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2);
+        if (!ok) return GDR_ERR_CUDA;
+    }
     const int roles = a.pass ? (2 * a.nseg - 3 > 1 ? 2 * a.nseg - 3 : 1) : a.nseg;
-    chunk_tc_kernel<<<(unsigned)(a.B * a.H * roles), kThreads, SMEM_BYTES, s>>>(a);
+    kern<<<(unsigned)(a.B * a.H * roles), kThreads, SMEM_BYTES, s>>>(a, tm);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

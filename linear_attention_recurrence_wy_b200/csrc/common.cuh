@@ -22,6 +22,17 @@ struct ChunkArgs {
     // segments 1 .. nseg-2 (ws_m; identity start state, values taken as zero).
     int nseg, seg_len, pass;
     float *ws_send, *ws_m, *ws_sstart;   // [B*H][nseg][dk][dv] fp32 each
+    // Token mixer (tensor-core kernel only).  mixer != 0: q, k, v, g, b, w hold the raw
+    // projections and the kernel applies the block's activations as it loads them
+    // (q, k L2-normalised per token, g = -softplus(g), b = b_range * sigmoid(b),
+    // w = sigmoid(w); the tied modes' write gate is beta = b_range * sigmoid(b)), and o
+    // receives y = o * rsqrt(mean_v o^2 + eps) * nw * z * sigmoid(z).
+    // tstride: rows between consecutive tokens of one head, 1 for [B,H,T,D] or H for
+    // [B,T,H,D] (the token-major layout of the projections).
+    int mixer, tstride;
+    const void *z;
+    const float *nw;
+    float b_range, eps;
 };
 
 struct DecodeArgs {

@@ -3,6 +3,7 @@
 // Validation happens before anything is enqueued, so a rejected call launches
 // nothing.  Dispatch picks one device kernel per call; there is no host or
 // library fallback for any step of the computation.
+#include <math.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -46,7 +47,8 @@ ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_
                     int dk, int dv, int chunk, int mode, int dtype) {
     ChunkArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, o, S_T,
                 B, H, T, dk, dv, chunk, mode, dtype,
-                1, T, 0, nullptr, nullptr, nullptr};
+                1, T, 0, nullptr, nullptr, nullptr,
+                0, 1, nullptr, nullptr, 1.f, 0.f};
     return a;
 }
 
@@ -161,6 +163,33 @@ extern "C" gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const 
     return launch_chunk_tc(a, s);
 }
 
+extern "C" gdr_status_t gdr_mixer_fwd(const void *q, const void *k, const void *v, const float *xg,
+                                      const void *xb, const void *xw, const void *z,
+                                      const float *norm_weight, const float *S0, void *y,
+                                      float *S_T, int B, int H, int T, int dk, int dv, int chunk,
+                                      gdr_mode_t mode, gdr_dtype_t dtype, gdr_layout_t layout,
+                                      float b_range, float eps, void *stream) {
+    gdr_status_t st = check_chunk(q, k, v, xg, xb, xw, S0, y, S_T, B, H, T, dk, dv, chunk, mode, dtype);
+    if (st != GDR_OK) return st;
+    if (dtype != GDR_BF16) return GDR_ERR_DTYPE;
+    if (dk != 128 || dv != 128 || chunk != 64) return GDR_ERR_DIM;
+    if (layout != GDR_LAYOUT_BHTD && layout != GDR_LAYOUT_BTHD) return GDR_ERR_VALUE;
+    if (!(eps > 0.f) || !(eps < INFINITY) || !(b_range >= 0.f) || !(b_range < INFINITY)) return GDR_ERR_VALUE;
+    if ((int64_t)B * H * T > 0 && (!z || !norm_weight)) return GDR_ERR_NULL;
+    if (!aligned16(z) || !aligned16(norm_weight)) return GDR_ERR_ALIGN;
+    ChunkArgs a = make_args(q, k, v, xg, xb, xw, S0, y, S_T, B, H, T, dk, dv, chunk, mode, dtype);
+    a.mixer = 1;
+    a.tstride = layout == GDR_LAYOUT_BTHD ? H : 1;
+    a.z = z;
+    a.nw = norm_weight;
+    a.b_range = b_range;
+    a.eps = eps;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((int64_t)B * H == 0) return GDR_OK;
+    if (T == 0) return launch_state_copy(a, s);
+    return launch_chunk_tc(a, s);
+}
+
 extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v,
                                         const float *g_log, const void *b, const void *w,
                                         float *S, void *o, int N, int H, int dk, int dv,
@@ -199,6 +228,7 @@ extern "C" const char *gdr_status_string(gdr_status_t status) {
         case GDR_ERR_CUDA: return "GDR_ERR_CUDA: CUDA launch or runtime error";
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait expired";
         case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case GDR_ERR_VALUE: return "GDR_ERR_VALUE: scalar argument out of range";
     }
     return "unknown gdr_status_t";
 }

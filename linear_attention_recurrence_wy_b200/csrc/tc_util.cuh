@@ -196,6 +196,38 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst_saddr, const void *src, ui
 __device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
+// Tiled tensor copy (TMA) of one box of a 4-D tensor map into shared memory, completing on
+// mbar; tmap is the generic address of a __grid_constant__ CUtensorMap parameter.  The
+// innermost coordinate c0 must be a multiple of 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst_saddr, const void *tmap, int c0, int c1, int c2,
+                                            int c3, uint32_t mbar_saddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+        "%4, %5}], [%6];" ::"r"(dst_saddr),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(mbar_saddr)
+        : "memory");
+}
+// Tiled tensor store (TMA) of one box from shared memory; out-of-range rows are clipped.
+// Completion is tracked by the issuing thread's bulk async-groups.
+__device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src_saddr, int c0, int c1, int c2,
+                                             int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(tmap),
+        "r"(src_saddr), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until the committed bulk stores have read their shared-memory source
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// wait until the committed bulk stores have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void tma_prefetch_4d(const void *tmap, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(tmap),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

@@ -13,7 +13,7 @@ from linear_attention_recurrence_wy_b200 import build as gbuild
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "gdr.h")
 
-OK, NULL, DIM, MODE, DTYPE, ALIGN, WORKSPACE = 0, -1, -2, -3, -4, -5, -8
+OK, NULL, DIM, MODE, DTYPE, ALIGN, WORKSPACE, VALUE = 0, -1, -2, -3, -4, -5, -8, -9
 
 
 @pytest.fixture(scope="module")
@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -9):
         s = gdr.gdr_status_string(code)
         assert s.startswith("GDR_")
     assert "unknown" in gdr.gdr_status_string(42)
@@ -131,3 +131,29 @@ def test_split_workspace_size_and_segments(L):
 ])
 def test_split_rejects(L, kw, code):
     assert call_split(**kw) == code
+
+
+def call_mixer(q=A, k=A, v=A, xg=A, xb=A, xw=A, z=A, nw=A, S0=None, y=A, ST=None, B=1, H=2, T=8,
+               dk=128, dv=128, chunk=64, mode=0, dtype=1, layout=1, b_range=1.0, eps=1e-5):
+    return gdr.gdr_mixer_fwd(q, k, v, xg, xb, xw, z, nw, S0, y, ST, B, H, T, dk, dv, chunk, mode, dtype,
+                             layout, b_range, eps, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=7), MODE), (dict(dtype=0), DTYPE), (dict(dtype=3), DTYPE), (dict(dk=64), DIM),
+    (dict(dv=64), DIM), (dict(chunk=32), DIM), (dict(T=-1), DIM), (dict(layout=2), VALUE),
+    (dict(layout=-1), VALUE), (dict(eps=0.0), VALUE), (dict(eps=-1.0), VALUE),
+    (dict(eps=float("nan")), VALUE), (dict(eps=float("inf")), VALUE), (dict(b_range=-0.5), VALUE),
+    (dict(b_range=float("nan")), VALUE), (dict(q=None), NULL), (dict(xg=None), NULL),
+    (dict(xb=None), NULL), (dict(xw=None), NULL), (dict(z=None), NULL), (dict(nw=None), NULL),
+    (dict(y=None), NULL), (dict(z=A + 2), ALIGN), (dict(nw=A + 4), ALIGN), (dict(xg=A + 8), ALIGN),
+])
+def test_mixer_rejects(L, kw, code):
+    assert call_mixer(**kw) == code
+
+
+def test_mixer_tied_modes_and_empty_batch(L):
+    # xw is ignored in the tied modes; with B = 0 nothing is launched
+    assert call_mixer(xw=None, mode=1, B=0) == OK
+    assert call_mixer(xw=None, mode=2, B=0) == OK
+    assert call_mixer(q=None, k=None, v=None, xg=None, xb=None, xw=None, z=None, nw=None, y=None, B=0) == OK

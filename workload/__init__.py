@@ -174,6 +174,46 @@ def make_decode_pool(cfg=DECODE, N=None, pool=None):
                 S0=S0.contiguous(), mode=cfg["mode"])
 
 
+# The token-mixer workload: the raw projections of the T=4K shape, token-major as a
+# block's projections produce them.  xg ~ N(-2.5, 1) puts the decay g = -softplus(xg)
+# near the T=4K workload's typical size (about -0.1 per token).
+MIXER = dict(name="mixer_t4k", B=8, H=16, T=4096, dk=128, dv=128, chunk=64, mode="gdn2",
+             layout="bthd", seed=5, xg_shift=-2.5, s0_std=0.02)
+
+
+def make_mixer_inputs(B, H, T, dk, dv, mode="gdn2", layout="bhtd", seed=0, xg_shift=-2.5,
+                      xg_scale=1.0, s0_std=0.0, b_range=1.0):
+    """Raw inputs of the token-mixer block (gdr_mixer_fwd): q, k, v, the pre-activation
+    gates xg (fp32), xb, xw, the output gate z (bf16) and the RMSNorm weight (fp32 [dv]).
+    layout "bhtd" draws [B, H, T, .], "bthd" draws [B, T, H, .].  Draw order from one
+    torch CPU generator: q, k, v, xg, xb, xw, S0, z, weight."""
+    assert mode in MODES and layout in ("bhtd", "bthd")
+    gen = torch.Generator().manual_seed(seed)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+    lead = (B, H, T) if layout == "bhtd" else (B, T, H)
+    q = randn(*lead, dk)
+    k = randn(*lead, dk)
+    v = randn(*lead, dv)
+    xg = (randn(*lead) if mode == "gdn" else randn(*lead, dk)) * xg_scale + xg_shift
+    xb = randn(*lead, dk) if mode in ("gdn2", "bonly") else randn(*lead)
+    if mode in ("gdn2", "wonly"):
+        xw = randn(*lead, dv)
+    elif mode == "bonly":
+        xw = randn(*lead)
+    else:
+        xw = None
+    S0 = randn(B, H, dk, dv) * s0_std if s0_std > 0 else None
+    z = randn(*lead, dv)
+    weight = 1.0 + 0.1 * randn(dv)
+    bf = lambda x: None if x is None else x.to(torch.bfloat16).contiguous()
+    return dict(q=bf(q), k=bf(k), v=bf(v), xg=xg.contiguous(), xb=bf(xb), xw=bf(xw), z=bf(z),
+                weight=weight.contiguous(), S0=None if S0 is None else S0.contiguous(), mode=mode,
+                layout=layout, b_range=b_range)
+
+
 def shard_range(n_units: int, rank: int, world: int):
     """Contiguous [lo, hi) share of n_units for one rank (independent units)."""
     base, rem = divmod(n_units, world)
