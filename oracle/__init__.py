@@ -9,7 +9,9 @@ only marshals arrays.
 Every oracle function is pinned by independent checks in tests/test_oracle_pins.py
 (chunkwise rederivation, tied-gate reductions, closed forms for beta = 0, exact
 recall, the linear-attention special case, exact rational arithmetic on tiny
-inputs, decode/forward equivalence).
+inputs, decode/forward equivalence); the backward (bwd) in tests/test_oracle_bwd_pins.py
+(central finite differences in every mode, closed forms for linear attention and for
+a pure decay).
 """
 from __future__ import annotations
 
@@ -45,6 +47,8 @@ def _load():
         lib.gdr_oracle_fwd.restype = ctypes.c_int
         lib.gdr_oracle_decode.argtypes = [dp] * 8 + [ctypes.c_int] * 6
         lib.gdr_oracle_decode.restype = ctypes.c_int
+        lib.gdr_oracle_bwd.argtypes = [dp] * 16 + [ctypes.c_int] * 7
+        lib.gdr_oracle_bwd.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -99,6 +103,27 @@ def decode(q, k, v, g, b, w=None, S=None, mode="gdn2", nthreads=None):
     if rc != 0:
         raise ValueError("gdr_oracle_decode: bad arguments")
     return o, S
+
+
+def bwd(q, k, v, g, b, w=None, S0=None, dO=None, dST=None, mode="gdn2", nthreads=None):
+    """Gradient of L = sum(o * dO) + sum(S_T * dST) with respect to every input of fwd
+    (adjoint of the sequential recurrence, gdr_oracle_bwd).  Returns a dict with dq, dk,
+    dv, dg, db, dw (None when the mode has no w) and dS0, each shaped like its input
+    (dS0 like S0, [B,H,dk,dv], also when S0 is None)."""
+    lib = _load()
+    q, k, v, g, b, w, S0, dO, dST = map(_f64, (q, k, v, g, b, w, S0, dO, dST))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    out = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dg=np.zeros_like(g),
+               db=np.zeros_like(b), dw=None if w is None else np.zeros_like(w),
+               dS0=np.zeros((B, H, dk, dv)))
+    rc = lib.gdr_oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w), _ptr(S0), _ptr(dO),
+                            _ptr(dST), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dg"]),
+                            _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]), B, H, T, dk, dv,
+                            _MODE[mode], nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("gdr_oracle_bwd: bad arguments")
+    return out
 
 
 def fwd_heads(inp, heads, nthreads=None):
