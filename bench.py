@@ -11,6 +11,8 @@ head), inputs resident in HBM.  Workloads (synthetic, seeded; workload/):
   gdn2_t4k_bonly / gdn2_t4k_wonly: the b-only / w-only gate-ablation variants of gdn2_t4k
   mixer_t4k  the T=4K shape through gdr_mixer_fwd: raw token-major projections in, the
              RMSNorm-SiLU-gated output out (activations and epilogue fused in the kernel)
+  bwd_t4k    the backward (gdr_chunk_bwd) of gdn2_t4k: dq, dk, dv, dg, db, dw and dS0 from dO
+             and dS_T (three launches; fp32 CUDA cores)
   decode     256 sequences x 16 heads, one token per step, state in place
 Metric: token-heads/s (tokens/s per head-layer) = B*H*T / step time (decode:
 step-heads/s).  With N ranks every rank runs its own copy of the workload on its
@@ -74,6 +76,27 @@ def mixer_bytes(cfg) -> float:
     per_tok = (2 * dk + dv) * 2 + dk * 4 + dk * 2 + dv * 2 + dv * 2 + dv * 2
     per_head = (2 if cfg["s0_std"] > 0 else 1) * dk * dv * 4
     return cfg["B"] * cfg["H"] * (cfg["T"] * per_tok + per_head)
+
+
+def bwd_bytes(wl: workload.Workload) -> float:
+    """Inputs (q, k, v, g, b, w) and dO read once, the gradients written once, S0 and dS_T
+    read and dS0 written once per head (GDN-2, bf16 storage, fp32 g, dg and states)."""
+    dk, dv = wl.dk, wl.dv
+    per_tok = (2 * dk + dv) * 2 + dk * 4 + dk * 2 + dv * 2 + dv * 2    # q k v g b w dO
+    per_tok += (2 * dk + dv) * 2 + dk * 4 + dk * 2 + dv * 2            # dq dk dv dg db dw
+    return wl.units * per_tok + wl.B * wl.H * 3 * dk * dv * 4
+
+
+def bwd_flops(wl: workload.Workload) -> float:
+    """Dense products of the chunkwise backward (32-token chunks) per token-head:
+    24 C d + 20 d^2 (states 4C^2d + 4Cd^2, state gradient 4C^2d + 6Cd^2, per-chunk
+    gradients 16C^2d + 10Cd^2 per chunk of C tokens)."""
+    C, d = 32, max(wl.dk, wl.dv)
+    return wl.units * (24.0 * C * d + 20.0 * d * d)
+
+
+# fp32 FMA lanes of a B200 at its maximum SM clock: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
+ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def decode_bytes(cfg) -> float:
@@ -189,6 +212,8 @@ def rank_workload(name: str, rank: int):
         cfg = dict(workload.MIXER)
         cfg["seed"] = cfg["seed"] + 1000 * rank
         return cfg, cfg["mode"]
+    if name == "bwd_t4k":
+        name = "gdn2_t4k"
     base, mode = name, None
     for m in ("kda", "bonly", "wonly"):
         if name.endswith("_" + m):
@@ -237,6 +262,28 @@ def cpu_oracle_sample(name, target_cpu_s=15.0):
         dt = time.perf_counter() - t0
         return dict(value=n * c["T"] / dt, unit="token-heads/s", cores=1, kind="oracle",
                     sample=f"{n} sequence-heads x T={c['T']} of mixer_t4k, one after another")
+    if name == "bwd_t4k":
+        wl, mode = rank_workload(name, 0)
+        small = workload.Workload("sample", B=1, H=1, T=wl.T, dk=wl.dk, dv=wl.dv, chunk=wl.chunk,
+                                  dtype=wl.dtype, mode=wl.mode, seed=wl.seed, g_scale=wl.g_scale,
+                                  s0_std=wl.s0_std)
+        d = workload.make_inputs(small, mode=mode)
+        gen = torch.Generator().manual_seed(99)
+        dO = torch.randn(1, 1, wl.T, wl.dv, generator=gen).to(torch.bfloat16)
+        dST = torch.randn(1, 1, wl.dk, wl.dv, generator=gen) * 0.1
+        t0 = time.perf_counter()
+        oracle.bwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], dO, dST, mode=mode, nthreads=1)
+        t_head = time.perf_counter() - t0
+        n_heads = max(cores, int(round(target_cpu_s / max(t_head, 1e-3) / cores)) * cores)
+        n_heads = min(n_heads, wl.B * wl.H)
+        rep = lambda x: None if x is None else x.expand(n_heads, *x.shape[1:]).contiguous()
+        dd = {k: rep(d[k]) for k in ("q", "k", "v", "g", "b", "w", "S0")}
+        t0 = time.perf_counter()
+        oracle.bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["b"], dd["w"], dd["S0"], rep(dO), rep(dST), mode=mode,
+                   nthreads=cores)
+        dt = time.perf_counter() - t0
+        return dict(value=n_heads * wl.T / dt, unit="token-heads/s", cores=min(cores, n_heads), kind="oracle",
+                    sample=f"{n_heads} sequence-heads x T={wl.T} of bwd_t4k (adjoint oracle)")
     wl, mode = rank_workload(name, 0)
     T = wl.T
     small = workload.Workload("sample", B=1, H=1, T=T, dk=wl.dk, dv=wl.dv, chunk=wl.chunk,
@@ -287,6 +334,8 @@ def metric_name(name):
         return "decode step-heads/s (256 seqs x 16 heads, dk=dv=128); % HBM roofline"
     if name == "mixer_t4k":
         return "token-mixer fwd tokens/s per head·layer at T=4K (fused prologue/epilogue); % HBM roofline"
+    if name == "bwd_t4k":
+        return "chunked bwd tokens/s per head·layer at T=4K (dq, dk, dv, dg, db, dw, dS0); % fp32 ALU roofline"
     return "chunked fwd tokens/s per head·layer at T=4K; % tensor-pipe / HBM roofline"
 
 
@@ -301,6 +350,11 @@ def config_of(name, world):
         return {"workload": name, "B": c["B"], "H": c["H"], "T": c["T"], "dk": c["dk"], "dv": c["dv"],
                 "chunk": c["chunk"], "mode": c["mode"], "layout": "[B,T,H,D]", "inputs": "bf16 raw projections",
                 "state": "fp32", "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
+    if name == "bwd_t4k":
+        wl, mode = rank_workload(name, 0)
+        return {"workload": name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk, "dv": wl.dv, "chunk": 32,
+                "mode": mode, "inputs": wl.dtype, "state": "fp32", "grad": "dO bf16 N(0,1), dS_T N(0,0.1)",
+                "l2": "inputs larger than L2 (no flush)", "parallelism": f"replicas{world}"}
     wl, mode = rank_workload(name, 0)
     return {"workload": name, "B": wl.B, "H": wl.H, "T": wl.T, "dk": wl.dk, "dv": wl.dv,
             "chunk": wl.chunk, "mode": mode, "inputs": wl.dtype, "state": "fp32",
@@ -334,6 +388,27 @@ def run_ours(args, rank, world, local):
         units = c["B"] * c["H"] * c["T"]
         bytes_per_launch = mixer_bytes(c)
         launches_per_step = 1
+        unit = "token-heads/s"
+        nseg = 1
+    elif name == "bwd_t4k":
+        inp = workload.make_inputs(wl, mode=mode)
+        d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
+        gen = torch.Generator().manual_seed(99 + rank)
+        dO = torch.randn(wl.B, wl.H, wl.T, wl.dv, generator=gen).to(torch.bfloat16).to(dev)
+        dST = (torch.randn(wl.B, wl.H, wl.dk, wl.dv, generator=gen) * 0.1).to(dev)
+        ws = torch.empty(gdr.gdr_chunk_bwd_workspace(wl.B, wl.H, wl.T, wl.dk, wl.dv), dtype=torch.uint8,
+                         device=dev)
+        grads = dict(dq=torch.empty_like(d["q"]), dk=torch.empty_like(d["k"]), dv=torch.empty_like(d["v"]),
+                     dg=torch.empty_like(d["g"]), db=torch.empty_like(d["b"]), dw=torch.empty_like(d["w"]),
+                     dS0=torch.empty_like(d["S0"]))
+
+        def fwd():
+            gdr.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], dO, dST, mode=mode,
+                          workspace=ws, out=grads)
+        step = fwd
+        units = wl.units
+        bytes_per_launch = bwd_bytes(wl)
+        launches_per_step = 3
         unit = "token-heads/s"
         nseg = 1
     elif name == "decode":
@@ -422,7 +497,35 @@ def run_ours(args, rank, world, local):
 
     # end to end through the public API with host buffers (pinned), copies inside
     e2e = None
-    if not args.no_e2e and name == "mixer_t4k":
+    if not args.no_e2e and name == "bwd_t4k":
+        hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
+        dOh, dSTh = dO.cpu().pin_memory(), dST.cpu().pin_memory()
+        outh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in grads.items()}
+        h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v)) + \
+            dOh.numel() * dOh.element_size() + dSTh.numel() * dSTh.element_size()
+        d2h = sum(x.numel() * x.element_size() for x in outh.values())
+        n_e2e = max(1, min(args.steps, 3))
+
+        def call():
+            x = {k: (v.to(dev, non_blocking=True) if torch.is_tensor(v) else v) for k, v in hin.items()}
+            g_ = gdr.chunk_bwd(x["q"], x["k"], x["v"], x["g"], x["b"], x["w"], x["S0"],
+                               dOh.to(dev, non_blocking=True), dSTh.to(dev, non_blocking=True), mode=mode,
+                               workspace=ws)
+            for k_, v_ in g_.items():
+                outh[k_].copy_(v_, non_blocking=True)
+        call()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
+        e2e = {"value": units * world / (e2e_ms * 1e-3), "unit": unit,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    elif not args.no_e2e and name == "mixer_t4k":
         c = wl
         hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
         h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v))
@@ -477,6 +580,10 @@ def run_ours(args, rank, world, local):
     elif name == "mixer_t4k":
         launch_ms = kern_ms
         kname = "gdr chunk_tc_kernel<mixer> (tcgen05, fused prologue/epilogue)"
+    elif name == "bwd_t4k":
+        # one step = the whole backward (states, state gradient, per-chunk gradients)
+        launch_ms = kern_ms
+        kname = "gdr chunk_simt_kernel + bwd_dstate_kernel + bwd_chunk_kernel (backward, 3 launches)"
     else:
         # one step = the whole forward; with a sequence split it is three launches
         # (state pass, combine, output pass) and the step is the unit of the roofline
@@ -487,7 +594,14 @@ def run_ours(args, rank, world, local):
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic_for(name, kname), "peak_source": f"{peak_src} hbm_gbs",
             "kernel": kname}
-    if name not in ("decode", "mixer_t4k"):
+    if name == "bwd_t4k":
+        fl = bwd_flops(wl) / (launch_ms * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": fl, "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
+                "frac": fl / ALU_FP32_TFLOPS, "traffic": None,
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz", "kernel": kname,
+                "hbm_context": {"bytes_per_step": bytes_per_launch, "achieved_gbs": achieved,
+                                "frac": achieved / hbm}}
+    if name not in ("decode", "mixer_t4k", "bwd_t4k"):
         fl = chunk_flops(wl)
         roof["tensor_context"] = {"flops_per_launch": fl,
                                   "achieved_tflops": fl / (launch_ms * 1e-3) / 1e12,
@@ -496,7 +610,8 @@ def run_ours(args, rank, world, local):
     line = {"metric": metric_name(name), "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if (name in ("decode", "mixer_t4k") or wl.dtype == "bf16") else "f32",
+            "dtype": "f32" if name == "bwd_t4k" else
+                     ("bf16" if (name in ("decode", "mixer_t4k") or wl.dtype == "bf16") else "f32"),
             "data": "synthetic", "config": config_of(name, world), "roofline": roof,
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "wall_total_ms": total_ms}
@@ -554,7 +669,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gdn2_t4k",
                     choices=["gdn2_t4k", "gdn_t2k", "gdn2_t16k", "gdn2_t16k_kda", "gdn2_tiny", "decode",
-                             "gdn2_t4k_bonly", "gdn2_t4k_wonly", "mixer_t4k"])
+                             "gdn2_t4k_bonly", "gdn2_t4k_wonly", "mixer_t4k", "bwd_t4k"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-cpu-s", type=float, default=15.0)

@@ -223,6 +223,38 @@ gdr_status_t gdr_mixer_fwd(const void *q, const void *k, const void *v, const fl
                            void *stream);
 
 /*
+ * gdr_chunk_bwd -- the gate-aware backward of gdr_chunk_fwd.
+ *
+ * Gradients of L = sum_t <o_t, dO_t> + <S_T, dS_T> with respect to q, k, v, g_log, b, w
+ * and S0, for the forward of gdr_chunk_fwd on the same inputs (the pages' training path
+ * runs the chunkwise WY algorithm with a gate-aware backward: Gated DeltaNet-2 Review
+ * §4-3; Gated DeltaNet-2 Q&A page, Q4).  The backward differentiates the chunkwise form
+ * in 32-token chunks: it recomputes the chunk-start states, walks the chunks backwards
+ * for the state gradient, then forms every chunk's input gradients in parallel, in fp32
+ * on CUDA cores.  Equal to the adjoint of the sequential recurrence up to rounding.
+ *
+ *   dO      [B,H,T,dv], element type `dtype`.       dS_T  fp32 [B,H,dk,dv] or NULL (= 0).
+ *   dq, dk  [B,H,T,dk]; dv [B,H,T,dv]; db, dw shaped like b, w; all of type `dtype`.
+ *           Tied and scalar modes receive the summed gradient of the shared parameter
+ *           (KDA, GDN: d beta = sum_c db + sum_v dw in db; b-only: the scalar write gate's
+ *           gradient in dw; w-only: the scalar erase gate's in db).  dw may be NULL in KDA
+ *           and GDN.
+ *   dg      fp32, shaped like g_log.                 dS0   fp32 [B,H,dk,dv] or NULL.
+ *   workspace  caller-owned device memory of at least gdr_chunk_bwd_workspace(B, H, T, dk,
+ *           dv) bytes, 16-byte aligned (GDR_ERR_WORKSPACE otherwise); scratch, no
+ *           initialisation needed.  Outputs must not overlap inputs or the workspace.
+ *   Sizes as gdr_chunk_fwd (dk, dv in {16, 32, 64, 128}); T == 0 writes dS0 = dS_T (or 0).
+ */
+unsigned long long gdr_chunk_bwd_workspace(int B, int H, int T, int dk, int dv);
+
+gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *v, const float *g_log,
+                           const void *b, const void *w, const float *S0, const void *dO,
+                           const float *dS_T, void *dq, void *dk_, void *dv_, float *dg,
+                           void *db, void *dw, float *dS0, int B, int H, int T, int dk, int dv,
+                           gdr_mode_t mode, gdr_dtype_t dtype, void *workspace,
+                           unsigned long long workspace_bytes, void *stream);
+
+/*
  * gdr_last_device_error -- read and clear the device-side error word.
  *
  * Synchronises `stream`, then returns GDR_ERR_TIMEOUT if a bounded wait inside a

@@ -7,9 +7,10 @@ PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raise
 
 Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
 gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
-gdr_mixer_fwd, gdr_decode_step, gdr_last_device_error, gdr_status_string.
+gdr_mixer_fwd, gdr_chunk_bwd, gdr_chunk_bwd_workspace, gdr_decode_step,
+gdr_last_device_error, gdr_status_string.
 Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
-decode_step.
+chunk_bwd, decode_step.
 """
 from __future__ import annotations
 
@@ -53,6 +54,10 @@ def lib():
         L.gdr_chunk_fwd_split_workspace.restype = ctypes.c_ulonglong
         L.gdr_mixer_fwd.argtypes = [vp] * 11 + [ci] * 9 + [ctypes.c_float] * 2 + [vp]
         L.gdr_mixer_fwd.restype = ci
+        L.gdr_chunk_bwd.argtypes = [vp] * 16 + [ci] * 7 + [vp, ctypes.c_ulonglong, vp]
+        L.gdr_chunk_bwd.restype = ci
+        L.gdr_chunk_bwd_workspace.argtypes = [ci] * 5
+        L.gdr_chunk_bwd_workspace.restype = ctypes.c_ulonglong
         L.gdr_decode_step.argtypes = [vp] * 8 + [ci] * 6 + [vp]
         L.gdr_decode_step.restype = ci
         L.gdr_last_device_error.argtypes = [vp]
@@ -93,6 +98,16 @@ def gdr_mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0, y, S_T, B, H, T, dk, 
                   dtype, layout, b_range, eps, stream):
     return lib().gdr_mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0, y, S_T, B, H, T, dk, dv,
                                chunk, mode, dtype, layout, b_range, eps, stream)
+
+
+def gdr_chunk_bwd(q, k, v, g_log, b, w, S0, dO, dS_T, dq, dk_, dv_, dg, db, dw, dS0, B, H, T, dk, dv,
+                  mode, dtype, workspace, workspace_bytes, stream):
+    return lib().gdr_chunk_bwd(q, k, v, g_log, b, w, S0, dO, dS_T, dq, dk_, dv_, dg, db, dw, dS0, B, H,
+                               T, dk, dv, mode, dtype, workspace, workspace_bytes, stream)
+
+
+def gdr_chunk_bwd_workspace(B, H, T, dk, dv):
+    return lib().gdr_chunk_bwd_workspace(B, H, T, dk, dv)
 
 
 def gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, stream):
@@ -281,6 +296,47 @@ def mixer_fwd_host(q, k, v, xg, xb, xw, z, norm_weight, S0=None, *, mode="gdn2",
                torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True))
     out[0].copy_(y_d, non_blocking=True)
     out[1].copy_(S_d, non_blocking=True)
+    return out
+
+
+def chunk_bwd(q, k, v, g, b, w, S0, dO, dS_T=None, *, mode="gdn2", workspace=None, out=None,
+              return_dS0=True):
+    """Gradients of L = sum(o * dO) + sum(S_T * dS_T) through chunk_fwd (gdr_chunk_bwd).
+    Inputs as chunk_fwd; dO like o, dS_T fp32 [B,H,dk,dv] or None.  Returns a dict with dq,
+    dk, dv, db, dw (None when the mode has no w) in the input dtype, dg and dS0 in fp32,
+    each shaped like its input.  The workspace (uint8 CUDA tensor of at least
+    gdr_chunk_bwd_workspace bytes) is allocated here when not given."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    if dt not in DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    gshape, bshape, wshape = _gate_shapes(mode, (B, H, T), dk, dv)
+    for t, name, shape, tdt in ((q, "q", (B, H, T, dk), dt), (k, "k", (B, H, T, dk), dt),
+                                (v, "v", (B, H, T, dv), dt), (g, "g", gshape, torch.float32),
+                                (b, "b", bshape, dt), (dO, "dO", (B, H, T, dv), dt)):
+        _check(t, name, shape, tdt, dev)
+    if wshape is not None:
+        _check(w, "w", wshape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    if dS_T is not None:
+        _check(dS_T, "dS_T", (B, H, dk, dv), torch.float32, dev)
+    need = gdr_chunk_bwd_workspace(B, H, T, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+                   dg=torch.empty_like(g), db=torch.empty_like(b),
+                   dw=None if wshape is None else torch.empty_like(w),
+                   dS0=torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev) if return_dS0 else None)
+    rc = gdr_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b), _ptr(w) if wshape is not None else None,
+                       _ptr(S0), _ptr(dO), _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                       _ptr(out["dg"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out["dS0"]), B, H, T, dk, dv,
+                       MODES[mode], DTYPES[dt], _ptr(workspace), workspace.numel() * workspace.element_size(),
+                       _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_bwd")
     return out
 
 

@@ -1,0 +1,519 @@
+// bwd.cu -- chunkwise backward of the gated delta rule on CUDA cores (fp32 arithmetic).
+//
+// The gradient of L = sum_t <o_t, dO_t> + <S_T, dS_T> with respect to q, k, v, the decay,
+// both gates and S0 (the gate-aware backward of Gated DeltaNet-2 Review §4-3 and the
+// Gated DeltaNet-2 Q&A page, Q4).  It differentiates the chunkwise WY form of the forward
+// (Gated DeltaNet-2 Review §3-2.5), chunk by chunk, in 32-token chunks.  For one chunk,
+// with gamma the chunk-local cumulative log-decay, F_ij = exp(gamma_i - gamma_j) per key
+// channel, Kh = b.k.e^gamma, Qg = q.e^gamma, Ke = k.e^(gamma_C - gamma):
+//
+//   forward   A = strict_lower(sum_c b_i k_i k_j F_ij)   T = (I + A)^-1
+//             P = lower_incl(sum_c q_i k_j F_ij)         R = w.v - Kh S     E = T R
+//             O = Qg S + P E                             S' = e^gamma_C S + Ke^T E
+//   backward  dE = P^T dO + Ke dS'        dR = T^T dE      dv = dR.w   dw = dR.v
+//             dS = e^gamma_C dS' + Qg^T dO - Kh^T dR
+//             dP = lower_incl(dO E^T)     dA = strict_lower(-T^T (dE R^T) T^T)
+//   and q, k, b, gamma collect the products' terms: dO S^T through Qg, -dR S^T through
+//   Kh, E dS'^T through Ke, dP and dA through the pair decays F; the decay gradient is
+//   the reverse cumulative sum of the gamma gradient over the chunk.
+//
+// Three launches:
+//   1. the chunk-start states S_c of every chunk (the CUDA-core forward kernel, writing
+//      its checkpoints and no output) -> workspace;
+//   2. bwd_dstate_kernel: the state gradient dS' entering every chunk from above, walking
+//      the chunks backwards (sequential, parallel over value-column slices) -> workspace,
+//      and dS0;
+//   3. bwd_chunk_kernel: every chunk in parallel, from S_c and dS' -> dq, dk, dv, dg, db, dw.
+// Pair decays are formed as exp(gamma_i - gamma_j) with i >= j, never as a product of two
+// exponentials, so no factor overflows for a forgetting decay.
+#include "common.cuh"
+
+namespace gdr {
+namespace {
+
+constexpr int C = kBwdChunk;
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float ld_b(const BwdArgs &a, size_t tk, int c) {   // erase gate b_tc
+    return mode_b_vec(a.mode) ? ld_elem(a.b, tk * a.dk_ + c, a.dtype) : ld_elem(a.b, tk, a.dtype);
+}
+__device__ __forceinline__ float ld_w(const BwdArgs &a, size_t tk, int j) {   // write gate w_tj
+    if (mode_w_vec(a.mode)) return ld_elem(a.w, tk * a.dv_ + j, a.dtype);
+    return ld_elem(a.mode == GDR_MODE_BONLY ? a.w : a.b, tk, a.dtype);
+}
+__device__ __forceinline__ float ld_g(const BwdArgs &a, size_t tk, int c) {
+    return a.mode == GDR_MODE_GDN ? a.g[tk] : a.g[tk * a.dk_ + c];
+}
+
+// The chunk's raw q, k, b (expanded to dk channels) and gamma into shared memory ([C][dk]
+// each; tokens past the end are zero, so they neither decay nor write), gamma_C, and the
+// C x C matrices A (strictly lower), P (lower incl.) and T = (I + A)^-1.  All threads of
+// the block call it; it ends with a barrier.
+__device__ void chunk_core(const BwdArgs &a, size_t tok0, int n, float *qq, float *kk, float *bb,
+                           float *gm, float *gC, float *Am, float *Tm, float *Pm) {
+    const int dk = a.dk_, tid = threadIdx.x, nth = blockDim.x;
+    for (int idx = tid; idx < C * dk; idx += nth) {
+        const int t = idx / dk, d = idx - t * dk;
+        float qv = 0.f, kv = 0.f, bv = 0.f, gv = 0.f;
+        if (t < n) {
+            const size_t tk = tok0 + t;
+            qv = ld_elem(a.q, tk * dk + d, a.dtype);
+            kv = ld_elem(a.k, tk * dk + d, a.dtype);
+            bv = ld_b(a, tk, d);
+            gv = ld_g(a, tk, d);
+        }
+        qq[idx] = qv;
+        kk[idx] = kv;
+        bb[idx] = bv;
+        gm[idx] = gv;
+    }
+    __syncthreads();
+    for (int d = tid; d < dk; d += nth) {
+        float acc = 0.f;
+        for (int t = 0; t < C; ++t) {
+            acc += gm[t * dk + d];
+            gm[t * dk + d] = acc;
+        }
+        gC[d] = acc;
+    }
+    __syncthreads();
+    constexpr int npairs = C * (C + 1) / 2;
+    for (int p = tid; p < npairs; p += nth) {
+        int i = (int)((sqrtf(8.f * p + 1.f) - 1.f) * 0.5f);
+        while (i * (i + 1) / 2 > p) --i;
+        while ((i + 1) * (i + 2) / 2 <= p) ++i;
+        const int j = p - i * (i + 1) / 2;
+        float av = 0.f, pv = 0.f;
+        for (int cc = 0; cc < dk; ++cc) {
+            const int c = (cc + (tid & 31)) & (dk - 1);   // staggered: no bank conflicts
+            const float e = kk[j * dk + c] * __expf(gm[i * dk + c] - gm[j * dk + c]);
+            av = fmaf(bb[i * dk + c] * kk[i * dk + c], e, av);
+            pv = fmaf(qq[i * dk + c], e, pv);
+        }
+        Am[i * C + j] = (j < i) ? av : 0.f;
+        Am[j * C + i] = 0.f;
+        Pm[i * C + j] = pv;
+        if (j < i) Pm[j * C + i] = 0.f;
+    }
+    __syncthreads();
+    for (int j = tid; j < C; j += nth) {   // T: one column per thread, forward substitution
+        for (int i = 0; i <= j; ++i) Tm[i * C + j] = (i == j) ? 1.f : 0.f;
+        for (int i = j + 1; i < C; ++i) {
+            float acc = 0.f;
+            for (int m = j; m < i; ++m) acc = fmaf(Am[i * C + m], Tm[m * C + j], acc);
+            Tm[i * C + j] = -acc;
+        }
+    }
+    __syncthreads();
+}
+
+__host__ __device__ inline int dslice(int dv) { return dv < 32 ? dv : 32; }
+
+__host__ __device__ inline size_t dstate_smem_floats(int dk, int VS) {
+    return 4 * (size_t)C * dk + dk + 3 * (size_t)C * C + (size_t)dk * VS + 3 * (size_t)C * VS;
+}
+
+// Launch 2: the state gradient, chunks in reverse.  One CTA per (sequence-head, slice of VS
+// value columns): the columns of dS are independent of one another.
+__global__ void __launch_bounds__(kThreads) bwd_dstate_kernel(BwdArgs a) {
+    const int dk = a.dk_, dv = a.dv_, T = a.T;
+    const int VS = dslice(dv);
+    const int bh = blockIdx.x, v0 = blockIdx.y * VS;
+    const int tid = threadIdx.x, nth = blockDim.x;
+    extern __shared__ float sm[];
+    float *qq = sm, *kk = qq + C * dk, *bb = kk + C * dk, *gm = bb + C * dk;
+    float *gC = gm + C * dk;
+    float *Am = gC + dk, *Tm = Am + C * C, *Pm = Tm + C * C;
+    float *dS = Pm + C * C;          // [dk][VS]: gradient with respect to the chunk's end state
+    float *dO = dS + dk * VS;        // [C][VS]
+    float *dE = dO + C * VS;         // [C][VS]
+    float *dR = dE + C * VS;         // [C][VS]
+    const int nc = (T + C - 1) / C;
+    const size_t tok0 = (size_t)bh * T;
+
+    for (int idx = tid; idx < dk * VS; idx += nth) {
+        const int d = idx / VS, j = idx - d * VS;
+        dS[idx] = a.dST ? a.dST[((size_t)bh * dk + d) * dv + v0 + j] : 0.f;
+    }
+    for (int c = nc - 1; c >= 0; --c) {
+        const int t0 = c * C, n = min(C, T - t0);
+        __syncthreads();
+        float *dst = a.ws_dstates + ((size_t)bh * nc + c) * dk * dv + v0;
+        for (int idx = tid; idx < dk * VS; idx += nth) {
+            const int d = idx / VS, j = idx - d * VS;
+            dst[(size_t)d * dv + j] = dS[idx];
+        }
+        for (int idx = tid; idx < C * VS; idx += nth) {
+            const int t = idx / VS, j = idx - t * VS;
+            dO[idx] = t < n ? ld_elem(a.dO, (tok0 + t0 + t) * dv + v0 + j, a.dtype) : 0.f;
+        }
+        chunk_core(a, tok0 + t0, n, qq, kk, bb, gm, gC, Am, Tm, Pm);
+        // decayed operands in place: Ke = k e^(gamma_C - gamma), Qg = q e^gamma, Kh = b k e^gamma
+        for (int idx = tid; idx < C * dk; idx += nth) {
+            const int d = idx % dk;
+            const float gam = gm[idx], e = __expf(gam);
+            bb[idx] *= kk[idx] * e;
+            qq[idx] *= e;
+            kk[idx] *= __expf(gC[d] - gam);
+        }
+        __syncthreads();
+        // dE = P^T dO + Ke dS
+        for (int idx = tid; idx < C * VS; idx += nth) {
+            const int j = idx / VS, v = idx - j * VS;
+            float acc = 0.f;
+            for (int t = j; t < C; ++t) acc = fmaf(Pm[t * C + j], dO[t * VS + v], acc);
+            for (int d = 0; d < dk; ++d) acc = fmaf(kk[j * dk + d], dS[d * VS + v], acc);
+            dE[idx] = acc;
+        }
+        __syncthreads();
+        // dR = T^T dE  (T lower triangular)
+        for (int idx = tid; idx < C * VS; idx += nth) {
+            const int i = idx / VS, v = idx - i * VS;
+            float acc = 0.f;
+            for (int j = i; j < C; ++j) acc = fmaf(Tm[j * C + i], dE[j * VS + v], acc);
+            dR[idx] = acc;
+        }
+        __syncthreads();
+        // dS <- e^gamma_C dS + Qg^T dO - Kh^T dR   (the gradient with respect to S_c)
+        for (int idx = tid; idx < dk * VS; idx += nth) {
+            const int d = idx / VS, v = idx - d * VS;
+            float acc = __expf(gC[d]) * dS[idx];
+            for (int t = 0; t < C; ++t) {
+                acc = fmaf(qq[t * dk + d], dO[t * VS + v], acc);
+                acc = fmaf(-bb[t * dk + d], dR[t * VS + v], acc);
+            }
+            dS[idx] = acc;
+        }
+    }
+    __syncthreads();
+    if (a.dS0) {
+        for (int idx = tid; idx < dk * VS; idx += nth) {
+            const int d = idx / VS, j = idx - d * VS;
+            a.dS0[((size_t)bh * dk + d) * dv + v0 + j] = dS[idx];
+        }
+    }
+}
+
+__host__ __device__ inline size_t chunk_smem_floats(int dk, int dv) {
+    return 5 * (size_t)C * dk + 2 * (size_t)dk + 5 * (size_t)C * C + 3 * (size_t)C * dv +
+           (size_t)dk * (dv + 1) + 3 * (size_t)C;
+}
+
+// Launch 3: every chunk in parallel.  Thread (c = tid % dk, group tid / dk) owns key channel
+// c of RPG consecutive tokens and accumulates their dq, dk, db and d gamma in registers.
+template <int RPG>
+__global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
+    const int dk = a.dk_, dv = a.dv_, T = a.T;
+    const int nc = (T + C - 1) / C;
+    const int bh = blockIdx.x / nc, c_idx = blockIdx.x - bh * nc;
+    const int t0 = c_idx * C, n = min(C, T - t0);
+    const size_t tok0 = (size_t)bh * T + t0;
+    const int tid = threadIdx.x, nth = blockDim.x;
+    const int ch = tid % dk, i0 = (tid / dk) * RPG;   // this thread's channel and first token
+    const int SLD = dv + 1;                            // padded row stride of the state tile
+
+    extern __shared__ float sm[];
+    float *qq = sm, *kk = qq + C * dk, *bb = kk + C * dk, *gm = bb + C * dk;
+    float *ex = gm + C * dk;         // [C][dk]: e^gamma, later Ke = k e^(gamma_C - gamma)
+    float *gC = ex + C * dk, *dgC = gC + dk;
+    float *Am = dgC + dk, *Tm = Am + C * C, *Pm = Tm + C * C, *dA = Pm + C * C, *dP = dA + C * C;
+    float *X1 = dP + C * C;          // [C][dv]: dO, then dR
+    float *X2 = X1 + C * dv;         // [C][dv]: w.v, then R
+    float *X3 = X2 + C * dv;         // [C][dv]: E, then dE
+    float *Ss = X3 + C * dv;         // [dk][dv+1]: S_c, then dS', then S_c
+    float *fb = Ss + dk * SLD;       // [C]: folded scalar erase-gate gradient
+    float *fw = fb + C;              // [C]: folded scalar write-gate gradient
+    float *fg = fw + C;              // [C]: folded scalar decay gradient
+    const float *Sg = a.ws_states + ((size_t)bh * nc + c_idx) * dk * dv;
+    const float *dSg = a.ws_dstates + ((size_t)bh * nc + c_idx) * dk * dv;
+
+    float aq[RPG], ak[RPG], ab[RPG], ag[RPG];
+#pragma unroll
+    for (int r = 0; r < RPG; ++r) aq[r] = ak[r] = ab[r] = ag[r] = 0.f;
+
+    // ---- inputs, S_c, and the chunk's A, P, T ----
+    for (int idx = tid; idx < C * dv; idx += nth) {
+        const int t = idx / dv, j = idx - t * dv;
+        float x = 0.f, o = 0.f;
+        if (t < n) {
+            x = ld_w(a, tok0 + t, j) * ld_elem(a.v, (tok0 + t) * dv + j, a.dtype);
+            o = ld_elem(a.dO, (tok0 + t) * dv + j, a.dtype);
+        }
+        X2[idx] = x;
+        X1[idx] = o;
+    }
+    for (int idx = tid; idx < dk * dv; idx += nth) {
+        const int d = idx / dv, j = idx - d * dv;
+        Ss[d * SLD + j] = Sg[idx];
+    }
+    for (int i = tid; i < C; i += nth) fb[i] = fw[i] = fg[i] = 0.f;
+    for (int d = tid; d < dk; d += nth) dgC[d] = 0.f;
+    chunk_core(a, tok0, n, qq, kk, bb, gm, gC, Am, Tm, Pm);
+    for (int idx = tid; idx < C * dk; idx += nth) ex[idx] = __expf(gm[idx]);
+    __syncthreads();
+    // ---- R = w.v - Kh S ----
+    for (int idx = tid; idx < C * dv; idx += nth) {
+        const int i = idx / dv, j = idx - i * dv;
+        float acc = X2[idx];
+        for (int d = 0; d < dk; ++d) acc = fmaf(-bb[i * dk + d] * kk[i * dk + d] * ex[i * dk + d], Ss[d * SLD + j], acc);
+        X2[idx] = acc;
+    }
+    __syncthreads();
+    // ---- E = T R;  DY = dO S^T (into dq and d gamma) ----
+    for (int idx = tid; idx < C * dv; idx += nth) {
+        const int i = idx / dv, j = idx - i * dv;
+        float acc = 0.f;
+        for (int m = 0; m <= i; ++m) acc = fmaf(Tm[i * C + m], X2[m * dv + j], acc);
+        X3[idx] = acc;
+    }
+    {
+        float y[RPG];
+#pragma unroll
+        for (int r = 0; r < RPG; ++r) y[r] = 0.f;
+        for (int j = 0; j < dv; ++j) {
+            const float s = Ss[ch * SLD + j];
+#pragma unroll
+            for (int r = 0; r < RPG; ++r) y[r] = fmaf(X1[(i0 + r) * dv + j], s, y[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < RPG; ++r) {
+            const int i = i0 + r;
+            const float e = ex[i * dk + ch];
+            aq[r] = fmaf(e, y[r], aq[r]);
+            ag[r] = fmaf(qq[i * dk + ch] * e, y[r], ag[r]);
+        }
+    }
+    __syncthreads();
+    // ---- dP = lower_incl(dO E^T); dS' replaces S_c; rowsum(S_c . dS') into d gamma_C ----
+    for (int p = tid; p < C * C; p += nth) {
+        const int t = p / C, j = p - t * C;
+        float acc = 0.f;
+        if (j <= t)
+            for (int v0 = 0; v0 < dv; ++v0) {
+                const int v = (v0 + (tid & 31)) & (dv - 1);   // staggered: no bank conflicts
+                acc = fmaf(X1[t * dv + v], X3[j * dv + v], acc);
+            }
+        dP[p] = acc;
+    }
+    for (int idx = tid; idx < dk * dv; idx += nth) {
+        const int d = idx / dv, j = idx - d * dv;
+        Ss[d * SLD + j] = dSg[idx];
+    }
+    if (tid < dk) {
+        float acc = 0.f;
+        for (int j = 0; j < dv; ++j) acc = fmaf(Sg[(size_t)tid * dv + j], dSg[(size_t)tid * dv + j], acc);
+        dgC[tid] = __expf(gC[tid]) * acc;
+    }
+    __syncthreads();
+    // ---- DK = E dS'^T (into dk, d gamma, d gamma_C), through Ke = k e^(gamma_C - gamma) ----
+    {
+        float y[RPG];
+#pragma unroll
+        for (int r = 0; r < RPG; ++r) y[r] = 0.f;
+        for (int j = 0; j < dv; ++j) {
+            const float s = Ss[ch * SLD + j];
+#pragma unroll
+            for (int r = 0; r < RPG; ++r) y[r] = fmaf(X3[(i0 + r) * dv + j], s, y[r]);
+        }
+        float part = 0.f;
+#pragma unroll
+        for (int r = 0; r < RPG; ++r) {
+            const int i = i0 + r;
+            const float f = __expf(gC[ch] - gm[i * dk + ch]);
+            const float kf = kk[i * dk + ch] * f;
+            ak[r] = fmaf(f, y[r], ak[r]);
+            ag[r] = fmaf(-kf, y[r], ag[r]);
+            part = fmaf(kf, y[r], part);
+        }
+        atomicAdd(&dgC[ch], part);
+    }
+    __syncthreads();
+    // Ke in place of e^gamma (e^gamma is recomputed where still needed)
+    for (int idx = tid; idx < C * dk; idx += nth) {
+        const int d = idx % dk;
+        ex[idx] = kk[idx] * __expf(gC[d] - gm[idx]);
+    }
+    __syncthreads();
+    // ---- dE = P^T dO + Ke dS'  (E is no longer needed) ----
+    for (int idx = tid; idx < C * dv; idx += nth) {
+        const int j = idx / dv, v = idx - j * dv;
+        float acc = 0.f;
+        for (int t = j; t < C; ++t) acc = fmaf(Pm[t * C + j], X1[t * dv + v], acc);
+        for (int d = 0; d < dk; ++d) acc = fmaf(ex[j * dk + d], Ss[d * SLD + v], acc);
+        X3[idx] = acc;
+    }
+    __syncthreads();
+    // ---- dR = T^T dE (dO is no longer needed); dT = dE R^T into dA ----
+    for (int idx = tid; idx < C * dv; idx += nth) {
+        const int i = idx / dv, v = idx - i * dv;
+        float acc = 0.f;
+        for (int j = i; j < C; ++j) acc = fmaf(Tm[j * C + i], X3[j * dv + v], acc);
+        X1[idx] = acc;
+    }
+    for (int p = tid; p < C * C; p += nth) {
+        const int i = p / C, j = p - i * C;
+        float acc = 0.f;
+        for (int v0 = 0; v0 < dv; ++v0) {
+            const int v = (v0 + (tid & 31)) & (dv - 1);
+            acc = fmaf(X3[i * dv + v], X2[j * dv + v], acc);
+        }
+        dA[p] = acc;
+    }
+    __syncthreads();
+    // ---- dA = strict_lower(-T^T dT T^T): M = dT T^T into Am (A itself is done with) ----
+    for (int p = tid; p < C * C; p += nth) {
+        const int i = p / C, j = p - i * C;
+        float acc = 0.f;
+        for (int m0 = 0; m0 < C; ++m0) {
+            const int m = (m0 + (tid & 31)) & (C - 1);
+            if (m <= j) acc = fmaf(dA[i * C + m], Tm[j * C + m], acc);
+        }
+        Am[p] = acc;
+    }
+    __syncthreads();
+    for (int p = tid; p < C * C; p += nth) {
+        const int i = p / C, j = p - i * C;
+        float acc = 0.f;
+        if (j < i)
+            for (int m = i; m < C; ++m) acc = fmaf(Tm[m * C + i], Am[m * C + j], acc);
+        dA[p] = -acc;
+    }
+    // ---- dv = dR.w, dw = dR.v (scalar write gates fold over the value channels); S_c back ----
+    for (int idx = tid; idx < C * dv; idx += nth) {
+        const int t = idx / dv, j = idx - t * dv;
+        if (t < n) {
+            const size_t tk = tok0 + t;
+            const float r = X1[idx];
+            st_elem(a.dv, tk * dv + j, a.dtype, r * ld_w(a, tk, j));
+            const float gw = r * ld_elem(a.v, tk * dv + j, a.dtype);
+            if (mode_w_vec(a.mode)) st_elem(a.dw, tk * dv + j, a.dtype, gw);
+            else atomicAdd(&fw[t], gw);
+        }
+    }
+    for (int idx = tid; idx < dk * dv; idx += nth) {
+        const int d = idx / dv, j = idx - d * dv;
+        Ss[d * SLD + j] = Sg[idx];
+    }
+    __syncthreads();
+    // ---- DX = dR S^T (through Kh = b k e^gamma, with a minus sign: R = w.v - Kh S) ----
+    {
+        float y[RPG];
+#pragma unroll
+        for (int r = 0; r < RPG; ++r) y[r] = 0.f;
+        for (int j = 0; j < dv; ++j) {
+            const float s = Ss[ch * SLD + j];
+#pragma unroll
+            for (int r = 0; r < RPG; ++r) y[r] = fmaf(X1[(i0 + r) * dv + j], s, y[r]);
+        }
+#pragma unroll
+        for (int r = 0; r < RPG; ++r) {
+            const int i = i0 + r;
+            const float e = __expf(gm[i * dk + ch]);
+            const float kv = kk[i * dk + ch], bv = bb[i * dk + ch];
+            ab[r] = fmaf(-kv * e, y[r], ab[r]);
+            ak[r] = fmaf(-bv * e, y[r], ak[r]);
+            ag[r] = fmaf(-bv * kv * e, y[r], ag[r]);
+        }
+    }
+    // ---- pair terms of P and A, exact decays F_ij = exp(gamma_i - gamma_j), i >= j ----
+#pragma unroll
+    for (int r = 0; r < RPG; ++r) {
+        const int i = i0 + r;
+        const float gi = gm[i * dk + ch], qi = qq[i * dk + ch], ki = kk[i * dk + ch], bi = bb[i * dk + ch];
+        float sq = 0.f, sk = 0.f, sb = 0.f, sg = 0.f;
+        for (int j = 0; j <= i; ++j) {   // row terms: token i pairs with earlier tokens j
+            const float f = __expf(gi - gm[j * dk + ch]);
+            const float kj = kk[j * dk + ch] * f;
+            const float p = dP[i * C + j], al = dA[i * C + j];
+            sq = fmaf(p, kj, sq);
+            sk = fmaf(al * bi, kj, sk);
+            sb = fmaf(al * ki, kj, sb);
+            sg = fmaf(p * qi + al * bi * ki, kj, sg);
+        }
+        float ck = 0.f, cg = 0.f;
+        for (int m = i; m < C; ++m) {     // column terms: token i pairs with later tokens m
+            const float f = __expf(gm[m * dk + ch] - gi);
+            const float u = (dP[m * C + i] * qq[m * dk + ch] + dA[m * C + i] * bb[m * dk + ch] * kk[m * dk + ch]) * f;
+            ck += u;
+            cg = fmaf(-u, ki, cg);
+        }
+        aq[r] += sq;
+        ak[r] += sk + ck;
+        ab[r] += sb;
+        ag[r] += sg + cg;
+    }
+    __syncthreads();
+    // ---- d gamma -> d g (reverse cumulative sum over the chunk, gamma_C on the last token) ----
+#pragma unroll
+    for (int r = 0; r < RPG; ++r) qq[(i0 + r) * dk + ch] = ag[r];
+    __syncthreads();
+    for (int d = tid; d < dk; d += nth) {
+        float acc = dgC[d];
+        for (int t = C - 1; t >= 0; --t) {
+            acc += qq[t * dk + d];
+            qq[t * dk + d] = acc;
+        }
+    }
+    __syncthreads();
+    // ---- outputs ----
+    const bool scalar_b = !mode_b_vec(a.mode), scalar_g = a.mode == GDR_MODE_GDN;
+#pragma unroll
+    for (int r = 0; r < RPG; ++r) {
+        const int i = i0 + r;
+        if (i < n) {
+            const size_t tk = tok0 + i;
+            st_elem(a.dq, tk * dk + ch, a.dtype, aq[r]);
+            st_elem(a.dk, tk * dk + ch, a.dtype, ak[r]);
+            if (scalar_b) atomicAdd(&fb[i], ab[r]);
+            else st_elem(a.db, tk * dk + ch, a.dtype, ab[r]);
+            if (scalar_g) atomicAdd(&fg[i], qq[i * dk + ch]);
+            else a.dg[tk * dk + ch] = qq[i * dk + ch];
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += nth) {
+        const size_t tk = tok0 + i;
+        const bool tied = a.mode == GDR_MODE_KDA || a.mode == GDR_MODE_GDN;
+        if (scalar_b) st_elem(a.db, tk, a.dtype, tied ? fb[i] + fw[i] : fb[i]);
+        if (a.mode == GDR_MODE_BONLY) st_elem(a.dw, tk, a.dtype, fw[i]);
+        if (scalar_g) a.dg[tk] = fg[i];
+    }
+}
+
+}  // namespace
+
+unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv) {
+    const unsigned long long nc = (unsigned long long)((T + C - 1) / C);
+    return 2ull * (unsigned long long)B * H * nc * dk * dv * sizeof(float);
+}
+
+gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
+    // 1. chunk-start states (the fp32 CUDA-core forward, checkpoints only)
+    ChunkArgs f{a.q, a.k, a.v, a.b, mode_uses_w(a.mode) ? a.w : nullptr, a.g, a.S0, nullptr, nullptr,
+                a.B, a.H, a.T, a.dk_, a.dv_, C, a.mode, a.dtype,
+                1, a.T, 0, nullptr, nullptr, nullptr,
+                0, 1, nullptr, nullptr, 1.f, 0.f, a.ws_states};
+    gdr_status_t st = launch_chunk_simt(f, s);
+    if (st != GDR_OK) return st;
+    // 2. state gradients, chunks in reverse
+    const int VS = dslice(a.dv_);
+    const size_t smem2 = dstate_smem_floats(a.dk_, VS) * sizeof(float);
+    if (cudaFuncSetAttribute(bwd_dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
+        cudaSuccess)
+        return GDR_ERR_CUDA;
+    bwd_dstate_kernel<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreads, smem2, s>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
+    // 3. per-chunk gradients
+    const int nc = (a.T + C - 1) / C;
+    const size_t smem3 = chunk_smem_floats(a.dk_, a.dv_) * sizeof(float);
+    auto kern = a.dk_ == 128 ? bwd_chunk_kernel<C * 128 / kThreads>
+              : a.dk_ == 64  ? bwd_chunk_kernel<C * 64 / kThreads>
+              : a.dk_ == 32  ? bwd_chunk_kernel<C * 32 / kThreads>
+                             : bwd_chunk_kernel<C * 16 / kThreads>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    kern<<<(unsigned)((size_t)a.B * a.H * nc), kThreads, smem3, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+}  // namespace gdr

@@ -57,9 +57,17 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
     const size_t tok0 = (size_t)bh * T;
     const int npairs = C * (C + 1) / 2;
 
+    const int nchunks = (T + C - 1) / C;
     for (int c0 = 0; c0 < T; c0 += C) {
         const int n = min(C, T - c0);
         __syncthreads();
+        if (a.chunk_states) {   // checkpoint: the state this chunk starts from
+            float *dst = a.chunk_states + ((size_t)bh * nchunks + c0 / C) * dk * dv + v0;
+            for (int idx = tid; idx < dk * VS; idx += nth) {
+                const int d = idx / VS, j = idx - d * VS;
+                dst[(size_t)d * dv + j] = Ss[idx];
+            }
+        }
         // ---- load the chunk; tokens past the end are zero (exact padding) ----
         for (int idx = tid; idx < C * dk; idx += nth) {
             const int t = idx / dk, d = idx - t * dk;
@@ -163,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
         }
         __syncthreads();
         // ---- O = Q_g S + P E for the chunk's real tokens ----
-        for (int idx = tid; idx < n * VS; idx += nth) {
+        for (int idx = tid; a.o && idx < n * VS; idx += nth) {
             const int t = idx / VS, j = idx - t * VS;
             float acc = 0.f;
             for (int d = 0; d < dk; ++d) acc = fmaf(qq[t * dk + d], Ss[d * VS + j], acc);

@@ -33,6 +33,9 @@ struct ChunkArgs {
     const void *z;
     const float *nw;
     float b_range, eps;
+    // CUDA-core kernel only: when set, the state at the start of every chunk is written to
+    // chunk_states[B*H][nchunks][dk][dv] (fp32; the backward's checkpoints), and o may be NULL.
+    float *chunk_states;
 };
 
 struct DecodeArgs {
@@ -68,6 +71,21 @@ gdr_status_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 // Reads and zeroes the device error word of the streaming decode kernel's bounded waits.
 cudaError_t decode_read_and_clear_error(int *err);
 gdr_status_t launch_state_copy(const ChunkArgs &a, cudaStream_t s);
+
+// Backward (bwd.cu): everything the three backward kernels need.
+struct BwdArgs {
+    const void *q, *k, *v, *b, *w;
+    const float *g, *S0;
+    const void *dO;
+    const float *dST;
+    void *dq, *dk, *dv, *db, *dw;
+    float *dg, *dS0;
+    int B, H, T, dk_, dv_, mode, dtype;
+    float *ws_states, *ws_dstates;   // [B*H][nchunks][dk][dv] fp32 each
+};
+constexpr int kBwdChunk = 32;   // tokens per chunk of the backward
+unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
+gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s);
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);
 
 }  // namespace gdr

@@ -48,7 +48,7 @@ ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_
     ChunkArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, o, S_T,
                 B, H, T, dk, dv, chunk, mode, dtype,
                 1, T, 0, nullptr, nullptr, nullptr,
-                0, 1, nullptr, nullptr, 1.f, 0.f};
+                0, 1, nullptr, nullptr, 1.f, 0.f, nullptr};
     return a;
 }
 
@@ -188,6 +188,45 @@ extern "C" gdr_status_t gdr_mixer_fwd(const void *q, const void *k, const void *
     if ((int64_t)B * H == 0) return GDR_OK;
     if (T == 0) return launch_state_copy(a, s);
     return launch_chunk_tc(a, s);
+}
+
+extern "C" unsigned long long gdr_chunk_bwd_workspace(int B, int H, int T, int dk, int dv) {
+    if (B < 0 || H < 0 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return 0;
+    return bwd_workspace_bytes(B, H, T, dk, dv);
+}
+
+extern "C" gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *v, const float *g_log,
+                                      const void *b, const void *w, const float *S0, const void *dO,
+                                      const float *dS_T, void *dq, void *dk_, void *dv_, float *dg,
+                                      void *db, void *dw, float *dS0, int B, int H, int T, int dk,
+                                      int dv, gdr_mode_t mode, gdr_dtype_t dtype, void *workspace,
+                                      unsigned long long workspace_bytes, void *stream) {
+    gdr_status_t st = check_common(mode, dtype, B, H, dk, dv);
+    if (st != GDR_OK) return st;
+    if (T < 0 || (int64_t)B * H > INT32_MAX / 1024) return GDR_ERR_DIM;
+    const bool work = (int64_t)B * H * T > 0;
+    if (work) {
+        if (!q || !k || !v || !g_log || !b || !dO || !dq || !dk_ || !dv_ || !dg || !db) return GDR_ERR_NULL;
+        if (mode_uses_w(mode) && (!w || !dw)) return GDR_ERR_NULL;
+    }
+    const void *ptrs[] = {q, k, v, g_log, b, w, S0, dO, dS_T, dq, dk_, dv_, dg, db, dw, dS0, workspace};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDR_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((int64_t)B * H == 0) return GDR_OK;
+    if (T == 0) {   // dS0 = dS_T (or zeros); nothing else to write
+        ChunkArgs a = make_args(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, dS_T, nullptr, dS0,
+                                B, H, 0, dk, dv, 32, mode, dtype);
+        return launch_state_copy(a, s);
+    }
+    const unsigned long long need = bwd_workspace_bytes(B, H, T, dk, dv);
+    if (!workspace || workspace_bytes < need) return GDR_ERR_WORKSPACE;
+    const size_t per = need / 2 / sizeof(float);
+    BwdArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, dO, dS_T,
+              dq, dk_, dv_, db, mode_uses_w(mode) ? dw : nullptr, dg, dS0,
+              B, H, T, dk, dv, (int)mode, (int)dtype,
+              static_cast<float *>(workspace), static_cast<float *>(workspace) + per};
+    return launch_bwd(a, s);
 }
 
 extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void *v,

@@ -157,3 +157,33 @@ def test_mixer_tied_modes_and_empty_batch(L):
     assert call_mixer(xw=None, mode=1, B=0) == OK
     assert call_mixer(xw=None, mode=2, B=0) == OK
     assert call_mixer(q=None, k=None, v=None, xg=None, xb=None, xw=None, z=None, nw=None, y=None, B=0) == OK
+
+
+def call_bwd(q=A, k=A, v=A, g=A, b=A, w=A, S0=None, dO=A, dST=None, dq=A, dk_=A, dv_=A, dg=A, db=A, dw=A,
+             dS0=A, B=1, H=2, T=40, dk=64, dv=64, mode=0, dtype=0, ws=A, ws_bytes=1 << 40):
+    return gdr.gdr_chunk_bwd(q, k, v, g, b, w, S0, dO, dST, dq, dk_, dv_, dg, db, dw, dS0, B, H, T, dk, dv, mode,
+                             dtype, ws, ws_bytes, None)
+
+
+def test_bwd_workspace_size(L):
+    # two fp32 states per 32-token chunk and sequence-head
+    assert gdr.gdr_chunk_bwd_workspace(2, 3, 100, 64, 32) == 2 * 2 * 3 * 4 * 64 * 32 * 4
+    assert gdr.gdr_chunk_bwd_workspace(2, 3, 0, 64, 32) == 0
+    assert gdr.gdr_chunk_bwd_workspace(2, 3, 10, 48, 32) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mode=9), MODE), (dict(dtype=5), DTYPE), (dict(dk=24), DIM), (dict(T=-1), DIM), (dict(B=-1), DIM),
+    (dict(q=None), NULL), (dict(dO=None), NULL), (dict(dq=None), NULL), (dict(dg=None), NULL),
+    (dict(db=None), NULL), (dict(dw=None), NULL), (dict(w=None), NULL),
+    (dict(ws=None), WORKSPACE), (dict(ws_bytes=100), WORKSPACE),
+    (dict(dq=A + 2), ALIGN), (dict(ws=A + 8), ALIGN), (dict(dS0=A + 4), ALIGN),
+])
+def test_bwd_rejects(L, kw, code):
+    assert call_bwd(**kw) == code
+
+
+def test_bwd_tied_modes_need_no_w(L):
+    assert call_bwd(w=None, dw=None, mode=1, B=0) == OK
+    assert call_bwd(q=None, k=None, v=None, g=None, b=None, w=None, dO=None, dq=None, dk_=None, dv_=None,
+                    dg=None, db=None, dw=None, dS0=None, H=0) == OK
