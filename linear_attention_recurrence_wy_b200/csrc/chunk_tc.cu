@@ -82,9 +82,8 @@ constexpr int RAW_K = RAW_Q + 16384;            // raw k                    16 K
 constexpr int RAW_B = RAW_K + 16384;            // raw b (GDN-2)            16 KB
 constexpr int RAW_G = RAW_B + 16384;            // raw g_log fp32 [64][128] 32 KB, then gamma
 constexpr int RAW_END = RAW_G + 32768;
-constexpr int OFF_A32 = RAW_END;                // inverse scratch: A fp32 [64][68]
-constexpr int OFF_T32 = OFF_A32 + 64 * kAS * 4; //                  T fp32 [64][68]
-constexpr int OFF_X = OFF_T32 + 64 * kAS * 4;   //                  4 x [16][20] fp32
+constexpr int OFF_A32 = RAW_END;                // inverse scratch: A, then T, fp32 [64][68]
+constexpr int OFF_X = OFF_A32 + 64 * kAS * 4;   //                  4 x [16][20] fp32
 constexpr int OFF_QK = (OFF_X + 4 * 16 * tri::XLD * 4 + 1023) / 1024 * 1024;
                                                 // [Kh;Qg] bf16 [128][128]  32 KB
 constexpr int OFF_KB = OFF_QK + 32768;          // Kb bf16 [2][64 t][128 d] 32 KB
@@ -369,7 +368,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
     const bool write_o = !a.pass;
 
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
-    float *sT32 = reinterpret_cast<float *>(sm + OFF_T32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
     float *sGam = reinterpret_cast<float *>(sm + RAW_G);
     float *sGs = reinterpret_cast<float *>(sm + OFF_GS);
@@ -734,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             // ---- W7: T = (I + A)^-1 by warps 0-3, straight into the bf16 tile, while
             //      warps 4-7 scan the next chunk's log-decay ----
             if (warp < 4) {
-                tri::inverse64(sA32, sT32, sX, warp, lane, Bar128{}, TileOut{t_tile});
+                tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{t_tile});   // in place
                 fence_async_smem();
                 Bar128{}();
                 if (wtid == 0) mbar_arrive(bar_h2 + 8 * pb);   // H2: T and P of chunk c ready

@@ -11,6 +11,12 @@
 // fp32 accumulation), so the shared-memory traffic is a few fragment loads per product.
 // T is rounded to bf16 by its consumers, so TF32's 2^-11 operand rounding stays below
 // the final precision.
+//
+// A and T may be the same array (in place): every block of A is read before the block of
+// T that takes its place is written, and within a phase no warp writes a block another
+// warp reads (diagonal blocks: each warp its own; T_10 and T_32 replace A_10 and A_32
+// after their own warp has read them; the lower-left 32 x 32 reads A_2x, A_3x in one
+// phase and writes T_2x, T_3x in the next).
 #pragma once
 #include <stdint.h>
 
