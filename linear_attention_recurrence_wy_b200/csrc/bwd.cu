@@ -18,15 +18,17 @@
 //   the reverse cumulative sum of the gamma gradient over the chunk.
 //
 // Three launches:
-//   1. the chunk-start states S_c of every chunk (the CUDA-core forward kernel, writing
-//      its checkpoints and no output) -> workspace;
+//   1. the states at every 64-token boundary (the forward kernel of the shape, tcgen05 or
+//      CUDA cores, writing checkpoints and no output) -> workspace;
 //   2. bwd_dstate_kernel: the state gradient dS' entering every chunk from above, walking
 //      the chunks backwards (sequential, parallel over value-column slices) -> workspace,
 //      and dS0;
-//   3. bwd_chunk_kernel: every chunk in parallel, from S_c and dS' -> dq, dk, dv, dg, db, dw.
+//   3. bwd_chunk_kernel: every 64-token span in parallel (its two chunks in turn; the first
+//      forms the middle state for the second), from S_c and dS' -> dq, dk, dv, dg, db, dw.
 // Pair decays are formed as exp(gamma_i - gamma_j) with i >= j, never as a product of two
 // exponentials, so no factor overflows for a forgetting decay.
 #include "common.cuh"
+#include "chunk_tc.cuh"
 
 namespace gdr {
 namespace {
@@ -199,16 +201,24 @@ __host__ __device__ inline size_t chunk_smem_floats(int dk, int dv) {
            (size_t)dk * (dv + 1) + 3 * (size_t)C;
 }
 
-// Launch 3: every chunk in parallel.  Thread (c = tid % dk, group tid / dk) owns key channel
-// c of RPG consecutive tokens and accumulates their dq, dk, db and d gamma in registers.
+// Launch 3: every 64-token span in parallel, its two 32-token chunks in turn.  The
+// checkpoint pass stored the state at the span's start; the first chunk also forms the
+// state at the span's middle, S_mid = e^gamma_C S + Ke^T E, for the second.  Thread
+// (c = tid % dk, group tid / dk) owns key channel c of RPG consecutive tokens and
+// accumulates their dq, dk, db and d gamma in registers.
 template <int RPG>
 __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     const int dk = a.dk_, dv = a.dv_, T = a.T;
-    const int nc = (T + C - 1) / C;
-    const int bh = blockIdx.x / nc, c_idx = blockIdx.x - bh * nc;
+    const int nc = (T + C - 1) / C, nspan = (T + 2 * C - 1) / (2 * C);
+    const int bh = blockIdx.x / nspan, span = blockIdx.x - bh * nspan;
+    const int tid = threadIdx.x, nth = blockDim.x;
+  for (int hf = 0; hf < 2; ++hf) {
+    const int c_idx = 2 * span + hf;
+    if (c_idx >= nc) break;
     const int t0 = c_idx * C, n = min(C, T - t0);
     const size_t tok0 = (size_t)bh * T + t0;
-    const int tid = threadIdx.x, nth = blockDim.x;
+    const bool make_mid = hf == 0 && c_idx + 1 < nc;   // the second chunk needs S_mid
+    __syncthreads();
     const int ch = tid % dk, i0 = (tid / dk) * RPG;   // this thread's channel and first token
     const int SLD = dv + 1;                            // padded row stride of the state tile
 
@@ -224,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     float *fb = Ss + dk * SLD;       // [C]: folded scalar erase-gate gradient
     float *fw = fb + C;              // [C]: folded scalar write-gate gradient
     float *fg = fw + C;              // [C]: folded scalar decay gradient
-    const float *Sg = a.ws_states + ((size_t)bh * nc + c_idx) * dk * dv;
+    float *Sg = a.ws_states + ((size_t)bh * nc + c_idx) * dk * dv;
     const float *dSg = a.ws_dstates + ((size_t)bh * nc + c_idx) * dk * dv;
 
     float aq[RPG], ak[RPG], ab[RPG], ag[RPG];
@@ -284,6 +294,23 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
         }
     }
     __syncthreads();
+    // Ke = k e^(gamma_C - gamma) in place of e^gamma (e^gamma is recomputed where still needed)
+    for (int idx = tid; idx < C * dk; idx += nth) {
+        const int d = idx % dk;
+        ex[idx] = kk[idx] * __expf(gC[d] - gm[idx]);
+    }
+    __syncthreads();
+    if (make_mid) {
+        // S_mid = e^gamma_C S + Ke^T E  -> the second chunk's checkpoint slot
+        float *Sm = Sg + (size_t)dk * dv;
+        for (int idx = tid; idx < dk * dv; idx += nth) {
+            const int d = idx / dv, j = idx - d * dv;
+            float acc = __expf(gC[d]) * Ss[d * SLD + j];
+            for (int t = 0; t < C; ++t) acc = fmaf(ex[t * dk + d], X3[t * dv + j], acc);
+            Sm[idx] = acc;
+        }
+        __syncthreads();
+    }
     // ---- dP = lower_incl(dO E^T); dS' replaces S_c; rowsum(S_c . dS') into d gamma_C ----
     for (int p = tid; p < C * C; p += nth) {
         const int t = p / C, j = p - t * C;
@@ -326,12 +353,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
             part = fmaf(kf, y[r], part);
         }
         atomicAdd(&dgC[ch], part);
-    }
-    __syncthreads();
-    // Ke in place of e^gamma (e^gamma is recomputed where still needed)
-    for (int idx = tid; idx < C * dk; idx += nth) {
-        const int d = idx % dk;
-        ex[idx] = kk[idx] * __expf(gC[d] - gm[idx]);
     }
     __syncthreads();
     // ---- dE = P^T dO + Ke dS'  (E is no longer needed) ----
@@ -478,6 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
         if (a.mode == GDR_MODE_BONLY) st_elem(a.dw, tk, a.dtype, fw[i]);
         if (scalar_g) a.dg[tk] = fg[i];
     }
+  }
 }
 
 }  // namespace
@@ -488,12 +510,13 @@ unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv) {
 }
 
 gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
-    // 1. chunk-start states (the fp32 CUDA-core forward, checkpoints only)
+    // 1. checkpoints: the state at every 64-token boundary, from the forward kernel of the
+    //    shape (the tcgen05 kernel for bf16, dk = dv = 128; else the fp32 CUDA-core one)
     ChunkArgs f{a.q, a.k, a.v, a.b, mode_uses_w(a.mode) ? a.w : nullptr, a.g, a.S0, nullptr, nullptr,
-                a.B, a.H, a.T, a.dk_, a.dv_, C, a.mode, a.dtype,
+                a.B, a.H, a.T, a.dk_, a.dv_, 2 * C, a.mode, a.dtype,
                 1, a.T, 0, nullptr, nullptr, nullptr,
                 0, 1, nullptr, nullptr, 1.f, 0.f, a.ws_states};
-    gdr_status_t st = launch_chunk_simt(f, s);
+    gdr_status_t st = chunk_tc_supported(f) ? launch_chunk_tc(f, s) : launch_chunk_simt(f, s);
     if (st != GDR_OK) return st;
     // 2. state gradients, chunks in reverse
     const int VS = dslice(a.dv_);
@@ -503,8 +526,8 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
         return GDR_ERR_CUDA;
     bwd_dstate_kernel<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreads, smem2, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
-    // 3. per-chunk gradients
-    const int nc = (a.T + C - 1) / C;
+    // 3. per-chunk gradients, one CTA per 64-token span
+    const int nspan = (a.T + 2 * C - 1) / (2 * C);
     const size_t smem3 = chunk_smem_floats(a.dk_, a.dv_) * sizeof(float);
     auto kern = a.dk_ == 128 ? bwd_chunk_kernel<C * 128 / kThreads>
               : a.dk_ == 64  ? bwd_chunk_kernel<C * 64 / kThreads>
@@ -512,7 +535,7 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
                              : bwd_chunk_kernel<C * 16 / kThreads>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
         return GDR_ERR_CUDA;
-    kern<<<(unsigned)((size_t)a.B * a.H * nc), kThreads, smem3, s>>>(a);
+    kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreads, smem3, s>>>(a);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -57,12 +57,12 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
     const size_t tok0 = (size_t)bh * T;
     const int npairs = C * (C + 1) / 2;
 
-    const int nchunks = (T + C - 1) / C;
     for (int c0 = 0; c0 < T; c0 += C) {
         const int n = min(C, T - c0);
         __syncthreads();
-        if (a.chunk_states) {   // checkpoint: the state this chunk starts from
-            float *dst = a.chunk_states + ((size_t)bh * nchunks + c0 / C) * dk * dv + v0;
+        if (a.chunk_states) {   // checkpoint: the state this chunk starts from, in the
+                                // slot of its first 32-token chunk
+            float *dst = a.chunk_states + ((size_t)bh * ((T + 31) / 32) + c0 / 32) * dk * dv + v0;
             for (int idx = tid; idx < dk * VS; idx += nth) {
                 const int d = idx / VS, j = idx - d * VS;
                 dst[(size_t)d * dv + j] = Ss[idx];

@@ -331,8 +331,10 @@ struct TokenMaps {
 };
 
 // kMixer: the token-mixer instantiation (activations on load, output epilogue, either
-// layout; ChunkArgs::mixer).  The plain instantiation is the recurrence alone on [B,H,T,D].
-template <bool kMixer>
+// layout; ChunkArgs::mixer).  kStates: the backward's checkpoint pass, which also writes
+// the fp32 state at the start of every chunk to ChunkArgs::chunk_states (slot 2c of the
+// backward's 32-token chunk slots).  The plain instantiation is the recurrence alone.
+template <bool kMixer, bool kStates>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, const __grid_constant__ TokenMaps tm) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -365,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         S0p = (!transfer && seg == 0 && a.S0) ? a.S0 + (size_t)bh * DK * DV : nullptr;
         STp = transfer ? a.ws_m + sidx : a.ws_send + sidx;
     }
-    const bool write_o = !a.pass;
+    const bool write_o = !a.pass && !kStates;
 
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
@@ -778,6 +780,19 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
             const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
             const float *egc = sEGC + (c & 3) * 128;
+            if (kStates) {
+                // checkpoint: S_c (S^T columns [64 half, +64) of this lane), before this
+                // chunk's update; coalesced over the value channels (lanes)
+                float *dst = a.chunk_states + ((size_t)bh * ((a.T + 31) / 32) + 2 * c) * DK * DV + v;
+#pragma unroll 1
+                for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_base + TM_S + d0, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dst[(size_t)(d0 + j) * DV] = x[j];
+                }
+            }
             // (w.v)^T for this thread's lane and token columns, read from global memory
             // before the wait for the operands; tokens past the end give zero
             float wvt[32];
@@ -1087,7 +1102,8 @@ bool encode_head_major(CUtensorMap *m, const void *base, int B, int T, int H, CU
 gdr_status_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(DK == DV, "one box shape serves every per-channel tensor");
-    auto kern = a.mixer ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+    auto kern = a.mixer ? chunk_tc_kernel<true, false>
+              : a.chunk_states ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     TokenMaps tm;

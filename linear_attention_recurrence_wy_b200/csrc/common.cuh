@@ -33,8 +33,9 @@ struct ChunkArgs {
     const void *z;
     const float *nw;
     float b_range, eps;
-    // CUDA-core kernel only: when set, the state at the start of every chunk is written to
-    // chunk_states[B*H][nchunks][dk][dv] (fp32; the backward's checkpoints), and o may be NULL.
+    // The backward's checkpoints: when set, the state at the start of every chunk is written
+    // to chunk_states[B*H][ceil(T/32)][dk][dv] (fp32), in the slot of the chunk's first
+    // 32-token chunk (a 64-token chunk c fills slot 2c), and o may be NULL.
     float *chunk_states;
 };
 
