@@ -27,6 +27,8 @@
 //      forms the middle state for the second), from S_c and dS' -> dq, dk, dv, dg, db, dw.
 // Pair decays are formed as exp(gamma_i - gamma_j) with i >= j, never as a product of two
 // exponentials, so no factor overflows for a forgetting decay.
+#include <type_traits>
+
 #include "common.cuh"
 #include "chunk_tc.cuh"
 
@@ -109,15 +111,39 @@ __device__ void chunk_core(const BwdArgs &a, size_t tok0, int n, float *qq, floa
     __syncthreads();
 }
 
-__host__ __device__ inline int dslice(int dv) { return dv < 32 ? dv : 32; }
+// The state-gradient kernel keeps a whole head's dS (all dv columns) in one CTA of
+// kThreadsS threads: one wave of B*H CTAs, and A, P, T formed once per chunk.
+constexpr int kThreadsS = 1024;
+__host__ __device__ inline int dslice(int dv) { return dv; }
+
+// Register-tiled product over shared-memory operands, for a 32-row result: warp w owns rows
+// 4w .. 4w + 3 and lane l the columns l + 32 e (e < NE, columns below n only):
+//   acc[r][e] += sum_{k in [k0, k1)} A(4w + r, k) * B(k, l + 32 e)
+// Per k a warp loads four A values (one address each, broadcast) and NE B values (32
+// consecutive columns): four times fewer shared-memory loads than one output per thread.
+template <int NE, class FA, class FB>
+__device__ __forceinline__ void tile_mm(float (&acc)[4][NE], int k0, int k1, int n, FA A, FB Bop) {
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    for (int k = k0; k < k1; ++k) {
+        float av[4], bv[NE];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) av[r] = A(4 * w + r, k);
+#pragma unroll
+        for (int e = 0; e < NE; ++e) bv[e] = (l + 32 * e < n) ? Bop(k, l + 32 * e) : 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(av[r], bv[e], acc[r][e]);
+    }
+}
 
 __host__ __device__ inline size_t dstate_smem_floats(int dk, int VS) {
     return 4 * (size_t)C * dk + dk + 3 * (size_t)C * C + (size_t)dk * VS + 3 * (size_t)C * VS;
 }
 
-// Launch 2: the state gradient, chunks in reverse.  One CTA per (sequence-head, slice of VS
-// value columns): the columns of dS are independent of one another.
-__global__ void __launch_bounds__(kThreads) bwd_dstate_kernel(BwdArgs a) {
+// Launch 2: the state gradient, chunks in reverse.  One CTA per sequence-head holding all
+// dv columns of dS (the columns are independent, so a slice of VS columns would also do).
+__global__ void __launch_bounds__(kThreadsS, 1) bwd_dstate_kernel(BwdArgs a) {
     const int dk = a.dk_, dv = a.dv_, T = a.T;
     const int VS = dslice(dv);
     const int bh = blockIdx.x, v0 = blockIdx.y * VS;
@@ -206,7 +232,7 @@ __host__ __device__ inline size_t chunk_smem_floats(int dk, int dv) {
 // state at the span's middle, S_mid = e^gamma_C S + Ke^T E, for the second.  Thread
 // (c = tid % dk, group tid / dk) owns key channel c of RPG consecutive tokens and
 // accumulates their dq, dk, db and d gamma in registers.
-template <int RPG>
+template <int RPG, int NE>
 __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     const int dk = a.dk_, dv = a.dv_, T = a.T;
     const int nc = (T + C - 1) / C, nspan = (T + 2 * C - 1) / (2 * C);
@@ -224,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
 
     extern __shared__ float sm[];
     float *qq = sm, *kk = qq + C * dk, *bb = kk + C * dk, *gm = bb + C * dk;
-    float *ex = gm + C * dk;         // [C][dk]: e^gamma, later Ke = k e^(gamma_C - gamma)
+    float *ex = gm + C * dk;         // [C][dk]: Kh = b k e^gamma, later Ke = k e^(gamma_C - gamma)
     float *gC = ex + C * dk, *dgC = gC + dk;
     float *Am = dgC + dk, *Tm = Am + C * C, *Pm = Tm + C * C, *dA = Pm + C * C, *dP = dA + C * C;
     float *X1 = dP + C * C;          // [C][dv]: dO, then dR
@@ -259,22 +285,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     for (int i = tid; i < C; i += nth) fb[i] = fw[i] = fg[i] = 0.f;
     for (int d = tid; d < dk; d += nth) dgC[d] = 0.f;
     chunk_core(a, tok0, n, qq, kk, bb, gm, gC, Am, Tm, Pm);
-    for (int idx = tid; idx < C * dk; idx += nth) ex[idx] = __expf(gm[idx]);
+    for (int idx = tid; idx < C * dk; idx += nth) ex[idx] = bb[idx] * kk[idx] * __expf(gm[idx]);
     __syncthreads();
+    const int wrow = 4 * (tid >> 5), lane = tid & 31;   // tile_mm's rows and first column
     // ---- R = w.v - Kh S ----
-    for (int idx = tid; idx < C * dv; idx += nth) {
-        const int i = idx / dv, j = idx - i * dv;
-        float acc = X2[idx];
-        for (int d = 0; d < dk; ++d) acc = fmaf(-bb[i * dk + d] * kk[i * dk + d] * ex[i * dk + d], Ss[d * SLD + j], acc);
-        X2[idx] = acc;
+    {
+        float acc[4][NE] = {};
+        tile_mm<NE>(acc, 0, dk, dv, [&](int i, int d) { return ex[i * dk + d]; },
+                    [&](int d, int j) { return Ss[d * SLD + j]; });
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (lane + 32 * e < dv) X2[(wrow + r) * dv + lane + 32 * e] -= acc[r][e];
     }
     __syncthreads();
-    // ---- E = T R;  DY = dO S^T (into dq and d gamma) ----
-    for (int idx = tid; idx < C * dv; idx += nth) {
-        const int i = idx / dv, j = idx - i * dv;
-        float acc = 0.f;
-        for (int m = 0; m <= i; ++m) acc = fmaf(Tm[i * C + m], X2[m * dv + j], acc);
-        X3[idx] = acc;
+    // ---- E = T R  (T is zero above its diagonal);  DY = dO S^T (into dq and d gamma) ----
+    {
+        float acc[4][NE] = {};
+        tile_mm<NE>(acc, 0, wrow + 4, dv, [&](int i, int m) { return Tm[i * C + m]; },
+                    [&](int m, int j) { return X2[m * dv + j]; });
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (lane + 32 * e < dv) X3[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
     }
     {
         float y[RPG];
@@ -288,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
 #pragma unroll
         for (int r = 0; r < RPG; ++r) {
             const int i = i0 + r;
-            const float e = ex[i * dk + ch];
+            const float e = __expf(gm[i * dk + ch]);
             aq[r] = fmaf(e, y[r], aq[r]);
             ag[r] = fmaf(qq[i * dk + ch] * e, y[r], ag[r]);
         }
@@ -303,11 +338,22 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     if (make_mid) {
         // S_mid = e^gamma_C S + Ke^T E  -> the second chunk's checkpoint slot
         float *Sm = Sg + (size_t)dk * dv;
-        for (int idx = tid; idx < dk * dv; idx += nth) {
-            const int d = idx / dv, j = idx - d * dv;
-            float acc = __expf(gC[d]) * Ss[d * SLD + j];
-            for (int t = 0; t < C; ++t) acc = fmaf(ex[t * dk + d], X3[t * dv + j], acc);
-            Sm[idx] = acc;
+        for (int d0 = 0; d0 < dk; d0 += C) {   // 32 rows (key channels) of S_mid at a time
+            float acc[4][NE] = {};
+            tile_mm<NE>(acc, 0, C, dv, [&](int d, int t) { return d0 + d < dk ? ex[t * dk + d0 + d] : 0.f; },
+                        [&](int t, int j) { return X3[t * dv + j]; });
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int d = d0 + wrow + r;
+                if (d < dk) {
+                    const float eg = __expf(gC[d]);
+#pragma unroll
+                    for (int e = 0; e < NE; ++e) {
+                        const int j = lane + 32 * e;
+                        if (j < dv) Sm[(size_t)d * dv + j] = fmaf(eg, Ss[d * SLD + j], acc[r][e]);
+                    }
+                }
+            }
         }
         __syncthreads();
     }
@@ -355,21 +401,30 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
         atomicAdd(&dgC[ch], part);
     }
     __syncthreads();
-    // ---- dE = P^T dO + Ke dS'  (E is no longer needed) ----
-    for (int idx = tid; idx < C * dv; idx += nth) {
-        const int j = idx / dv, v = idx - j * dv;
-        float acc = 0.f;
-        for (int t = j; t < C; ++t) acc = fmaf(Pm[t * C + j], X1[t * dv + v], acc);
-        for (int d = 0; d < dk; ++d) acc = fmaf(ex[j * dk + d], Ss[d * SLD + v], acc);
-        X3[idx] = acc;
+    // ---- dE = P^T dO + Ke dS'  (E is no longer needed; P is zero above its diagonal) ----
+    {
+        float acc[4][NE] = {};
+        tile_mm<NE>(acc, wrow, C, dv, [&](int j, int t) { return Pm[t * C + j]; },
+                    [&](int t, int v) { return X1[t * dv + v]; });
+        tile_mm<NE>(acc, 0, dk, dv, [&](int j, int d) { return ex[j * dk + d]; },
+                    [&](int d, int v) { return Ss[d * SLD + v]; });
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (lane + 32 * e < dv) X3[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
     }
     __syncthreads();
     // ---- dR = T^T dE (dO is no longer needed); dT = dE R^T into dA ----
-    for (int idx = tid; idx < C * dv; idx += nth) {
-        const int i = idx / dv, v = idx - i * dv;
-        float acc = 0.f;
-        for (int j = i; j < C; ++j) acc = fmaf(Tm[j * C + i], X3[j * dv + v], acc);
-        X1[idx] = acc;
+    {
+        float acc[4][NE] = {};
+        tile_mm<NE>(acc, wrow, C, dv, [&](int i, int j) { return Tm[j * C + i]; },
+                    [&](int j, int v) { return X3[j * dv + v]; });
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (lane + 32 * e < dv) X1[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
     }
     for (int p = tid; p < C * C; p += nth) {
         const int i = p / C, j = p - i * C;
@@ -524,15 +579,21 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
     if (cudaFuncSetAttribute(bwd_dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
         cudaSuccess)
         return GDR_ERR_CUDA;
-    bwd_dstate_kernel<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreads, smem2, s>>>(a);
+    bwd_dstate_kernel<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreadsS, smem2, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     // 3. per-chunk gradients, one CTA per 64-token span
     const int nspan = (a.T + 2 * C - 1) / (2 * C);
     const size_t smem3 = chunk_smem_floats(a.dk_, a.dv_) * sizeof(float);
-    auto kern = a.dk_ == 128 ? bwd_chunk_kernel<C * 128 / kThreads>
-              : a.dk_ == 64  ? bwd_chunk_kernel<C * 64 / kThreads>
-              : a.dk_ == 32  ? bwd_chunk_kernel<C * 32 / kThreads>
-                             : bwd_chunk_kernel<C * 16 / kThreads>;
+    // RPG rows per thread for the (token, key channel) gradients; NE column groups of 32
+    // for the tiled products over the value channels
+    auto pick = [&](auto rpg) {
+        constexpr int R = decltype(rpg)::value;
+        return a.dv_ == 128 ? bwd_chunk_kernel<R, 4> : a.dv_ == 64 ? bwd_chunk_kernel<R, 2> : bwd_chunk_kernel<R, 1>;
+    };
+    auto kern = a.dk_ == 128 ? pick(std::integral_constant<int, C * 128 / kThreads>{})
+              : a.dk_ == 64  ? pick(std::integral_constant<int, C * 64 / kThreads>{})
+              : a.dk_ == 32  ? pick(std::integral_constant<int, C * 32 / kThreads>{})
+                             : pick(std::integral_constant<int, C * 16 / kThreads>{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
         return GDR_ERR_CUDA;
     kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreads, smem3, s>>>(a);
