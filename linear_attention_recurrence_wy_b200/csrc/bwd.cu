@@ -37,6 +37,8 @@ namespace {
 
 constexpr int C = kBwdChunk;
 constexpr int kThreads = 256;
+constexpr int kThreadsC = 512;          // the per-chunk kernel: 16 warps
+constexpr int RW = C / (kThreadsC / 32); // rows of a tiled product per warp (2)
 
 __device__ __forceinline__ float ld_b(const BwdArgs &a, size_t tk, int c) {   // erase gate b_tc
     return mode_b_vec(a.mode) ? ld_elem(a.b, tk * a.dk_ + c, a.dtype) : ld_elem(a.b, tk, a.dtype);
@@ -117,21 +119,21 @@ constexpr int kThreadsS = 1024;
 __host__ __device__ inline int dslice(int dv) { return dv; }
 
 // Register-tiled product over shared-memory operands, for a 32-row result: warp w owns rows
-// 4w .. 4w + 3 and lane l the columns l + 32 e (e < NE, columns below n only):
-//   acc[r][e] += sum_{k in [k0, k1)} A(4w + r, k) * B(k, l + 32 e)
-// Per k a warp loads four A values (one address each, broadcast) and NE B values (32
-// consecutive columns): four times fewer shared-memory loads than one output per thread.
+// RW w .. RW w + RW - 1 and lane l the columns l + 32 e (e < NE, columns below n only):
+//   acc[r][e] += sum_{k in [k0, k1)} A(RW w + r, k) * B(k, l + 32 e)
+// Per k a warp loads RW A values (one address each, broadcast) and NE B values (32
+// consecutive columns) for RW * NE multiply-adds.
 template <int NE, class FA, class FB>
-__device__ __forceinline__ void tile_mm(float (&acc)[4][NE], int k0, int k1, int n, FA A, FB Bop) {
+__device__ __forceinline__ void tile_mm(float (&acc)[RW][NE], int k0, int k1, int n, FA A, FB Bop) {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     for (int k = k0; k < k1; ++k) {
-        float av[4], bv[NE];
+        float av[RW], bv[NE];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) av[r] = A(4 * w + r, k);
+        for (int r = 0; r < RW; ++r) av[r] = A(RW * w + r, k);
 #pragma unroll
         for (int e = 0; e < NE; ++e) bv[e] = (l + 32 * e < n) ? Bop(k, l + 32 * e) : 0.f;
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < RW; ++r)
 #pragma unroll
             for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(av[r], bv[e], acc[r][e]);
     }
@@ -233,7 +235,7 @@ __host__ __device__ inline size_t chunk_smem_floats(int dk, int dv) {
 // (c = tid % dk, group tid / dk) owns key channel c of RPG consecutive tokens and
 // accumulates their dq, dk, db and d gamma in registers.
 template <int RPG, int NE>
-__global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     const int dk = a.dk_, dv = a.dv_, T = a.T;
     const int nc = (T + C - 1) / C, nspan = (T + 2 * C - 1) / (2 * C);
     const int bh = blockIdx.x / nspan, span = blockIdx.x - bh * nspan;
@@ -287,14 +289,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     chunk_core(a, tok0, n, qq, kk, bb, gm, gC, Am, Tm, Pm);
     for (int idx = tid; idx < C * dk; idx += nth) ex[idx] = bb[idx] * kk[idx] * __expf(gm[idx]);
     __syncthreads();
-    const int wrow = 4 * (tid >> 5), lane = tid & 31;   // tile_mm's rows and first column
+    const int wrow = RW * (tid >> 5), lane = tid & 31;   // tile_mm's rows and first column
     // ---- R = w.v - Kh S ----
     {
-        float acc[4][NE] = {};
+        float acc[RW][NE] = {};
         tile_mm<NE>(acc, 0, dk, dv, [&](int i, int d) { return ex[i * dk + d]; },
                     [&](int d, int j) { return Ss[d * SLD + j]; });
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < RW; ++r)
 #pragma unroll
             for (int e = 0; e < NE; ++e)
                 if (lane + 32 * e < dv) X2[(wrow + r) * dv + lane + 32 * e] -= acc[r][e];
@@ -302,11 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     __syncthreads();
     // ---- E = T R  (T is zero above its diagonal);  DY = dO S^T (into dq and d gamma) ----
     {
-        float acc[4][NE] = {};
-        tile_mm<NE>(acc, 0, wrow + 4, dv, [&](int i, int m) { return Tm[i * C + m]; },
+        float acc[RW][NE] = {};
+        tile_mm<NE>(acc, 0, wrow + RW, dv, [&](int i, int m) { return Tm[i * C + m]; },
                     [&](int m, int j) { return X2[m * dv + j]; });
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < RW; ++r)
 #pragma unroll
             for (int e = 0; e < NE; ++e)
                 if (lane + 32 * e < dv) X3[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
@@ -339,11 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
         // S_mid = e^gamma_C S + Ke^T E  -> the second chunk's checkpoint slot
         float *Sm = Sg + (size_t)dk * dv;
         for (int d0 = 0; d0 < dk; d0 += C) {   // 32 rows (key channels) of S_mid at a time
-            float acc[4][NE] = {};
+            float acc[RW][NE] = {};
             tile_mm<NE>(acc, 0, C, dv, [&](int d, int t) { return d0 + d < dk ? ex[t * dk + d0 + d] : 0.f; },
                         [&](int t, int j) { return X3[t * dv + j]; });
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = 0; r < RW; ++r) {
                 const int d = d0 + wrow + r;
                 if (d < dk) {
                     const float eg = __expf(gC[d]);
@@ -403,13 +405,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     __syncthreads();
     // ---- dE = P^T dO + Ke dS'  (E is no longer needed; P is zero above its diagonal) ----
     {
-        float acc[4][NE] = {};
+        float acc[RW][NE] = {};
         tile_mm<NE>(acc, wrow, C, dv, [&](int j, int t) { return Pm[t * C + j]; },
                     [&](int t, int v) { return X1[t * dv + v]; });
         tile_mm<NE>(acc, 0, dk, dv, [&](int j, int d) { return ex[j * dk + d]; },
                     [&](int d, int v) { return Ss[d * SLD + v]; });
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < RW; ++r)
 #pragma unroll
             for (int e = 0; e < NE; ++e)
                 if (lane + 32 * e < dv) X3[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
@@ -417,11 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_chunk_kernel(BwdArgs a) {
     __syncthreads();
     // ---- dR = T^T dE (dO is no longer needed); dT = dE R^T into dA ----
     {
-        float acc[4][NE] = {};
+        float acc[RW][NE] = {};
         tile_mm<NE>(acc, wrow, C, dv, [&](int i, int j) { return Tm[j * C + i]; },
                     [&](int j, int v) { return X3[j * dv + v]; });
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < RW; ++r)
 #pragma unroll
             for (int e = 0; e < NE; ++e)
                 if (lane + 32 * e < dv) X1[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
@@ -590,13 +592,13 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
         constexpr int R = decltype(rpg)::value;
         return a.dv_ == 128 ? bwd_chunk_kernel<R, 4> : a.dv_ == 64 ? bwd_chunk_kernel<R, 2> : bwd_chunk_kernel<R, 1>;
     };
-    auto kern = a.dk_ == 128 ? pick(std::integral_constant<int, C * 128 / kThreads>{})
-              : a.dk_ == 64  ? pick(std::integral_constant<int, C * 64 / kThreads>{})
-              : a.dk_ == 32  ? pick(std::integral_constant<int, C * 32 / kThreads>{})
-                             : pick(std::integral_constant<int, C * 16 / kThreads>{});
+    auto kern = a.dk_ == 128 ? pick(std::integral_constant<int, C * 128 / kThreadsC>{})
+              : a.dk_ == 64  ? pick(std::integral_constant<int, C * 64 / kThreadsC>{})
+              : a.dk_ == 32  ? pick(std::integral_constant<int, C * 32 / kThreadsC>{})
+                             : pick(std::integral_constant<int, C * 16 / kThreadsC>{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
         return GDR_ERR_CUDA;
-    kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreads, smem3, s>>>(a);
+    kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreadsC, smem3, s>>>(a);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
