@@ -123,20 +123,24 @@ __host__ __device__ inline int dslice(int dv) { return dv; }
 //   acc[r][e] += sum_{k in [k0, k1)} A(RW w + r, k) * B(k, l + 32 e)
 // Per k a warp loads RW A values (one address each, broadcast) and NE B values (32
 // consecutive columns) for RW * NE multiply-adds.
-template <int NE, class FA, class FB>
-__device__ __forceinline__ void tile_mm(float (&acc)[RW][NE], int k0, int k1, int n, FA A, FB Bop) {
+template <int RWT, int NE, class FA, class FB>
+__device__ __forceinline__ void tile_mm_rw(float (&acc)[RWT][NE], int k0, int k1, int n, FA A, FB Bop) {
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     for (int k = k0; k < k1; ++k) {
-        float av[RW], bv[NE];
+        float av[RWT], bv[NE];
 #pragma unroll
-        for (int r = 0; r < RW; ++r) av[r] = A(RW * w + r, k);
+        for (int r = 0; r < RWT; ++r) av[r] = A(RWT * w + r, k);
 #pragma unroll
         for (int e = 0; e < NE; ++e) bv[e] = (l + 32 * e < n) ? Bop(k, l + 32 * e) : 0.f;
 #pragma unroll
-        for (int r = 0; r < RW; ++r)
+        for (int r = 0; r < RWT; ++r)
 #pragma unroll
             for (int e = 0; e < NE; ++e) acc[r][e] = fmaf(av[r], bv[e], acc[r][e]);
     }
+}
+template <int NE, class FA, class FB>
+__device__ __forceinline__ void tile_mm(float (&acc)[RW][NE], int k0, int k1, int n, FA A, FB Bop) {
+    tile_mm_rw<RW, NE>(acc, k0, k1, n, A, Bop);
 }
 
 __host__ __device__ inline size_t dstate_smem_floats(int dk, int VS) {
@@ -145,6 +149,7 @@ __host__ __device__ inline size_t dstate_smem_floats(int dk, int VS) {
 
 // Launch 2: the state gradient, chunks in reverse.  One CTA per sequence-head holding all
 // dv columns of dS (the columns are independent, so a slice of VS columns would also do).
+template <int NE>
 __global__ void __launch_bounds__(kThreadsS, 1) bwd_dstate_kernel(BwdArgs a) {
     const int dk = a.dk_, dv = a.dv_, T = a.T;
     const int VS = dslice(dv);
@@ -187,32 +192,50 @@ __global__ void __launch_bounds__(kThreadsS, 1) bwd_dstate_kernel(BwdArgs a) {
             kk[idx] *= __expf(gC[d] - gam);
         }
         __syncthreads();
-        // dE = P^T dO + Ke dS
-        for (int idx = tid; idx < C * VS; idx += nth) {
-            const int j = idx / VS, v = idx - j * VS;
-            float acc = 0.f;
-            for (int t = j; t < C; ++t) acc = fmaf(Pm[t * C + j], dO[t * VS + v], acc);
-            for (int d = 0; d < dk; ++d) acc = fmaf(kk[j * dk + d], dS[d * VS + v], acc);
-            dE[idx] = acc;
+        // Register-tiled products (tile_mm_rw): 32 warps, row r of warp w, columns lane + 32 e
+        const int w = tid >> 5, lane = tid & 31;
+        // dE = P^T dO + Ke dS  (one row per warp; P is zero above its diagonal)
+        {
+            float acc[1][NE] = {};
+            tile_mm_rw<1, NE>(acc, w, C, VS, [&](int j, int t) { return Pm[t * C + j]; },
+                              [&](int t, int v) { return dO[t * VS + v]; });
+            tile_mm_rw<1, NE>(acc, 0, dk, VS, [&](int j, int d) { return kk[j * dk + d]; },
+                              [&](int d, int v) { return dS[d * VS + v]; });
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (lane + 32 * e < VS) dE[w * VS + lane + 32 * e] = acc[0][e];
         }
         __syncthreads();
         // dR = T^T dE  (T lower triangular)
-        for (int idx = tid; idx < C * VS; idx += nth) {
-            const int i = idx / VS, v = idx - i * VS;
-            float acc = 0.f;
-            for (int j = i; j < C; ++j) acc = fmaf(Tm[j * C + i], dE[j * VS + v], acc);
-            dR[idx] = acc;
+        {
+            float acc[1][NE] = {};
+            tile_mm_rw<1, NE>(acc, w, C, VS, [&](int i, int j) { return Tm[j * C + i]; },
+                              [&](int j, int v) { return dE[j * VS + v]; });
+#pragma unroll
+            for (int e = 0; e < NE; ++e)
+                if (lane + 32 * e < VS) dR[w * VS + lane + 32 * e] = acc[0][e];
         }
         __syncthreads();
-        // dS <- e^gamma_C dS + Qg^T dO - Kh^T dR   (the gradient with respect to S_c)
-        for (int idx = tid; idx < dk * VS; idx += nth) {
-            const int d = idx / VS, v = idx - d * VS;
-            float acc = __expf(gC[d]) * dS[idx];
-            for (int t = 0; t < C; ++t) {
-                acc = fmaf(qq[t * dk + d], dO[t * VS + v], acc);
-                acc = fmaf(-bb[t * dk + d], dR[t * VS + v], acc);
+        // dS <- e^gamma_C dS + Qg^T dO - Kh^T dR   (the gradient with respect to S_c); four
+        // key-channel rows per warp, 128 at most
+        {
+            float acc[4][NE] = {};
+            tile_mm_rw<4, NE>(acc, 0, C, VS, [&](int d, int t) { return d < dk ? qq[t * dk + d] : 0.f; },
+                              [&](int t, int v) { return dO[t * VS + v]; });
+            tile_mm_rw<4, NE>(acc, 0, C, VS, [&](int d, int t) { return d < dk ? -bb[t * dk + d] : 0.f; },
+                              [&](int t, int v) { return dR[t * VS + v]; });
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int d = 4 * w + r;
+                if (d < dk) {
+                    const float eg = __expf(gC[d]);
+#pragma unroll
+                    for (int e = 0; e < NE; ++e) {
+                        const int v = lane + 32 * e;
+                        if (v < VS) dS[d * VS + v] = fmaf(eg, dS[d * VS + v], acc[r][e]);
+                    }
+                }
             }
-            dS[idx] = acc;
         }
     }
     __syncthreads();
@@ -578,10 +601,10 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
     // 2. state gradients, chunks in reverse
     const int VS = dslice(a.dv_);
     const size_t smem2 = dstate_smem_floats(a.dk_, VS) * sizeof(float);
-    if (cudaFuncSetAttribute(bwd_dstate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
-        cudaSuccess)
+    auto kern2 = VS == 128 ? bwd_dstate_kernel<4> : VS == 64 ? bwd_dstate_kernel<2> : bwd_dstate_kernel<1>;
+    if (cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
         return GDR_ERR_CUDA;
-    bwd_dstate_kernel<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreadsS, smem2, s>>>(a);
+    kern2<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreadsS, smem2, s>>>(a);
     if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     // 3. per-chunk gradients, one CTA per 64-token span
     const int nspan = (a.T + 2 * C - 1) / (2 * C);
