@@ -263,6 +263,81 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     const int nc = (T + C - 1) / C, nspan = (T + 2 * C - 1) / (2 * C);
     const int bh = blockIdx.x / nspan, span = blockIdx.x - bh * nspan;
     const int tid = threadIdx.x, nth = blockDim.x;
+    if (a.mid_grad && 2 * span + 1 < nc) {
+        // The state gradient at the span's middle, from its end by one step of the reverse
+        // recurrence over the second chunk: dS_mid = e^gamma_C dS_end + Qg^T dO - Kh^T dR
+        // with dR = T^T (P^T dO + Ke dS_end)  -> the first chunk's slot of ws_dstates.
+        const int c1 = 2 * span + 1, t1 = c1 * C, n1 = min(C, T - t1);
+        const size_t tk1 = (size_t)bh * T + t1;
+        const int SLD = dv + 1;
+        extern __shared__ float sm[];
+        float *qq = sm, *kk = qq + C * dk, *bb = kk + C * dk, *gm = bb + C * dk;
+        float *ex = gm + C * dk, *gC = ex + C * dk;
+        float *Am = gC + 2 * dk, *Tm = Am + C * C, *Pm = Tm + C * C;
+        float *X1 = Pm + 3 * C * C, *X2 = X1 + C * dv, *X3 = X2 + C * dv, *Ss = X3 + C * dv;
+        const float *dSe = a.ws_dstates + ((size_t)bh * nc + c1) * dk * dv;
+        float *dSm = a.ws_dstates + ((size_t)bh * nc + c1 - 1) * dk * dv;
+        for (int idx = tid; idx < C * dv; idx += nth) {
+            const int t = idx / dv, j = idx - t * dv;
+            X1[idx] = t < n1 ? ld_elem(a.dO, (tk1 + t) * dv + j, a.dtype) : 0.f;
+        }
+        for (int idx = tid; idx < dk * dv; idx += nth) Ss[(idx / dv) * SLD + idx % dv] = dSe[idx];
+        chunk_core(a, tk1, n1, qq, kk, bb, gm, gC, Am, Tm, Pm);
+        for (int idx = tid; idx < C * dk; idx += nth) {   // Ke, Qg, Kh
+            const int d = idx % dk;
+            const float e = __expf(gm[idx]);
+            ex[idx] = kk[idx] * __expf(gC[d] - gm[idx]);
+            qq[idx] *= e;
+            bb[idx] *= kk[idx] * e;
+        }
+        __syncthreads();
+        const int wrow = RW * (tid >> 5), lane = tid & 31;
+        {   // dE = P^T dO + Ke dS_end -> X3
+            float acc[RW][NE] = {};
+            tile_mm<NE>(acc, wrow, C, dv, [&](int j, int t) { return Pm[t * C + j]; },
+                        [&](int t, int v) { return X1[t * dv + v]; });
+            tile_mm<NE>(acc, 0, dk, dv, [&](int j, int d) { return ex[j * dk + d]; },
+                        [&](int d, int v) { return Ss[d * SLD + v]; });
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    if (lane + 32 * e < dv) X3[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
+        }
+        __syncthreads();
+        {   // dR = T^T dE -> X2
+            float acc[RW][NE] = {};
+            tile_mm<NE>(acc, wrow, C, dv, [&](int i, int j) { return Tm[j * C + i]; },
+                        [&](int j, int v) { return X3[j * dv + v]; });
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+#pragma unroll
+                for (int e = 0; e < NE; ++e)
+                    if (lane + 32 * e < dv) X2[(wrow + r) * dv + lane + 32 * e] = acc[r][e];
+        }
+        __syncthreads();
+        {   // dS_mid, eight key-channel rows per warp (128 at most)
+            constexpr int RK = 8;
+            const int w = tid >> 5;
+            float acc[RK][NE] = {};
+            tile_mm_rw<RK, NE>(acc, 0, C, dv, [&](int d, int t) { return d < dk ? qq[t * dk + d] : 0.f; },
+                               [&](int t, int v) { return X1[t * dv + v]; });
+            tile_mm_rw<RK, NE>(acc, 0, C, dv, [&](int d, int t) { return d < dk ? -bb[t * dk + d] : 0.f; },
+                               [&](int t, int v) { return X2[t * dv + v]; });
+#pragma unroll
+            for (int r = 0; r < RK; ++r) {
+                const int d = RK * w + r;
+                if (d < dk) {
+                    const float eg = __expf(gC[d]);
+#pragma unroll
+                    for (int e = 0; e < NE; ++e) {
+                        const int v = lane + 32 * e;
+                        if (v < dv) dSm[(size_t)d * dv + v] = fmaf(eg, Ss[d * SLD + v], acc[r][e]);
+                    }
+                }
+            }
+        }
+    }
   for (int hf = 0; hf < 2; ++hf) {
     const int c_idx = 2 * span + hf;
     if (c_idx >= nc) break;
@@ -595,17 +670,33 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
     ChunkArgs f{a.q, a.k, a.v, a.b, mode_uses_w(a.mode) ? a.w : nullptr, a.g, a.S0, nullptr, nullptr,
                 a.B, a.H, a.T, a.dk_, a.dv_, 2 * C, a.mode, a.dtype,
                 1, a.T, 0, nullptr, nullptr, nullptr,
-                0, 1, nullptr, nullptr, 1.f, 0.f, a.ws_states};
-    gdr_status_t st = chunk_tc_supported(f) ? launch_chunk_tc(f, s) : launch_chunk_simt(f, s);
+                0, 1, nullptr, nullptr, 1.f, 0.f, a.ws_states, 0, nullptr};
+    const bool tc = chunk_tc_supported(f);
+    gdr_status_t st = tc ? launch_chunk_tc(f, s) : launch_chunk_simt(f, s);
     if (st != GDR_OK) return st;
-    // 2. state gradients, chunks in reverse
-    const int VS = dslice(a.dv_);
-    const size_t smem2 = dstate_smem_floats(a.dk_, VS) * sizeof(float);
-    auto kern2 = VS == 128 ? bwd_dstate_kernel<4> : VS == 64 ? bwd_dstate_kernel<2> : bwd_dstate_kernel<1>;
-    if (cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
-        return GDR_ERR_CUDA;
-    kern2<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreadsS, smem2, s>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
+    BwdArgs b = a;
+    if (tc) {
+        // 2. the state gradient on the tensor cores: the same kernel in reverse chunk order,
+        //    writing the gradient at every 64-token span's end (the per-chunk kernel forms the
+        //    middle ones) and dS0
+        ChunkArgs r = f;
+        r.S0 = a.dST;
+        r.ST = a.dS0;
+        r.chunk_states = a.ws_dstates;
+        r.reverse = 1;
+        r.dO = a.dO;
+        if ((st = launch_chunk_tc(r, s)) != GDR_OK) return st;
+        b.mid_grad = 1;
+    } else {
+        // 2. state gradients on CUDA cores, chunks in reverse (every 32-token chunk's end)
+        const int VS = dslice(a.dv_);
+        const size_t smem2 = dstate_smem_floats(a.dk_, VS) * sizeof(float);
+        auto kern2 = VS == 128 ? bwd_dstate_kernel<4> : VS == 64 ? bwd_dstate_kernel<2> : bwd_dstate_kernel<1>;
+        if (cudaFuncSetAttribute(kern2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) != cudaSuccess)
+            return GDR_ERR_CUDA;
+        kern2<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreadsS, smem2, s>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
+    }
     // 3. per-chunk gradients, one CTA per 64-token span
     const int nspan = (a.T + 2 * C - 1) / (2 * C);
     const size_t smem3 = chunk_smem_floats(a.dk_, a.dv_) * sizeof(float);
@@ -621,7 +712,7 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
                              : pick(std::integral_constant<int, C * 16 / kThreadsC>{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
         return GDR_ERR_CUDA;
-    kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreadsC, smem3, s>>>(a);
+    kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreadsC, smem3, s>>>(b);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -105,6 +105,7 @@ constexpr uint32_t TM_XO = 128;  // [X, then E^T | O^T] fp32                  64
 constexpr uint32_t TM_AP = 256;  // [A; P] fp32                                 64
 constexpr uint32_t TM_SB = 320;  // S^T bf16 (packed)                           64
 constexpr uint32_t TM_XB = 384;  // R^T, then E^T bf16 (packed)                 32
+constexpr uint32_t TM_DO = 416;   // state-gradient pass: dO^T bf16 (packed)      32
 constexpr uint32_t TM_ONES = 448; // mixer: bf16 ones, the A operand of the output's
                                   // sum of squares over value channels        64
 constexpr uint32_t TM_COLS = 512;
@@ -333,8 +334,10 @@ struct TokenMaps {
 // kMixer: the token-mixer instantiation (activations on load, output epilogue, either
 // layout; ChunkArgs::mixer).  kStates: the backward's checkpoint pass, which also writes
 // the fp32 state at the start of every chunk to ChunkArgs::chunk_states (slot 2c of the
-// backward's 32-token chunk slots).  The plain instantiation is the recurrence alone.
-template <bool kMixer, bool kStates>
+// backward's 32-token chunk slots).  kReverse: the backward's state-gradient pass
+// (ChunkArgs::reverse), chunks in reverse order; see the state group.  The plain
+// instantiation is the recurrence alone.
+template <bool kMixer, bool kStates, bool kReverse>
 __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, const __grid_constant__ TokenMaps tm) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -357,6 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
     if (kMixer && ts != 1) tok0 = ((size_t)(bh / a.H) * a.T + t_begin) * a.H + bh % a.H;
     const int hc = bh % a.H, bc = bh / a.H;   // tensor-map coordinates of this head
     const int nchunks = (T + C - 1) / C;
+    // iteration c (barrier phases, buffers, ring slots) works on data chunk dch(c)
+    auto dch = [&](int c) { return kReverse ? nchunks - 1 - c : c; };
     const size_t sidx = ((size_t)bh * a.nseg + seg) * DK * DV;
     const float *S0p = nullptr;        // initial state (NULL: zero, unless the identity)
     float *STp = nullptr;              // end state destination (NULL: not written)
@@ -367,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         S0p = (!transfer && seg == 0 && a.S0) ? a.S0 + (size_t)bh * DK * DV : nullptr;
         STp = transfer ? a.ws_m + sidx : a.ws_send + sidx;
     }
-    const bool write_o = !a.pass && !kStates;
+    const bool write_o = !a.pass && !kStates && !kReverse;
 
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
     // chunks only)
     auto prefetch_inputs = [&](int c) {
         if (kMixer && ts != 1) {
-            const int tt = t_begin + c * C;
+            const int tt = t_begin + dch(c) * C;
             tma_prefetch_4d(&tm.q, 0, hc, tt, bc);
             tma_prefetch_4d(&tm.k, 0, hc, tt, bc);
             tma_prefetch_4d(&tm.v, 0, hc, tt, bc);
@@ -443,13 +448,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             if (vec_g) tma_prefetch_4d(&tm.g, 0, hc, tt, bc);
             return;
         }
-        const int t0 = c * C, n = min(C, T - t0);
+        const int t0 = dch(c) * C, n = min(C, T - t0);
         const size_t e = (tok0 + t0) * DK;
         prefetch_l2(Q + e, n * DK * 2);
         prefetch_l2(K + e, n * DK * 2);
-        prefetch_l2(V + e, n * DV * 2);
+        if (kReverse) {
+            prefetch_l2(reinterpret_cast<const __nv_bfloat16 *>(a.dO) + e, n * DV * 2);
+        } else {
+            prefetch_l2(V + e, n * DV * 2);
+            if (vec_w) prefetch_l2(Wg + e, n * DV * 2);
+        }
         if (vec_b) prefetch_l2(Bg + e, n * DK * 2);
-        if (vec_w) prefetch_l2(Wg + e, n * DV * 2);
         if (vec_g) prefetch_l2(a.g + e, n * DK * 4);
         if (kMixer) prefetch_l2(Z + e, n * DV * 2);
     };
@@ -468,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
                 // token-major: one tiled tensor copy per tensor; a box is always whole
                 // (64 rows, zero-filled past the end), so its bytes are counted whole
                 if (lane != 0 || warp < 4) return;
-                const int tt = t_begin + c * C;
+                const int tt = t_begin + dch(c) * C;
                 constexpr uint32_t box16 = C * DK * 2;
                 fence_async_smem();
                 if (warp == 4) {
@@ -487,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
                 return;
             }
             if (lane != 0 || warp < 4) return;
-            const int t0 = c * C, n = min(C, T - t0);
+            const int t0 = dch(c) * C, n = min(C, T - t0);
             const size_t e = (tok0 + t0) * DK;
             const uint32_t row16 = (uint32_t)n * DK * 2;
             fence_async_smem();
@@ -513,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         // gamma_C, exp(gamma_C) and the exact-path flag.  False if the wait failed.
         auto scan = [&](int c) -> bool {
             const int d = wtid - 128;   // 0 .. 127
-            const int t0 = c * C, n = min(C, T - t0);
+            const int t0 = dch(c) * C, n = min(C, T - t0);
             // scalar gates (they need no staging copy): GDN's g_log by threads 0-63, a
             // scalar erase gate (beta, or w-only's b) by threads 64-127 for the operand build
             if (!vec_g && d < 64) {
@@ -584,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         // iteration c = -1 only scans chunk 0 (one call site keeps one copy of the scan)
         for (int c = -1; c < nchunks; ++c) {
           if (c >= 0) {
-            const int t0 = c * C, n = min(C, T - t0);
+            const int t0 = dch(c) * C, n = min(C, T - t0);
             const int pb = c & 1;   // P, T and Kb buffer of this chunk
             // ---- W1: the scan of chunk c (warps 4-7) has finished, and the state group has
             //      consumed Kh and Qg of chunk c-1 (H3), so they may be rebuilt ----
@@ -774,8 +783,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         tmem_wait_st();
         tc_fence_before();
         group_sync(BAR_ST);
-        for (int c = 0; c < nchunks; ++c) {
-            const int t0 = c * C, n = min(C, T - t0);
+        for (int c = 0; !kReverse && c < nchunks; ++c) {
+            const int t0 = dch(c) * C, n = min(C, T - t0);
             const int pb = c & 1;
             const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
             const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
@@ -1007,6 +1016,143 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             group_sync(BAR_ST);
             if (stid == 0) mbar_arrive(bar_h4 + 8 * pb);   // H4: chunk c finished
         }
+        // ---- the backward's state-gradient pass (kReverse): G = dL/dS walks the chunks from
+        //      the last to the first.  In TMEM G^T as the state S^T is (lane = value channel);
+        //      the WY group supplies the same tiles as for the forward (Kh, Qg, Kb, P, T), and
+        //      per chunk (Gated DeltaNet-2 Review §3-2.5, differentiated):
+        //        dE^T = (G^T diag(e^gamma_C)) Kb^T + dO^T P      (Kb: K_end on the exact path)
+        //        dR^T = dE^T T
+        //        G^T <- G^T diag(e^gamma_C) + dO^T Qg - dR^T Kh
+        //      Before each chunk's update G is the gradient at the chunk's end: it goes to the
+        //      checkpoint slot of the chunk's last 32-token chunk. ----
+        for (int c = 0; kReverse && c < nchunks; ++c) {
+            const int cd = dch(c);
+            const int t0 = cd * C, n = min(C, T - t0);
+            const int pb = c & 1;
+            const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
+            const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
+            const float *egc = sEGC + (c & 3) * 128;
+            {
+                const int nslot = (T + 31) / 32;
+                float *dst = a.chunk_states + ((size_t)bh * nslot + min(2 * cd + 1, nslot - 1)) * DK * DV + v;
+#pragma unroll 1
+                for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_base + TM_S + d0, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dst[(size_t)(d0 + j) * DV] = x[j];
+                }
+            }
+            {   // dO^T of this lane and token columns -> bf16 in TMEM; tokens past the end give zero
+                const int last = min(31, n - 1 - j0);
+                const __nv_bfloat16 *op = reinterpret_cast<const __nv_bfloat16 *>(a.dO) + (tok0 + t0 + j0) * DV + v;
+                float x[32];
+                if (last >= 0) {   // rows past the end re-read the last row and give zero
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float y = __bfloat162float(op[min(j, last) * DV]);
+                        x[j] = j <= last ? y : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) x[j] = 0.f;
+                }
+                st_tmem_bf16(tmem + lane_base + TM_DO + j0 / 2, x);
+            }
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_h1, (uint32_t)(c & 1)));
+            if (!ok) break;
+            const bool exact = sExact[c & 3] != 0;
+            // G^T diag(e^gamma_C): the update's accumulator (fp32) and the operand of Kb (bf16;
+            // the exact path's K_end carries the decay itself)
+            for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
+                float x[32], y[32];
+                tmem_ld32(tmem + lane_base + TM_S + d0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) y[j] = x[j] * egc[d0 + j];
+                tmem_st32(tmem + lane_base + TM_S + d0, y);
+                st_tmem_bf16(tmem + lane_base + TM_SB + d0 / 2, exact ? x : y);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            group_sync(BAR_ST);
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id64 = idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)   // dE^T = G~^T Kb^T
+                    mma_bf16_ts(tmem + TM_XO, tmem + TM_SB + s * 8, desc_kmajor(kb_tile, 64, 0, s), id64, s > 0);
+                const uint32_t id128 = idesc_bf16(128, 128, false, true, false);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)    // G^T += dO^T Qg
+                    mma_bf16_ts(tmem + TM_S, tmem + TM_DO + s * 8, desc_mnmajor(sbase + OFF_QK, 128, 64, s), id128, 1u);
+            }
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_h2 + 8 * pb, (uint32_t)((c >> 1) & 1)));
+            if (!ok) break;
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, true, false);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)    // dE^T += dO^T P
+                    mma_bf16_ts(tmem + TM_XO, tmem + TM_DO + s * 8, desc_mnmajor(p_tile, 64, 0, s), id, 1u);
+                mma_commit(bar_st);
+            }
+            ++mma_st;
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            {   // dE^T -> bf16
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_XO + j0, x);
+                tmem_wait_ld();
+                st_tmem_bf16(tmem + lane_base + TM_XB + j0 / 2, x);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            group_sync(BAR_ST);
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 64, false, true, false);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)    // dR^T = dE^T T
+                    mma_bf16_ts(tmem + TM_XO + 64, tmem + TM_XB + s * 8, desc_mnmajor(t_tile, 64, 0, s), id, s > 0);
+                mma_commit(bar_st);
+            }
+            ++mma_st;
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            {   // -dR^T -> bf16
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_XO + 64 + j0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) x[j] = -x[j];
+                st_tmem_bf16(tmem + lane_base + TM_XB + j0 / 2, x);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            group_sync(BAR_ST);
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128, false, true, false);
+#pragma unroll
+                for (int s = 0; s < C / 16; ++s)    // G^T -= dR^T Kh
+                    mma_bf16_ts(tmem + TM_S, tmem + TM_XB + s * 8, desc_mnmajor(sbase + OFF_QK, 128, 0, s), id, 1u);
+                mma_commit(bar_st);
+            }
+            ++mma_st;
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            tc_fence_before();
+            group_sync(BAR_ST);
+            if (stid == 0) {
+                mbar_arrive(bar_h3);            // H3: Kh, Qg of chunk c consumed
+                mbar_arrive(bar_h4 + 8 * pb);   // H4: chunk c finished
+            }
+        }
         // end state: S^T columns [64 half, +64) of this thread's lane, from TMEM
         if (ok && STp) {
             tc_fence_after();
@@ -1102,8 +1248,9 @@ bool encode_head_major(CUtensorMap *m, const void *base, int B, int T, int H, CU
 gdr_status_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
     static_assert(DK == DV, "one box shape serves every per-channel tensor");
-    auto kern = a.mixer ? chunk_tc_kernel<true, false>
-              : a.chunk_states ? chunk_tc_kernel<false, true> : chunk_tc_kernel<false, false>;
+    auto kern = a.mixer ? chunk_tc_kernel<true, false, false>
+              : a.reverse ? chunk_tc_kernel<false, false, true>
+              : a.chunk_states ? chunk_tc_kernel<false, true, false> : chunk_tc_kernel<false, false, false>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     TokenMaps tm;

@@ -37,6 +37,11 @@ struct ChunkArgs {
     // to chunk_states[B*H][ceil(T/32)][dk][dv] (fp32), in the slot of the chunk's first
     // 32-token chunk (a 64-token chunk c fills slot 2c), and o may be NULL.
     float *chunk_states;
+    // The backward's state-gradient pass (tensor-core kernel, reverse != 0): S0 holds dS_T,
+    // ST receives dS0, dO is the output gradient [B,H,T,dv], and chunk_states receives the
+    // gradient at every 64-token chunk's end (slot of its last 32-token chunk).
+    int reverse;
+    const void *dO;
 };
 
 struct DecodeArgs {
@@ -83,6 +88,9 @@ struct BwdArgs {
     float *dg, *dS0;
     int B, H, T, dk_, dv_, mode, dtype;
     float *ws_states, *ws_dstates;   // [B*H][nchunks][dk][dv] fp32 each
+    // 1: ws_dstates holds the state gradient only at the ends of 64-token spans (the
+    // tensor-core state-gradient pass); the per-chunk kernel forms the middle ones
+    int mid_grad;
 };
 constexpr int kBwdChunk = 32;   // tokens per chunk of the backward
 unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv);

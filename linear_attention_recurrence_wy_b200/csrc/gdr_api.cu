@@ -48,7 +48,7 @@ ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_
     ChunkArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, o, S_T,
                 B, H, T, dk, dv, chunk, mode, dtype,
                 1, T, 0, nullptr, nullptr, nullptr,
-                0, 1, nullptr, nullptr, 1.f, 0.f, nullptr};
+                0, 1, nullptr, nullptr, 1.f, 0.f, nullptr, 0, nullptr};
     return a;
 }
 
@@ -225,7 +225,7 @@ extern "C" gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *
     BwdArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, dO, dS_T,
               dq, dk_, dv_, db, mode_uses_w(mode) ? dw : nullptr, dg, dS0,
               B, H, T, dk, dv, (int)mode, (int)dtype,
-              static_cast<float *>(workspace), static_cast<float *>(workspace) + per};
+              static_cast<float *>(workspace), static_cast<float *>(workspace) + per, 0};
     return launch_bwd(a, s);
 }
 

@@ -144,3 +144,29 @@ def test_t4k_workload_sampled_heads(cuda_ok):
     for n in NAMES:
         got = np.stack([np64(out[n][b, h]) for b, h in heads])
         check_grad(f"t4k {n}", got, ref[n][:, 0], "bf16")
+
+
+# ---- the tensor-core shape (bf16, dk = dv = 128): checkpoints and the state gradient run on
+#      tcgen05 (the forward kernel and its reverse-order instantiation) -------------------------
+@pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
+@pytest.mark.parametrize("T", [20, 64, 96, 150])
+def test_tensor_core_state_gradient(cuda_ok, mode, T):
+    # T = 20, 96: a last 64-token span with one 32-token chunk; 64: one whole span
+    d, dO, dST = make_case(2, 2, T, 128, 128, mode, "bf16", seed=T + 31, g_scale=0.1, s0=0.05)
+    run_case(d, dO, dST, "bf16")
+
+
+@pytest.mark.parametrize("g_const", [-1.5, -4.0])
+def test_tensor_core_state_gradient_strong_decay(cuda_ok, g_const):
+    # cumulative decays past the forward kernel's factorisation limit (|gamma| > 60 within a
+    # 64-token chunk): the exact path's K_end tiles feed the reverse chain unscaled.  (Much
+    # stronger decays leave dg as the exact difference of O(1) pair terms, about zero, where
+    # a relative error says nothing; the fp32 path's scaled check covers g = -20.)
+    d, dO, dST = make_case(1, 2, 140, 128, 128, "gdn2", "bf16", seed=41, s0=0.05)
+    d["g"] = torch.full_like(d["g"], g_const)
+    run_case(d, dO, dST, "bf16")
+
+
+def test_tensor_core_state_gradient_without_state_gradient_input(cuda_ok):
+    d, dO, dST = make_case(2, 2, 130, 128, 128, "gdn2", "bf16", seed=43, s0=0.0, dst=False)
+    run_case(d, dO, dST, "bf16")
