@@ -20,13 +20,15 @@
 // Three launches:
 //   1. the states at every 64-token boundary (the forward kernel of the shape, tcgen05 or
 //      CUDA cores, writing checkpoints and no output) -> workspace;
-//   2. bwd_dstate_kernel: the state gradient dS' entering every chunk from above, walking
-//      the chunks backwards (sequential, parallel over value-column slices) -> workspace,
-//      and dS0;
+//   2. the state gradient dS' entering chunks from above, walking the chunks backwards ->
+//      workspace, and dS0: for bf16 with dk = dv = 128 the tcgen05 kernel's reverse
+//      instantiation (64-token chunks; gradients at the span ends), else bwd_dstate_kernel
+//      (CUDA cores, 32-token chunks, every chunk's end);
 //   3. bwd_chunk_kernel: every 64-token span in parallel (its two chunks in turn; the first
 //      forms the middle state for the second), from S_c and dS' -> dq, dk, dv, dg, db, dw.
 // Pair decays are formed as exp(gamma_i - gamma_j) with i >= j, never as a product of two
-// exponentials, so no factor overflows for a forgetting decay.
+// exponentials, so no factor overflows for a forgetting decay.  The CUDA-core kernels are
+// fp32 throughout.
 #include <type_traits>
 
 #include "common.cuh"
