@@ -254,14 +254,17 @@ def cpu_oracle_sample(name, target_cpu_s=15.0):
         mixer.mixer_fwd(d["q"], d["k"], d["v"], d["xg"], d["xb"], d["xw"], d["z"], d["weight"], d["S0"],
                         mode=c["mode"], token_major=True)
         t_head = time.perf_counter() - t0
-        n = max(1, min(c["B"] * c["H"], int(target_cpu_s / max(t_head, 1e-3))))
+        # a batch of sampled sequence-heads (the same draw repeated), so that the recurrence
+        # oracle's threads have one head each
+        n = max(cores, int(round(target_cpu_s / max(t_head, 1e-3) / cores)) * cores)
+        n = min(n, c["B"] * c["H"])
+        rep = lambda x: None if x is None else x.expand(n, *x.shape[1:]).contiguous()
         t0 = time.perf_counter()
-        for _ in range(n):
-            mixer.mixer_fwd(d["q"], d["k"], d["v"], d["xg"], d["xb"], d["xw"], d["z"], d["weight"], d["S0"],
-                            mode=c["mode"], token_major=True)
+        mixer.mixer_fwd(rep(d["q"]), rep(d["k"]), rep(d["v"]), rep(d["xg"]), rep(d["xb"]), rep(d["xw"]),
+                        rep(d["z"]), d["weight"], rep(d["S0"]), mode=c["mode"], token_major=True)
         dt = time.perf_counter() - t0
-        return dict(value=n * c["T"] / dt, unit="token-heads/s", cores=1, kind="oracle",
-                    sample=f"{n} sequence-heads x T={c['T']} of mixer_t4k, one after another")
+        return dict(value=n * c["T"] / dt, unit="token-heads/s", cores=min(cores, n), kind="oracle",
+                    sample=f"{n} sequence-heads x T={c['T']} of mixer_t4k, one batch")
     if name == "bwd_t4k":
         wl, mode = rank_workload(name, 0)
         small = workload.Workload("sample", B=1, H=1, T=wl.T, dk=wl.dk, dv=wl.dv, chunk=wl.chunk,
@@ -627,9 +630,9 @@ def run_ours(args, rank, world, local):
 # keyed by workload and by a digest of the kernel's sources at capture time (a changed
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
-    ("gdn2_t4k", "chunk_tc"): (948.148736e6 + 124.496384e6, "94174cc5"),
+    ("gdn2_t4k", "chunk_tc"): (948.148736e6 + 124.496384e6, "153348a5"),
     ("decode", "decode"): (275.810304e6 + 212.322560e6, "6e1ae928"),
-    ("mixer_t4k", "chunk_tc"): (1090.819072e6 + 124.780800e6, "94174cc5"),
+    ("mixer_t4k", "chunk_tc"): (1090.819072e6 + 124.780800e6, "153348a5"),
 }
 
 
@@ -676,8 +679,6 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="decode steps per bench step (default: the workload's 1000); fewer keep an "
                          "ncu capture's launch count small")
-    ap.add_argument("--traffic", type=float, default=None,
-                    help="ncu dram bytes per launch of the dominant kernel, if captured for this build")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -38,7 +38,6 @@ namespace gdr {
 namespace {
 
 constexpr int C = kBwdChunk;
-constexpr int kThreads = 256;
 constexpr int kThreadsC = 512;          // the per-chunk kernel: 16 warps
 constexpr int RW = C / (kThreadsC / 32); // rows of a tiled product per warp (2)
 

@@ -153,7 +153,7 @@ __device__ __forceinline__ void st_tmem_bf16(uint32_t taddr, const float (&x)[32
 __device__ __forceinline__ void group_sync(int id) {
     asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
 }
-// barrier over one warp group that also returns the AND (or the OR) of v over it
+// barrier over one warp group that also returns the AND of v over it
 __device__ __forceinline__ bool group_and(int id, bool v) {
     uint32_t r;
     asm volatile(
@@ -166,22 +166,7 @@ __device__ __forceinline__ bool group_and(int id, bool v) {
         : "memory");
     return r != 0;
 }
-__device__ __forceinline__ bool group_or(int id, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.or.pred p, %2, 256, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "r"(id)
-        : "memory");
-    return r != 0;
-}
 // the same over 128 threads (warps 4-7 of the WY group)
-__device__ __forceinline__ void bar128_sync(int id) {
-    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
-}
 __device__ __forceinline__ bool bar128_and(int id, bool v) {
     uint32_t r;
     asm volatile(
