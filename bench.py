@@ -12,7 +12,8 @@ head), inputs resident in HBM.  Workloads (synthetic, seeded; workload/):
   mixer_t4k  the T=4K shape through gdr_mixer_fwd: raw token-major projections in, the
              RMSNorm-SiLU-gated output out (activations and epilogue fused in the kernel)
   bwd_t4k    the backward (gdr_chunk_bwd) of gdn2_t4k: dq, dk, dv, dg, db, dw and dS0 from dO
-             and dS_T (three launches; fp32 CUDA cores)
+             and dS_T (four launches on the tcgen05 tensor cores; the last, for strong-decay
+             spans, has none here)
   decode     256 sequences x 16 heads, one token per step, state in place
 Metric: token-heads/s (tokens/s per head-layer) = B*H*T / step time (decode:
 step-heads/s).  With N ranks every rank runs its own copy of the workload on its
@@ -88,15 +89,11 @@ def bwd_bytes(wl: workload.Workload) -> float:
 
 
 def bwd_flops(wl: workload.Workload) -> float:
-    """Dense products of the chunkwise backward (32-token chunks) per token-head:
-    24 C d + 20 d^2 (states 4C^2d + 4Cd^2, state gradient 4C^2d + 6Cd^2, per-chunk
-    gradients 16C^2d + 10Cd^2 per chunk of C tokens)."""
-    C, d = 32, max(wl.dk, wl.dv)
-    return wl.units * (24.0 * C * d + 20.0 * d * d)
-
-
-# fp32 FMA lanes of a B200 at its maximum SM clock: 148 SMs x 128 lanes x 2 flops x 1.965 GHz
-ALU_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+    """Tensor-core products of the backward per token-head, 64-token chunks: 22 d^2 + 40 C d
+    (checkpoints: the forward's 6 d^2 + 10 C d; state gradient 6 d^2 + 8 C d; per-chunk
+    gradients 10 d^2 + 22 C d, i.e. 5 C d^2 + 11 C^2 d multiply-adds per chunk)."""
+    C, d = 64, max(wl.dk, wl.dv)
+    return wl.units * (22.0 * d * d + 40.0 * C * d)
 
 
 def decode_bytes(cfg) -> float:
@@ -338,7 +335,7 @@ def metric_name(name):
     if name == "mixer_t4k":
         return "token-mixer fwd tokens/s per head·layer at T=4K (fused prologue/epilogue); % HBM roofline"
     if name == "bwd_t4k":
-        return "chunked bwd tokens/s per head·layer at T=4K (dq, dk, dv, dg, db, dw, dS0); % fp32 ALU roofline"
+        return "chunked bwd tokens/s per head·layer at T=4K (dq, dk, dv, dg, db, dw, dS0); % HBM roofline"
     return "chunked fwd tokens/s per head·layer at T=4K; % tensor-pipe / HBM roofline"
 
 
@@ -411,7 +408,7 @@ def run_ours(args, rank, world, local):
         step = fwd
         units = wl.units
         bytes_per_launch = bwd_bytes(wl)
-        launches_per_step = 3
+        launches_per_step = 4
         unit = "token-heads/s"
         nseg = 1
     elif name == "decode":
@@ -584,9 +581,11 @@ def run_ours(args, rank, world, local):
         launch_ms = kern_ms
         kname = "gdr chunk_tc_kernel<mixer> (tcgen05, fused prologue/epilogue)"
     elif name == "bwd_t4k":
-        # one step = the whole backward (states, state gradient, per-chunk gradients)
+        # one step = the whole backward (states, state gradient, per-chunk gradients, and the
+        # CUDA-core kernel for strong-decay spans, none here), the unit of the roofline
         launch_ms = kern_ms
-        kname = "gdr chunk_simt_kernel + bwd_dstate_kernel + bwd_chunk_kernel (backward, 3 launches)"
+        kname = ("gdr chunk_tc_kernel (checkpoints) + chunk_tc_kernel (state gradient) + bwd_tc_kernel"
+                 " + bwd_chunk_kernel (backward, 4 launches, tcgen05)")
     else:
         # one step = the whole forward; with a sequence split it is three launches
         # (state pass, combine, output pass) and the step is the unit of the roofline
@@ -597,15 +596,8 @@ def run_ours(args, rank, world, local):
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": traffic_for(name, kname), "peak_source": f"{peak_src} hbm_gbs",
             "kernel": kname}
-    if name == "bwd_t4k":
-        fl = bwd_flops(wl) / (launch_ms * 1e-3) / 1e12
-        roof = {"bound": "alu", "achieved": fl, "peak": ALU_FP32_TFLOPS, "unit": "TFLOP/s",
-                "frac": fl / ALU_FP32_TFLOPS, "traffic": None,
-                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz", "kernel": kname,
-                "hbm_context": {"bytes_per_step": bytes_per_launch, "achieved_gbs": achieved,
-                                "frac": achieved / hbm}}
-    if name not in ("decode", "mixer_t4k", "bwd_t4k"):
-        fl = chunk_flops(wl)
+    if name not in ("decode", "mixer_t4k"):
+        fl = bwd_flops(wl) if name == "bwd_t4k" else chunk_flops(wl)
         roof["tensor_context"] = {"flops_per_launch": fl,
                                   "achieved_tflops": fl / (launch_ms * 1e-3) / 1e12,
                                   "peak_tflops": tf_burst,
@@ -613,8 +605,7 @@ def run_ours(args, rank, world, local):
     line = {"metric": metric_name(name), "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32" if name == "bwd_t4k" else
-                     ("bf16" if (name in ("decode", "mixer_t4k") or wl.dtype == "bf16") else "f32"),
+            "dtype": "bf16" if (name in ("decode", "mixer_t4k", "bwd_t4k") or wl.dtype == "bf16") else "f32",
             "data": "synthetic", "config": config_of(name, world), "roofline": roof,
             "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "wall_total_ms": total_ms}

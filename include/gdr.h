@@ -230,10 +230,11 @@ gdr_status_t gdr_mixer_fwd(const void *q, const void *k, const void *v, const fl
  * runs the chunkwise WY algorithm with a gate-aware backward: Gated DeltaNet-2 Review
  * §4-3; Gated DeltaNet-2 Q&A page, Q4).  The backward differentiates the chunkwise form:
  * it recomputes the states at every 64-token boundary, walks the chunks backwards for the
- * state gradient, then forms every 32-token chunk's input gradients in parallel.  For
- * bf16 with dk = dv = 128 the first two run on the tcgen05 tensor cores (bf16 operands,
- * fp32 accumulation); the per-chunk gradients, and everything for other shapes, run in
- * fp32 on CUDA cores.  Equal to the adjoint of the sequential recurrence up to rounding.
+ * state gradient, then forms every chunk's input gradients in parallel.  For bf16 with
+ * dk = dv = 128 all three run on the tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation), 64-token chunks; a chunk whose cumulative decay exceeds e^-60 is done in
+ * fp32 on CUDA cores with exact per-pair decays, as is everything for other shapes (32-token
+ * chunks).  Equal to the adjoint of the sequential recurrence up to rounding.
  *
  *   dO      [B,H,T,dv], element type `dtype`.       dS_T  fp32 [B,H,dk,dv] or NULL (= 0).
  *   dq, dk  [B,H,T,dk]; dv [B,H,T,dv]; db, dw shaped like b, w; all of type `dtype`.

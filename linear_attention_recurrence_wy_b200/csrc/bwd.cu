@@ -29,10 +29,12 @@
 // Pair decays are formed as exp(gamma_i - gamma_j) with i >= j, never as a product of two
 // exponentials, so no factor overflows for a forgetting decay.  The CUDA-core kernels are
 // fp32 throughout.
+#include <algorithm>
 #include <type_traits>
 
-#include "common.cuh"
+#include "bwd_tc.cuh"
 #include "chunk_tc.cuh"
+#include "common.cuh"
 
 namespace gdr {
 namespace {
@@ -262,8 +264,13 @@ template <int RPG, int NE>
 __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     const int dk = a.dk_, dv = a.dv_, T = a.T;
     const int nc = (T + C - 1) / C, nspan = (T + 2 * C - 1) / (2 * C);
-    const int bh = blockIdx.x / nspan, span = blockIdx.x - bh * nspan;
     const int tid = threadIdx.x, nth = blockDim.x;
+    // this CTA's span, or with tc_list every gridDim.x-th listed span
+    const int njobs = a.tc_list ? a.tc_list[0] : (int)gridDim.x;
+  for (int job = blockIdx.x; job < njobs; job += gridDim.x) {
+    const int blk = a.tc_list ? a.tc_list[1 + job] : job;
+    const int bh = blk / nspan, span = blk - bh * nspan;
+    __syncthreads();   // the previous span's shared-memory reads are done
     if (a.mid_grad && 2 * span + 1 < nc) {
         // The state gradient at the span's middle, from its end by one step of the reverse
         // recurrence over the second chunk: dS_mid = e^gamma_C dS_end + Qg^T dO - Kh^T dR
@@ -656,13 +663,21 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
         if (scalar_g) a.dg[tk] = fg[i];
     }
   }
+  }
 }
 
 }  // namespace
 
-unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv) {
+unsigned long long bwd_states_bytes(int B, int H, int T, int dk, int dv) {
     const unsigned long long nc = (unsigned long long)((T + C - 1) / C);
     return 2ull * (unsigned long long)B * H * nc * dk * dv * sizeof(float);
+}
+
+unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv) {
+    if (T <= 0) return 0;
+    const unsigned long long nspan = (unsigned long long)((T + 2 * C - 1) / (2 * C));
+    const unsigned long long list = (1ull + (unsigned long long)B * H * nspan) * sizeof(int);
+    return bwd_states_bytes(B, H, T, dk, dv) + (list + 15) / 16 * 16;
 }
 
 gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
@@ -688,6 +703,12 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
         r.dO = a.dO;
         if ((st = launch_chunk_tc(r, s)) != GDR_OK) return st;
         b.mid_grad = 1;
+        // 3. per-chunk gradients on the tensor cores; spans with a strong cumulative decay
+        //    are listed for the CUDA-core kernel below
+        b.tc_list = reinterpret_cast<int *>(reinterpret_cast<unsigned char *>(a.ws_states) +
+                                            bwd_states_bytes(a.B, a.H, a.T, a.dk_, a.dv_));
+        if (cudaMemsetAsync(b.tc_list, 0, sizeof(int), s) != cudaSuccess) return GDR_ERR_CUDA;
+        if ((st = launch_bwd_tc(b, s)) != GDR_OK) return st;
     } else {
         // 2. state gradients on CUDA cores, chunks in reverse (every 32-token chunk's end)
         const int VS = dslice(a.dv_);
@@ -698,8 +719,11 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
         kern2<<<dim3((unsigned)(a.B * a.H), (unsigned)(a.dv_ / VS)), kThreadsS, smem2, s>>>(a);
         if (cudaGetLastError() != cudaSuccess) return GDR_ERR_CUDA;
     }
-    // 3. per-chunk gradients, one CTA per 64-token span
+    // 3. per-chunk gradients on CUDA cores, one CTA per 64-token span (with tc_list: the
+    //    listed spans, over at most four CTAs per SM)
     const int nspan = (a.T + 2 * C - 1) / (2 * C);
+    size_t grid = (size_t)a.B * a.H * nspan;
+    if (b.tc_list) grid = std::min(grid, (size_t)4 * 148);
     const size_t smem3 = chunk_smem_floats(a.dk_, a.dv_) * sizeof(float);
     // RPG rows per thread for the (token, key channel) gradients; NE column groups of 32
     // for the tiled products over the value channels
@@ -713,7 +737,7 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
                              : pick(std::integral_constant<int, C * 16 / kThreadsC>{});
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3) != cudaSuccess)
         return GDR_ERR_CUDA;
-    kern<<<(unsigned)((size_t)a.B * a.H * nspan), kThreadsC, smem3, s>>>(b);
+    kern<<<(unsigned)grid, kThreadsC, smem3, s>>>(b);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

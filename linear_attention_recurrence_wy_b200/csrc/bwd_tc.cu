@@ -1,0 +1,644 @@
+// bwd_tc.cu -- the backward's per-chunk gradients on the tcgen05 tensor cores: bf16
+// operands, fp32 accumulation in tensor memory (TMEM).
+//
+// Shape: dk = dv = 128, bf16 inputs, 64-token chunks, any mode.  One CTA (256 threads) per
+// (sequence, head, 64-token chunk): given the state S at the chunk's start (the checkpoint
+// pass) and the state gradient dS' at its end (the state-gradient pass), every chunk is
+// independent.  With gamma the chunk-local cumulative log-decay, Kh = b.k.e^gamma,
+// Qg = q.e^gamma, Kb = k.e^-gamma, W = w.v and dS~ = diag(e^gamma_C) dS' (the chunkwise WY
+// form of Gated DeltaNet-2 Review §3-2.5, differentiated for the gate-aware backward of
+// §4-3 and of the Gated DeltaNet-2 Q&A page, Q4):
+//
+//   forward   [A; P] = [Kh; Qg] Kb^T        T = (I + A)^-1        X^T = S^T Kh^T
+//             R^T = W^T - X^T               E^T = R^T T^T          (E = T (W - Kh S))
+//   backward  dE^T = dS~^T Kb^T + dO^T P    dR^T = dE^T T          (dR = T^T dE)
+//             [dA; dP] = [-dR; dO] E^T      dA strictly lower, dP lower incl. (diagonal apart)
+//             [dKh | dQg]^T = S [-dR; dO]^T + Kb^T [dA; dP]^T
+//             dKb^T = [Kh; Qg]^T [dA; dP]   dKe^T = dS~ E^T
+//
+// The gradient of A needs no products with T: dA = -T^T (dE R^T) T^T = -(T^T dE)(T R)^T =
+// -dR E^T, so dA and dP share one MMA.  dKe is e^gamma_C times the gradient of
+// Ke = k.e^(gamma_C - gamma), the key operand of the state update, so it enters exactly
+// like dKb.  The diagonal of dP pairs a token with itself, where the decay factors cancel:
+// it is left out of the MMA operand (whose rounding would leave a residue in dgamma of the
+// size of the whole pair term) and added as dP_tt k_t to dq and dP_tt q_t to dk.  Per
+// (token, key channel), on CUDA cores:
+//
+//   dq = dQg e^gamma + dP_tt k      dk = dKh b e^gamma + (dKb + dKe) e^-gamma + dP_tt q
+//   db = dKh k e^gamma              dgamma = dQg Qg + dKh Kh - (dKb + dKe) Kb
+//   dgamma_C = sum_v S dS~ + sum_t dKe Kb       dg = dgamma_C + reverse cumulative sum of dgamma
+//
+// and per (token, value channel) dv = dR w, dw = dR v (scalar gates fold over channels).
+// Every factor stays within e^+-60 when |gamma| <= 60 on the whole chunk.  A chunk with a
+// stronger cumulative decay is left to the CUDA-core kernel (exact per-pair decays): the
+// CTA appends its index to the list that kernel works through.
+//
+// Every wait on an mbarrier is bounded; on expiry the CTA records the failure in
+// g_bwd_tc_error, waits (bounded) for its own tensor-core work and copies, frees its TMEM
+// and returns.
+#include "bwd_tc.cuh"
+#include "tc_util.cuh"
+#include "tri_inverse.cuh"
+
+namespace gdr {
+
+__device__ int g_bwd_tc_error = 0;
+
+namespace {
+
+using namespace tc;
+
+constexpr int C = 64, DK = 128, DV = 128;
+constexpr int kThreads = 256;
+constexpr uint32_t kWaitLimit = 1u << 24;
+constexpr float kFastLimit = 60.f;
+
+// shared memory map (byte offsets from a 1024-aligned base)
+constexpr int OFF_RQ = 0;                 // raw q bf16 [64][128]                        16 KB
+constexpr int OFF_RK = OFF_RQ + 16384;    // raw k                                       16 KB
+constexpr int OFF_RB = OFF_RK + 16384;    // raw b (per-channel erase gate)              16 KB
+constexpr int OFF_G = OFF_RB + 16384;     // raw g_log fp32 [64][128], e^gamma, dgamma   32 KB
+constexpr int OFF_SB = OFF_G + 32768;     // S   bf16 [128 d][128 v]                     32 KB
+constexpr int OFF_DSB = OFF_SB + 32768;   // dS~ bf16 [128 d][128 v]                     32 KB
+constexpr int OFF_QK = OFF_DSB + 32768;   // [Kh; Qg] bf16 [128][128 d]                  32 KB
+constexpr int OFF_KB = OFF_QK + 32768;    // Kb bf16 [64 t][128 d]                       16 KB
+constexpr int OFF_P = OFF_KB + 16384;     // P bf16 [64 t][64 j]                          8 KB
+constexpr int OFF_T = OFF_P + 8192;       // T bf16 [64 t][64 j]                          8 KB
+// regions reused once their first contents are dead
+constexpr int OFF_A32 = OFF_RQ;           // A, then T, fp32 [64][68] (after the operand build)
+constexpr int OFF_X = OFF_A32 + 64 * tri::LD * 4;   // the inverse's scratch, 4 x [16][20] fp32
+constexpr int OFF_DOR = OFF_RQ;           // [-dR^T | dO^T] bf16 [128 v][128] (after the inverse)
+constexpr int OFF_ET = OFF_RB;            // E^T bf16 [128 v][64 t]                      16 KB
+constexpr int OFF_DAP = OFF_P;            // [dA; dP] bf16 [128][64 j] (over P and T)    16 KB
+// small arrays
+constexpr int OFF_GC = OFF_T + 8192;      // gamma_C fp32 [128]
+constexpr int OFF_EGC = OFF_GC + 512;     // exp(gamma_C) [128]
+constexpr int OFF_DGC = OFF_EGC + 512;    // sum_v S dS~ per key channel [128]
+constexpr int OFF_CAR = OFF_DGC + 512;    // the epilogue's exchange between token halves [3][128]
+constexpr int OFF_BETA = OFF_CAR + 1536;  // scalar erase gate of the chunk's tokens [64]
+constexpr int OFF_GS = OFF_BETA + 256;    // scalar g_log (GDN) [64]
+constexpr int OFF_FOLD = OFF_GS + 256;    // scalar-gate gradients [3][64]: b, w, g
+constexpr int OFF_DPD = OFF_FOLD + 768;   // the diagonal of dP [64]
+constexpr int OFF_FLAG = OFF_DPD + 256;   // [0] strong decay (exact path), [1] abort
+constexpr int OFF_BAR = OFF_FLAG + 16;    // mbarriers: raw copies, MMA commits; TMEM slot
+constexpr int SMEM_BYTES = OFF_BAR + 2 * 8 + 8 + 1024;   // + alignment slack
+static_assert(OFF_X + 4 * 16 * tri::XLD * 4 <= OFF_RB, "the inverse's scratch fits over raw q and k");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+
+// TMEM columns (fp32 unless noted); lane = value channel for X, E, dE, dR, lane = key
+// channel for dKh, dQg, dKb, dKe, lane = row of [A; P] and [dA; dP]
+constexpr uint32_t TM_AP = 0;      // [A; P], then [dA; dP]                             64
+constexpr uint32_t TM_X = 64;      // X^T, then dR^T                                    64
+constexpr uint32_t TM_E = 128;     // E^T                                               64
+constexpr uint32_t TM_DE = 192;    // dE^T                                              64
+constexpr uint32_t TM_DQK = 256;   // [dKh | dQg]^T                                    128
+constexpr uint32_t TM_DKB = 384;   // dKb^T; before it, dE^T bf16 (packed)              64
+constexpr uint32_t TM_DKE = 448;   // dKe^T; before it, R^T and dO^T bf16 (packed)      64
+constexpr uint32_t TM_DEB = TM_DKB;
+constexpr uint32_t TM_RB = TM_DKE;
+constexpr uint32_t TM_DOB = TM_DKE + 32;
+constexpr uint32_t TM_COLS = 512;
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
+
+// sum over the 32 lanes of a warp, returned to every lane
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;                       // TMEM lanes 32 quarter .. + 31
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int r = quarter * 32 + lane;                  // this thread's TMEM lane
+    const int j0 = (warp >> 2) * 32;                    // and its 32 token columns
+
+    // ---- this CTA's chunk ----
+    const int T = a.T, mode = a.mode;
+    const int nchunk = (T + C - 1) / C;
+    const int bh = blockIdx.x / nchunk, c = blockIdx.x - bh * nchunk;
+    const int t0 = c * C, n = min(C, T - t0);
+    const size_t tok0 = (size_t)bh * T + t0;            // row of the chunk's first token
+    // the workspace holds one fp32 state per 32-token chunk: S at this chunk's start is in
+    // the slot of its first 32-token chunk, dS' at its end in the slot of its last one
+    const int nslot = (T + kBwdChunk - 1) / kBwdChunk;
+    const float *Sg = a.ws_states + ((size_t)bh * nslot + 2 * c) * DK * DV;
+    const float *dSg = a.ws_dstates + ((size_t)bh * nslot + min(2 * c + 1, nslot - 1)) * DK * DV;
+
+    const __nv_bfloat16 *Q = (const __nv_bfloat16 *)a.q, *K = (const __nv_bfloat16 *)a.k;
+    const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
+    const __nv_bfloat16 *Wg = (const __nv_bfloat16 *)a.w, *dOg = (const __nv_bfloat16 *)a.dO;
+    __nv_bfloat16 *dQo = (__nv_bfloat16 *)a.dq, *dKo = (__nv_bfloat16 *)a.dk;
+    __nv_bfloat16 *dVo = (__nv_bfloat16 *)a.dv, *dBo = (__nv_bfloat16 *)a.db, *dWo = (__nv_bfloat16 *)a.dw;
+    // gate shapes: per-channel erase b (GDN-2, b-only), per-channel write w (GDN-2, w-only),
+    // per-channel decay (all but GDN); a scalar write gate is w itself (b-only) or beta in b
+    const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
+    const bool tied = mode == GDR_MODE_KDA || mode == GDR_MODE_GDN;
+    const __nv_bfloat16 *Wsc = mode == GDR_MODE_BONLY ? Wg : Bg;
+
+    float *sG = reinterpret_cast<float *>(sm + OFF_G);
+    float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
+    float *sX = reinterpret_cast<float *>(sm + OFF_X);
+    float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
+    float *sEGC = reinterpret_cast<float *>(sm + OFF_EGC);
+    float *sDGC = reinterpret_cast<float *>(sm + OFF_DGC);
+    float *sCar = reinterpret_cast<float *>(sm + OFF_CAR);
+    float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
+    float *sGs = reinterpret_cast<float *>(sm + OFF_GS);
+    float *sFb = reinterpret_cast<float *>(sm + OFF_FOLD), *sFw = sFb + 64, *sFg = sFb + 128;
+    float *sDPd = reinterpret_cast<float *>(sm + OFF_DPD);
+    volatile int *sFlag = reinterpret_cast<volatile int *>(sm + OFF_FLAG);
+    const uint32_t bar_raw = sbase + OFF_BAR, bar_mma = bar_raw + 8;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
+
+    if (tid == 0) {
+        mbar_init(bar_raw, 1);
+        mbar_init(bar_mma, 1);
+        sFlag[0] = 0;
+        sFlag[1] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tslot), TM_COLS);
+        tmem_relinquish();
+    }
+    // the T tile's blocks above the diagonal are never written by the inverse
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid + kThreads] = make_uint4(0, 0, 0, 0);
+    static_assert(kThreads * 32 == 8192, "two 16-byte stores per thread clear the T tile");
+    if (tid < 192) sFb[tid] = 0.f;
+    // scalar gates of the chunk's tokens, zero past the end
+    if (tid < 64) {
+        if (!vec_g) sGs[tid] = tid < n ? a.g[tok0 + tid] : 0.f;
+    } else if (tid < 128) {
+        if (!vec_b) sBeta[tid - 64] = tid - 64 < n ? bf(Bg, tok0 + tid - 64) : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    int commits = 0;          // MMA commits issued on bar_mma (thread 0)
+    bool raw_pending = false;
+    // Bounded wait for a phase of an mbarrier: thread 0 polls, the block meets at a barrier.
+    auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (tid == 0 && !mbar_wait(bar, parity, kWaitLimit)) sFlag[1] = 1;
+        __syncthreads();
+        return sFlag[1] == 0;
+    };
+    auto wait_mma = [&]() -> bool { return wait_bar(bar_mma, (uint32_t)((commits - 1) & 1)); };
+
+    do {
+        // ---- 1. raw q, k, b, g_log of the chunk: one bulk copy per tensor ----
+        if (tid == 0) {
+            const uint32_t row16 = (uint32_t)n * DK * 2;
+            fence_async_smem();
+            mbar_arrive_expect_tx(bar_raw, 2 * row16 + (vec_b ? row16 : 0) + (vec_g ? 2 * row16 : 0));
+            bulk_g2s(sbase + OFF_RQ, Q + tok0 * DK, row16, bar_raw);
+            bulk_g2s(sbase + OFF_RK, K + tok0 * DK, row16, bar_raw);
+            if (vec_b) bulk_g2s(sbase + OFF_RB, Bg + tok0 * DK, row16, bar_raw);
+            if (vec_g) bulk_g2s(sbase + OFF_G, a.g + tok0 * DK, 2 * row16, bar_raw);
+        }
+        raw_pending = true;
+        // S -> bf16 tile (warp w: rows 16 w .. 16 w + 15; lane: columns 4 lane .. + 3)
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float4 x[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                x[i] = *reinterpret_cast<const float4 *>(Sg + (size_t)(warp * 16 + h * 8 + i) * DV + 4 * lane);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                st_shared_v2(sbase + OFF_SB + tile_off(128, warp * 16 + h * 8 + i, 4 * lane),
+                             pack_bf16(x[i].x, x[i].y), pack_bf16(x[i].z, x[i].w));
+        }
+        // dO^T of this thread's value channel and tokens -> bf16 in TMEM (zero past the end)
+        {
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = (j0 + j < n) ? bf(dOg, (tok0 + j0 + j) * DV + r) : 0.f;
+            st_tmem_bf16(tmem + lane_base + TM_DOB + j0 / 2, x);
+        }
+        if (!wait_bar(bar_raw, 0)) break;
+        raw_pending = false;
+        // ---- 2. cumulative log-decay: thread d < 128 scans key channel d and leaves e^gamma
+        //      in place of g_log; any |gamma| > 60 sends the chunk to the exact path ----
+        if (tid < DK) {
+            const int d = tid;
+            float acc = 0.f, mx = 0.f;
+#pragma unroll 1
+            for (int b = 0; b < C; b += 16) {
+                float x[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = vec_g ? sG[(b + i) * DK + d] : sGs[b + i];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    acc += (b + i < n) ? x[i] : 0.f;
+                    mx = fmaxf(mx, fabsf(acc));
+                    x[i] = __expf(acc);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sG[(b + i) * DK + d] = x[i];
+            }
+            sGC[d] = acc;
+            sEGC[d] = __expf(acc);
+            if (mx > kFastLimit) sFlag[0] = 1;
+        }
+        __syncthreads();
+        if (sFlag[0]) {
+            if (tid == 0) a.tc_list[1 + atomicAdd(a.tc_list, 1)] = blockIdx.x;
+            break;
+        }
+        // ---- 3. operands: Kh, Qg, Kb (thread (tg, cg): tokens 4 tg .. + 3, channels
+        //      8 cg .. + 7), and dS~ with sum_v S dS~ per key channel ----
+        {
+            const int tg = tid >> 4, cg = tid & 15;
+#pragma unroll 1
+            for (int i = 0; i < 4; ++i) {
+                const int t = tg * 4 + i;
+                const bool in = t < n;
+                const uint32_t ro = (uint32_t)(t * DK * 2 + cg * 16);
+                float fq[8], fk[8], fb[8];
+                bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + OFF_RQ + ro)), fq);
+                bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + OFF_RK + ro)), fk);
+                if (vec_b) {
+                    bf16x8_to_f32(sel(in, *reinterpret_cast<const uint4 *>(sm + OFF_RB + ro)), fb);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) fb[j] = sBeta[t];
+                }
+                const float4 g0 = *reinterpret_cast<const float4 *>(sG + t * DK + cg * 8);
+                const float4 g1 = *reinterpret_cast<const float4 *>(sG + t * DK + cg * 8 + 4);
+                const float e[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                float kh[8], qg[8], kb[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    kh[j] = fb[j] * fk[j] * e[j];
+                    qg[j] = fq[j] * e[j];
+                    kb[j] = fk[j] * rcp_approx(e[j]);
+                }
+                st_chunk(sbase + OFF_QK + tile_chunk(128, t, cg), kh);
+                st_chunk(sbase + OFF_QK + tile_chunk(128, 64 + t, cg), qg);
+                st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
+            }
+        }
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+            float4 xs[8], xd[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const size_t o = (size_t)(warp * 16 + h * 8 + i) * DV + 4 * lane;
+                xs[i] = *reinterpret_cast<const float4 *>(Sg + o);
+                xd[i] = *reinterpret_cast<const float4 *>(dSg + o);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int d = warp * 16 + h * 8 + i;
+                const float eg = sEGC[d];
+                const float y0 = xd[i].x * eg, y1 = xd[i].y * eg, y2 = xd[i].z * eg, y3 = xd[i].w * eg;
+                st_shared_v2(sbase + OFF_DSB + tile_off(128, d, 4 * lane), pack_bf16(y0, y1), pack_bf16(y2, y3));
+                const float s = warp_sum(xs[i].x * y0 + xs[i].y * y1 + xs[i].z * y2 + xs[i].w * y3);
+                if (lane == 0) sDGC[d] = s;
+            }
+        }
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        // ---- 4. [A; P] = [Kh; Qg] Kb^T,  X^T = S^T Kh^T,  dE^T = dS~^T Kb^T ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_kk = idesc_bf16(128, 64, false, false, false);
+            const uint32_t id_mk = idesc_bf16(128, 64, true, false, false);
+#pragma unroll
+            for (int s = 0; s < DK / 16; ++s) {
+                mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s), desc_kmajor(sbase + OFF_KB, 64, 0, s),
+                         id_kk, s > 0);
+                mma_bf16(tmem + TM_X, desc_mnmajor(sbase + OFF_SB, 128, 0, s), desc_kmajor(sbase + OFF_QK, 128, 0, s),
+                         id_mk, s > 0);
+                mma_bf16(tmem + TM_DE, desc_mnmajor(sbase + OFF_DSB, 128, 0, s), desc_kmajor(sbase + OFF_KB, 64, 0, s),
+                         id_mk, s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ++commits;
+        // W = w.v of this thread's value channel and tokens, while the MMAs run
+        float wv[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int t = j0 + j;
+            float x = 0.f;
+            if (t < n) {
+                const size_t tk = tok0 + t;
+                x = bf(V, tk * DV + r) * (vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk));
+            }
+            wv[j] = x;
+        }
+        if (!wait_mma()) break;
+        tc_fence_after();
+        // ---- 5. A (fp32, strictly lower) -> inverse scratch; P (lower incl.) -> bf16 tile;
+        //      R^T = W^T - X^T -> bf16 in TMEM ----
+        {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_AP + j0, x);
+            tmem_wait_ld();
+            if (r < 64) {
+                float4 *dst = reinterpret_cast<float4 *>(sA32 + r * tri::LD + j0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float y[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
+                    dst[q] = make_float4(y[0], y[1], y[2], y[3]);
+                }
+            } else {
+                const int t = r - 64;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
+                    st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+                }
+            }
+            tmem_ld32(tmem + lane_base + TM_X + j0, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = wv[j] - x[j];
+            st_tmem_bf16(tmem + lane_base + TM_RB + j0 / 2, x);
+        }
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        // ---- 6. dE^T += dO^T P; T = (I + A)^-1 by warps 0-3; then E^T = R^T T^T ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, false, true, false);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16_ts(tmem + TM_DE, tmem + TM_DOB + s * 8, desc_mnmajor(sbase + OFF_P, 64, 0, s), id, 1u);
+        }
+        if (warp < 4) {
+            tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});   // in place
+            fence_async_smem();
+        }
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16_ts(tmem + TM_E, tmem + TM_RB + s * 8, desc_kmajor(sbase + OFF_T, 64, 0, s), id, s > 0);
+            mma_commit(bar_mma);
+        }
+        ++commits;
+        if (!wait_mma()) break;
+        tc_fence_after();
+        // ---- 7. E^T -> bf16 tile [v][t]; dE^T -> bf16 in TMEM; dO^T -> the right half of
+        //      the [-dR^T | dO^T] tile ----
+        {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_E + j0, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = x[h * 8 + j];
+                st_chunk(sbase + OFF_ET + tile_chunk(128, r, j0 / 8 + h), f);
+            }
+            tmem_ld32(tmem + lane_base + TM_DE + j0, x);
+            tmem_wait_ld();
+            st_tmem_bf16(tmem + lane_base + TM_DEB + j0 / 2, x);
+            float p[16];   // packed bf16 pairs of dO^T, 8 tokens per 16-byte chunk
+            tmem_ld16(tmem + lane_base + TM_DOB + j0 / 2, p);
+            tmem_wait_ld();
+            const uint32_t *u = reinterpret_cast<const uint32_t *>(p);
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                st_shared_v4(sbase + OFF_DOR + tile_chunk(128, r, 8 + j0 / 8 + h), u[4 * h], u[4 * h + 1],
+                             u[4 * h + 2], u[4 * h + 3]);
+        }
+        fence_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        // ---- 8. dR^T = dE^T T,  dKe^T = dS~ E^T ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_t = idesc_bf16(128, 64, false, true, false);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16_ts(tmem + TM_X, tmem + TM_DEB + s * 8, desc_mnmajor(sbase + OFF_T, 64, 0, s), id_t, s > 0);
+#pragma unroll
+            for (int s = 0; s < DV / 16; ++s)
+                mma_bf16(tmem + TM_DKE, desc_kmajor(sbase + OFF_DSB, 128, 0, s), desc_mnmajor(sbase + OFF_ET, 128, 0, s),
+                         id_t, s > 0);
+            mma_commit(bar_mma);
+        }
+        ++commits;
+        if (!wait_mma()) break;
+        tc_fence_after();
+        // ---- 9. dv = dR w, dw = dR v; -dR^T -> the left half of the [-dR^T | dO^T] tile ----
+        {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_X + j0, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int t = j0 + j;
+                float gw = 0.f;
+                if (t < n) {
+                    const size_t tk = tok0 + t;
+                    const float wt = vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk);
+                    dVo[tk * DV + r] = __float2bfloat16_rn(x[j] * wt);
+                    gw = x[j] * bf(V, tk * DV + r);
+                    if (vec_w) dWo[tk * DV + r] = __float2bfloat16_rn(gw);
+                }
+                if (!vec_w) {   // t is the same across the warp: fold over the value channels
+                    const float s = warp_sum(gw);
+                    if (lane == 0 && t < n) atomicAdd(&sFw[t], s);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = -x[h * 8 + j];
+                st_chunk(sbase + OFF_DOR + tile_chunk(128, r, j0 / 8 + h), f);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- 10. [dA; dP] = [-dR; dO] E^T,  [dKh | dQg]^T = S [-dR; dO]^T ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_ap = idesc_bf16(128, 64, true, true, false);
+            const uint32_t id_qk = idesc_bf16(128, 128, false, true, false);
+#pragma unroll
+            for (int s = 0; s < DV / 16; ++s) {
+                mma_bf16(tmem + TM_AP, desc_mnmajor(sbase + OFF_DOR, 128, 0, s), desc_mnmajor(sbase + OFF_ET, 128, 0, s),
+                         id_ap, s > 0);
+                mma_bf16(tmem + TM_DQK, desc_kmajor(sbase + OFF_SB, 128, 0, s), desc_mnmajor(sbase + OFF_DOR, 128, 0, s),
+                         id_qk, s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        ++commits;
+        if (!wait_mma()) break;
+        tc_fence_after();
+        // ---- 11. dA and dP, both strictly lower, -> bf16 tile; dP's diagonal -> sDPd ----
+        {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_AP + j0, x);
+            tmem_wait_ld();
+            const int lim = r < 64 ? r : r - 64;   // columns j < lim are kept
+            if (r >= 64 && lim >= j0 && lim < j0 + 32) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (j0 + j == lim) sDPd[lim] = x[j];
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j < lim) ? x[h * 8 + j] : 0.f;
+                st_chunk(sbase + OFF_DAP + tile_chunk(128, r, j0 / 8 + h), f);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- 12. [dKh | dQg]^T += Kb^T [dA; dP]^T,  dKb^T = [Kh; Qg]^T [dA; dP] ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_qk = idesc_bf16(128, 128, true, false, false);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + TM_DQK, desc_mnmajor(sbase + OFF_KB, 64, 0, s), desc_kmajor(sbase + OFF_DAP, 128, 0, s),
+                         id_qk, 1u);
+            const uint32_t id_kb = idesc_bf16(128, 64, true, true, false);
+#pragma unroll
+            for (int s = 0; s < 128 / 16; ++s)
+                mma_bf16(tmem + TM_DKB, desc_mnmajor(sbase + OFF_QK, 128, 0, s), desc_mnmajor(sbase + OFF_DAP, 128, 0, s),
+                         id_kb, s > 0);
+            mma_commit(bar_mma);
+        }
+        ++commits;
+        if (!wait_mma()) break;
+        tc_fence_after();
+        // ---- 13. per (token, key channel): thread r = d, tokens j0 .. j0 + 31 ----
+        {
+            const int d = r;
+            float ske = 0.f, sdg = 0.f;   // sum_t dKe Kb, sum_t dgamma over this thread's tokens
+#pragma unroll 1
+            for (int g16 = 0; g16 < 2; ++g16) {
+                const int tb = j0 + 16 * g16;
+                float dkh[16], dqg[16], dkb[16], dke[16];
+                tmem_ld16(tmem + lane_base + TM_DQK + tb, dkh);
+                tmem_ld16(tmem + lane_base + TM_DQK + 64 + tb, dqg);
+                tmem_ld16(tmem + lane_base + TM_DKB + tb, dkb);
+                tmem_ld16(tmem + lane_base + TM_DKE + tb, dke);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = tb + i;
+                    const bool in = t < n;
+                    const size_t ix = (tok0 + t) * DK + d;
+                    const float e = sG[t * DK + d], ei = rcp_approx(e);
+                    const float qv = in ? bf(Q, ix) : 0.f, kv = in ? bf(K, ix) : 0.f;
+                    const float bv = vec_b ? (in ? bf(Bg, ix) : 0.f) : sBeta[t];
+                    const float dkbt = dkb[i] + dke[i], dpd = sDPd[t];
+                    const float kbv = kv * ei;
+                    const float gb = dkh[i] * kv * e;
+                    const float dgam = dqg[i] * qv * e + dkh[i] * bv * kv * e - dkbt * kbv;
+                    ske = fmaf(dke[i], kbv, ske);
+                    sdg += dgam;
+                    sG[t * DK + d] = dgam;   // dgamma replaces e^gamma
+                    if (in) {
+                        dQo[ix] = __float2bfloat16_rn(fmaf(dqg[i], e, dpd * kv));
+                        dKo[ix] = __float2bfloat16_rn(fmaf(dkh[i] * bv, e, fmaf(dkbt, ei, dpd * qv)));
+                        if (vec_b) dBo[ix] = __float2bfloat16_rn(gb);
+                    }
+                    if (!vec_b) {   // fold over the key channels
+                        const float s = warp_sum(gb);
+                        if (lane == 0 && in) atomicAdd(&sFb[t], s);
+                    }
+                }
+            }
+            // dgamma_C and the later half's total reach the earlier half through shared memory
+            if (j0) sCar[d] = sdg;
+            sCar[128 * (1 + (j0 >> 5)) + d] = ske;
+            __syncthreads();
+            float acc = sDGC[d] + sCar[128 + d] + sCar[256 + d] + (j0 ? 0.f : sCar[d]);
+#pragma unroll 4
+            for (int i = 31; i >= 0; --i) {
+                const int t = j0 + i;
+                acc += sG[t * DK + d];
+                if (vec_g) {
+                    if (t < n) a.dg[(tok0 + t) * DK + d] = acc;
+                } else {
+                    const float s = warp_sum(acc);
+                    if (lane == 0 && t < n) atomicAdd(&sFg[t], s);
+                }
+            }
+        }
+        __syncthreads();
+        // ---- 14. scalar gates: one gradient per token ----
+        if (tid < n) {
+            const size_t tk = tok0 + tid;
+            if (!vec_b) dBo[tk] = __float2bfloat16_rn(tied ? sFb[tid] + sFw[tid] : sFb[tid]);
+            if (mode == GDR_MODE_BONLY) dWo[tk] = __float2bfloat16_rn(sFw[tid]);
+            if (!vec_g) a.dg[tk] = sFg[tid];
+        }
+    } while (0);
+
+    tmem_wait_st();   // an early exit can leave this thread's dO^T store in flight
+    tc_fence_before();
+    __syncthreads();
+    if (sFlag[1] && tid == 0) {
+        // drain: the raw copies and every committed tensor-core operation
+        atomicExch(&g_bwd_tc_error, 1);
+        if (raw_pending) mbar_wait(bar_raw, 0, kWaitLimit);
+        mma_commit(bar_mma);
+        const int k = commits + 1;
+        if (k >= 2) mbar_wait(bar_mma, (uint32_t)((k - 2) & 1), kWaitLimit);
+        mbar_wait(bar_mma, (uint32_t)((k - 1) & 1), kWaitLimit);
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const BwdArgs &a) { return a.dtype == GDR_BF16 && a.dk_ == DK && a.dv_ == DV; }
+
+gdr_status_t launch_bwd_tc(const BwdArgs &a, cudaStream_t s) {
+    static_assert(2 * kBwdChunk == C, "a chunk here is two of the backward's 32-token chunks");
+    if (cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    const unsigned grid = (unsigned)((size_t)a.B * a.H * ((a.T + C - 1) / C));
+    bwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(a);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+cudaError_t bwd_tc_read_and_clear_error(int *err) {
+    cudaError_t e = cudaMemcpyFromSymbol(err, g_bwd_tc_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_bwd_tc_error, &zero, sizeof(int));
+}
+
+}  // namespace gdr

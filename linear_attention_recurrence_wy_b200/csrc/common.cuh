@@ -91,8 +91,14 @@ struct BwdArgs {
     // 1: ws_dstates holds the state gradient only at the ends of 64-token spans (the
     // tensor-core state-gradient pass); the per-chunk kernel forms the middle ones
     int mid_grad;
+    // [1 + B*H*nspan]: a count, then the indices (b*H + h)*nspan + span of the 64-token spans
+    // the tensor-core per-chunk kernel left to the CUDA-core one; NULL: that kernel takes
+    // every span
+    int *tc_list;
 };
 constexpr int kBwdChunk = 32;   // tokens per chunk of the backward
+// the two state arrays, then tc_list (16-byte multiple)
+unsigned long long bwd_states_bytes(int B, int H, int T, int dk, int dv);
 unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
 gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s);
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "bwd_tc.cuh"
 #include "chunk_tc.cuh"
 
 using namespace gdr;
@@ -221,11 +222,11 @@ extern "C" gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *
     }
     const unsigned long long need = bwd_workspace_bytes(B, H, T, dk, dv);
     if (!workspace || workspace_bytes < need) return GDR_ERR_WORKSPACE;
-    const size_t per = need / 2 / sizeof(float);
+    const size_t per = bwd_states_bytes(B, H, T, dk, dv) / 2 / sizeof(float);
     BwdArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S0, dO, dS_T,
               dq, dk_, dv_, db, mode_uses_w(mode) ? dw : nullptr, dg, dS0,
               B, H, T, dk, dv, (int)mode, (int)dtype,
-              static_cast<float *>(workspace), static_cast<float *>(workspace) + per, 0};
+              static_cast<float *>(workspace), static_cast<float *>(workspace) + per, 0, nullptr};
     return launch_bwd(a, s);
 }
 
@@ -250,10 +251,11 @@ extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void
 extern "C" gdr_status_t gdr_last_device_error(void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_CUDA;
-    int err = 0, derr = 0;
+    int err = 0, derr = 0, berr = 0;
     if (chunk_tc_read_and_clear_error(&err) != cudaSuccess) return GDR_ERR_CUDA;
     if (decode_read_and_clear_error(&derr) != cudaSuccess) return GDR_ERR_CUDA;
-    return (err || derr) ? GDR_ERR_TIMEOUT : GDR_OK;
+    if (bwd_tc_read_and_clear_error(&berr) != cudaSuccess) return GDR_ERR_CUDA;
+    return (err || derr || berr) ? GDR_ERR_TIMEOUT : GDR_OK;
 }
 
 extern "C" const char *gdr_status_string(gdr_status_t status) {

@@ -238,6 +238,60 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
+
+// ---- element conversions and tile stores ------------------------------------------------
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 x = __bfloat1622float2(h[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+    }
+}
+
+// 1/x to within an ulp or two (PTX rcp.approx); x is a normal number here
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// v where in, else zero (a staged row past the end of the input holds stale data)
+__device__ __forceinline__ uint4 sel(bool in, uint4 v) {
+    return make_uint4(in ? v.x : 0u, in ? v.y : 0u, in ? v.z : 0u, in ? v.w : 0u);
+}
+
+// eight fp32 values -> one 16-byte chunk of bf16 at saddr
+__device__ __forceinline__ void st_chunk(uint32_t saddr, const float (&f)[8]) {
+    st_shared_v4(saddr, pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                 pack_bf16(f[6], f[7]));
+}
+
+// 32 fp32 values -> 16 packed bf16 pairs -> TMEM
+__device__ __forceinline__ void st_tmem_bf16(uint32_t taddr, const float (&x)[32]) {
+    uint32_t r[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) r[j] = pack_bf16(x[2 * j], x[2 * j + 1]);
+    tmem_st16(taddr, r);
+}
+
+// Output hook of tri::inverse64 that writes T as bf16 into a 64 x 64 SW128 tile.
+struct TileOut {
+    uint32_t tile;   // shared address of the T tile ([64 t][64 j], 128-byte swizzled)
+    __device__ __forceinline__ void chunk(int row, int c8, const float (&v)[8]) {
+        st_chunk(tile + tile_chunk(64, row, c8), v);
+    }
+    __device__ __forceinline__ void pair(int row, int col, float v0, float v1) {
+        const uint32_t x = pack_bf16(v0, v1);
+        asm volatile("st.shared.b32 [%0], %1;" ::"r"(tile + tile_off(64, row, col)), "r"(x) : "memory");
+    }
+};
+
+// barrier over warps 0-3 (named barrier 1), the inverse's warps
+struct Bar128 {
+    __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+};
 #endif
 
 }  // namespace tc

@@ -166,8 +166,12 @@ def call_bwd(q=A, k=A, v=A, g=A, b=A, w=A, S0=None, dO=A, dST=None, dq=A, dk_=A,
 
 
 def test_bwd_workspace_size(L):
-    # two fp32 states per 32-token chunk and sequence-head
-    assert gdr.gdr_chunk_bwd_workspace(2, 3, 100, 64, 32) == 2 * 2 * 3 * 4 * 64 * 32 * 4
+    # two fp32 states per 32-token chunk and sequence-head, then a count and one index per
+    # 64-token span (the spans the tensor-core kernel leaves to the CUDA-core one), padded
+    # to 16 bytes
+    states = 2 * 2 * 3 * 4 * 64 * 32 * 4
+    assert gdr.gdr_chunk_bwd_workspace(2, 3, 100, 64, 32) == states + 64   # (1 + 2*3*2) ints
+    assert gdr.gdr_chunk_bwd_workspace(1, 1, 64, 128, 128) == 2 * 2 * 128 * 128 * 4 + 16
     assert gdr.gdr_chunk_bwd_workspace(2, 3, 0, 64, 32) == 0
     assert gdr.gdr_chunk_bwd_workspace(2, 3, 10, 48, 32) == 0
 
