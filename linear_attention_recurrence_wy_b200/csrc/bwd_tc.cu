@@ -97,6 +97,8 @@ constexpr uint32_t TM_DKE = 448;   // dKe^T; before it, R^T and dO^T bf16 (packe
 constexpr uint32_t TM_DEB = TM_DKB;
 constexpr uint32_t TM_RB = TM_DKE;
 constexpr uint32_t TM_DOB = TM_DKE + 32;
+constexpr uint32_t TM_VB = TM_DQK;         // v and w bf16 (packed), steps 4 to 9
+constexpr uint32_t TM_WB = TM_DQK + 32;
 constexpr uint32_t TM_COLS = 512;
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
@@ -188,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     const uint32_t tmem = *tslot;
 
     int commits = 0;          // MMA commits issued on bar_mma (thread 0)
+    int raw_copies = 0;       // rounds of raw input copies issued on bar_raw
     bool raw_pending = false;
     // Bounded wait for a phase of an mbarrier: thread 0 polls, the block meets at a barrier.
     auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
@@ -207,28 +210,34 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             bulk_g2s(sbase + OFF_RK, K + tok0 * DK, row16, bar_raw);
             if (vec_b) bulk_g2s(sbase + OFF_RB, Bg + tok0 * DK, row16, bar_raw);
             if (vec_g) bulk_g2s(sbase + OFF_G, a.g + tok0 * DK, 2 * row16, bar_raw);
+            // the value-side rows read by every thread later on
+            prefetch_l2(V + tok0 * DV, row16);
+            if (vec_w) prefetch_l2(Wg + tok0 * DV, row16);
         }
+        ++raw_copies;
         raw_pending = true;
-        // S -> bf16 tile (warp w: rows 16 w .. 16 w + 15; lane: columns 4 lane .. + 3)
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-            float4 x[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                x[i] = *reinterpret_cast<const float4 *>(Sg + (size_t)(warp * 16 + h * 8 + i) * DV + 4 * lane);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                st_shared_v2(sbase + OFF_SB + tile_off(128, warp * 16 + h * 8 + i, 4 * lane),
-                             pack_bf16(x[i].x, x[i].y), pack_bf16(x[i].z, x[i].w));
-        }
+        // Per-thread global loads below read a clamped row (the chunk's last) for tokens past
+        // the end and discard the value: no load sits behind a branch, so each batch costs
+        // one memory latency.
+        // S -> bf16 tile (warp w: rows 16 w .. 16 w + 15; lane: columns 4 lane .. + 3), and
         // dO^T of this thread's value channel and tokens -> bf16 in TMEM (zero past the end)
         {
-            float x[32];
+            float4 x[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = (j0 + j < n) ? bf(dOg, (tok0 + j0 + j) * DV + r) : 0.f;
-            st_tmem_bf16(tmem + lane_base + TM_DOB + j0 / 2, x);
+            for (int i = 0; i < 16; ++i)
+                x[i] = *reinterpret_cast<const float4 *>(Sg + (size_t)(warp * 16 + i) * DV + 4 * lane);
+            float y[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = bf(dOg, (tok0 + min(j0 + j, n - 1)) * DV + r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                st_shared_v2(sbase + OFF_SB + tile_off(128, warp * 16 + i, 4 * lane), pack_bf16(x[i].x, x[i].y),
+                             pack_bf16(x[i].z, x[i].w));
+#pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = (j0 + j < n) ? y[j] : 0.f;
+            st_tmem_bf16(tmem + lane_base + TM_DOB + j0 / 2, y);
         }
-        if (!wait_bar(bar_raw, 0)) break;
+        if (!wait_bar(bar_raw, (uint32_t)((raw_copies - 1) & 1))) break;
         raw_pending = false;
         // ---- 2. cumulative log-decay: thread d < 128 scans key channel d and leaves e^gamma
         //      in place of g_log; any |gamma| > 60 sends the chunk to the exact path ----
@@ -291,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                 st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
             }
         }
-#pragma unroll 1
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
             float4 xs[8], xd[8];
 #pragma unroll
@@ -331,17 +340,21 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             mma_commit(bar_mma);
         }
         ++commits;
-        // W = w.v of this thread's value channel and tokens, while the MMAs run
+        // W = w.v of this thread's value channel and tokens, while the MMAs run; v and w
+        // themselves wait in TMEM (the [dKh | dQg] columns, first written in step 10) for step 9
         float wv[32];
+        {
+            float vt[32], wt[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int t = j0 + j;
-            float x = 0.f;
-            if (t < n) {
-                const size_t tk = tok0 + t;
-                x = bf(V, tk * DV + r) * (vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk));
+            for (int j = 0; j < 32; ++j) {
+                const size_t tk = tok0 + min(j0 + j, n - 1);
+                vt[j] = bf(V, tk * DV + r);
+                wt[j] = vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk);
             }
-            wv[j] = x;
+            st_tmem_bf16(tmem + lane_base + TM_VB + j0 / 2, vt);
+            st_tmem_bf16(tmem + lane_base + TM_WB + j0 / 2, wt);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) wv[j] = (j0 + j < n) ? vt[j] * wt[j] : 0.f;
         }
         if (!wait_mma()) break;
         tc_fence_after();
@@ -449,22 +462,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         ++commits;
         if (!wait_mma()) break;
         tc_fence_after();
-        // ---- 9. dv = dR w, dw = dR v; -dR^T -> the left half of the [-dR^T | dO^T] tile ----
+        // ---- 9. dv = dR w, dw = dR v, staged [t][v] over dS~ (free since step 8) for one
+        //      bulk store each; -dR^T -> the left half of the [-dR^T | dO^T] tile ----
         {
-            float x[32];
-            tmem_ld32(tmem + lane_base + TM_X + j0, x);
-            tmem_wait_ld();
+            float x[32], vt[32], wt[32];
+            {
+                float pv[16], pw[16];
+                tmem_ld16(tmem + lane_base + TM_VB + j0 / 2, pv);
+                tmem_ld16(tmem + lane_base + TM_WB + j0 / 2, pw);
+                tmem_ld32(tmem + lane_base + TM_X + j0, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint32_t u = __float_as_uint(pv[j]), w = __float_as_uint(pw[j]);
+                    vt[2 * j] = __uint_as_float(u << 16);
+                    vt[2 * j + 1] = __uint_as_float(u & 0xFFFF0000u);
+                    wt[2 * j] = __uint_as_float(w << 16);
+                    wt[2 * j + 1] = __uint_as_float(w & 0xFFFF0000u);
+                }
+            }
+            __nv_bfloat16 *sdv = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_DSB);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int t = j0 + j;
-                float gw = 0.f;
-                if (t < n) {
-                    const size_t tk = tok0 + t;
-                    const float wt = vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk);
-                    dVo[tk * DV + r] = __float2bfloat16_rn(x[j] * wt);
-                    gw = x[j] * bf(V, tk * DV + r);
-                    if (vec_w) dWo[tk * DV + r] = __float2bfloat16_rn(gw);
-                }
+                const float gw = t < n ? x[j] * vt[j] : 0.f;
+                sdv[t * DV + r] = __float2bfloat16_rn(x[j] * wt[j]);
+                if (vec_w) sdv[C * DV + t * DV + r] = __float2bfloat16_rn(gw);
                 if (!vec_w) {   // t is the same across the warp: fold over the value channels
                     const float s = warp_sum(gw);
                     if (lane == 0 && t < n) atomicAdd(&sFw[t], s);
@@ -481,8 +504,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        // ---- 10. [dA; dP] = [-dR; dO] E^T,  [dKh | dQg]^T = S [-dR; dO]^T ----
+        // ---- 10. [dA; dP] = [-dR; dO] E^T,  [dKh | dQg]^T = S [-dR; dO]^T; dv, dw out ----
         if (tid == 0) {
+            const uint32_t row16 = (uint32_t)n * DV * 2;
+            bulk_s2g(dVo + tok0 * DV, sbase + OFF_DSB, row16);
+            if (vec_w) bulk_s2g(dWo + tok0 * DV, sbase + OFF_DSB + C * DV * 2, row16);
+            bulk_commit();
             tc_fence_after();
             const uint32_t id_ap = idesc_bf16(128, 64, true, true, false);
             const uint32_t id_qk = idesc_bf16(128, 128, false, true, false);
@@ -498,6 +525,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         ++commits;
         if (!wait_mma()) break;
         tc_fence_after();
+        // raw q, k, b again for step 13 (the first copies were overwritten), into the tiles
+        // the last MMAs have released
+        if (tid == 0) {
+            const uint32_t row16 = (uint32_t)n * DK * 2;
+            fence_async_smem();
+            mbar_arrive_expect_tx(bar_raw, 2 * row16 + (vec_b ? row16 : 0));
+            bulk_g2s(sbase + OFF_RQ, Q + tok0 * DK, row16, bar_raw);
+            bulk_g2s(sbase + OFF_RK, K + tok0 * DK, row16, bar_raw);
+            if (vec_b) bulk_g2s(sbase + OFF_RB, Bg + tok0 * DK, row16, bar_raw);
+        }
+        ++raw_copies;
+        raw_pending = true;
         // ---- 11. dA and dP, both strictly lower, -> bf16 tile; dP's diagonal -> sDPd ----
         {
             float x[32];
@@ -538,9 +577,17 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         ++commits;
         if (!wait_mma()) break;
         tc_fence_after();
-        // ---- 13. per (token, key channel): thread r = d, tokens j0 .. j0 + 31 ----
+        if (!wait_bar(bar_raw, (uint32_t)((raw_copies - 1) & 1))) break;
+        raw_pending = false;
+        // ---- 13. per (token, key channel): thread r = d, tokens j0 .. j0 + 31; dq, dk, db
+        //      staged [t][d] over S and [Kh; Qg] (both free now), dg in place of dgamma ----
         {
             const int d = r;
+            const __nv_bfloat16 *rq = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_RQ);
+            const __nv_bfloat16 *rk = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_RK);
+            const __nv_bfloat16 *rb = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_RB);
+            __nv_bfloat16 *sdq = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_SB), *sdk = sdq + C * DK;
+            __nv_bfloat16 *sdb = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_QK);
             float ske = 0.f, sdg = 0.f;   // sum_t dKe Kb, sum_t dgamma over this thread's tokens
 #pragma unroll 1
             for (int g16 = 0; g16 < 2; ++g16) {
@@ -555,10 +602,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                 for (int i = 0; i < 16; ++i) {
                     const int t = tb + i;
                     const bool in = t < n;
-                    const size_t ix = (tok0 + t) * DK + d;
                     const float e = sG[t * DK + d], ei = rcp_approx(e);
-                    const float qv = in ? bf(Q, ix) : 0.f, kv = in ? bf(K, ix) : 0.f;
-                    const float bv = vec_b ? (in ? bf(Bg, ix) : 0.f) : sBeta[t];
+                    const float qv = in ? __bfloat162float(rq[t * DK + d]) : 0.f;
+                    const float kv = in ? __bfloat162float(rk[t * DK + d]) : 0.f;
+                    const float bv = vec_b ? (in ? __bfloat162float(rb[t * DK + d]) : 0.f) : sBeta[t];
                     const float dkbt = dkb[i] + dke[i], dpd = sDPd[t];
                     const float kbv = kv * ei;
                     const float gb = dkh[i] * kv * e;
@@ -566,11 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                     ske = fmaf(dke[i], kbv, ske);
                     sdg += dgam;
                     sG[t * DK + d] = dgam;   // dgamma replaces e^gamma
-                    if (in) {
-                        dQo[ix] = __float2bfloat16_rn(fmaf(dqg[i], e, dpd * kv));
-                        dKo[ix] = __float2bfloat16_rn(fmaf(dkh[i] * bv, e, fmaf(dkbt, ei, dpd * qv)));
-                        if (vec_b) dBo[ix] = __float2bfloat16_rn(gb);
-                    }
+                    sdq[t * DK + d] = __float2bfloat16_rn(fmaf(dqg[i], e, dpd * kv));
+                    sdk[t * DK + d] = __float2bfloat16_rn(fmaf(dkh[i] * bv, e, fmaf(dkbt, ei, dpd * qv)));
+                    if (vec_b) sdb[t * DK + d] = __float2bfloat16_rn(gb);
                     if (!vec_b) {   // fold over the key channels
                         const float s = warp_sum(gb);
                         if (lane == 0 && in) atomicAdd(&sFb[t], s);
@@ -587,15 +632,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                 const int t = j0 + i;
                 acc += sG[t * DK + d];
                 if (vec_g) {
-                    if (t < n) a.dg[(tok0 + t) * DK + d] = acc;
+                    sG[t * DK + d] = acc;
                 } else {
                     const float s = warp_sum(acc);
                     if (lane == 0 && t < n) atomicAdd(&sFg[t], s);
                 }
             }
         }
+        fence_async_smem();
         __syncthreads();
-        // ---- 14. scalar gates: one gradient per token ----
+        // ---- 14. the staged gradients out; scalar gates: one gradient per token ----
+        if (tid == 0) {
+            const uint32_t row16 = (uint32_t)n * DK * 2;
+            bulk_s2g(dQo + tok0 * DK, sbase + OFF_SB, row16);
+            bulk_s2g(dKo + tok0 * DK, sbase + OFF_SB + C * DK * 2, row16);
+            if (vec_b) bulk_s2g(dBo + tok0 * DK, sbase + OFF_QK, row16);
+            if (vec_g) bulk_s2g(a.dg + tok0 * DK, sbase + OFF_G, 2 * row16);
+            bulk_commit();
+        }
         if (tid < n) {
             const size_t tk = tok0 + tid;
             if (!vec_b) dBo[tk] = __float2bfloat16_rn(tied ? sFb[tid] + sFw[tid] : sFb[tid]);
@@ -606,11 +660,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
 
     tmem_wait_st();   // an early exit can leave this thread's dO^T store in flight
     tc_fence_before();
+    if (tid == 0) bulk_wait_all();   // the bulk stores have read their staging and landed
     __syncthreads();
     if (sFlag[1] && tid == 0) {
         // drain: the raw copies and every committed tensor-core operation
         atomicExch(&g_bwd_tc_error, 1);
-        if (raw_pending) mbar_wait(bar_raw, 0, kWaitLimit);
+        if (raw_pending) mbar_wait(bar_raw, (uint32_t)((raw_copies - 1) & 1), kWaitLimit);
         mma_commit(bar_mma);
         const int k = commits + 1;
         if (k >= 2) mbar_wait(bar_mma, (uint32_t)((k - 2) & 1), kWaitLimit);

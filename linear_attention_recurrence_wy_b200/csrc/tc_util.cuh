@@ -216,6 +216,13 @@ __device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src_sadd
         "r"(src_saddr), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+// shared -> global bulk copy (16-byte aligned addresses, size % 16 == 0); completion is
+// tracked by the issuing thread's bulk async-groups
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src_saddr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src_saddr),
+                 "r"(bytes)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until the committed bulk stores have read their shared-memory source
 __device__ __forceinline__ void bulk_wait_read_all() {
