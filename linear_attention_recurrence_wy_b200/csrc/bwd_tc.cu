@@ -114,6 +114,9 @@ __device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_
     asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
 }
 
+// One instantiation per mode (the gate shapes are compile-time: the kernel's code is run
+// once per chunk, so every branch left in it costs instruction fetch).
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     const int j0 = (warp >> 2) * 32;                    // and its 32 token columns
 
     // ---- this CTA's chunk ----
-    const int T = a.T, mode = a.mode;
+    const int T = a.T;
     const int nchunk = (T + C - 1) / C;
     const int bh = blockIdx.x / nchunk, c = blockIdx.x - bh * nchunk;
     const int t0 = c * C, n = min(C, T - t0);
@@ -143,9 +146,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     __nv_bfloat16 *dVo = (__nv_bfloat16 *)a.dv, *dBo = (__nv_bfloat16 *)a.db, *dWo = (__nv_bfloat16 *)a.dw;
     // gate shapes: per-channel erase b (GDN-2, b-only), per-channel write w (GDN-2, w-only),
     // per-channel decay (all but GDN); a scalar write gate is w itself (b-only) or beta in b
-    const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
-    const bool tied = mode == GDR_MODE_KDA || mode == GDR_MODE_GDN;
-    const __nv_bfloat16 *Wsc = mode == GDR_MODE_BONLY ? Wg : Bg;
+    constexpr bool vec_b = mode_b_vec(MODE), vec_w = mode_w_vec(MODE), vec_g = mode_g_vec(MODE);
+    constexpr bool tied = MODE == GDR_MODE_KDA || MODE == GDR_MODE_GDN;
+    const __nv_bfloat16 *Wsc = MODE == GDR_MODE_BONLY ? Wg : Bg;
 
     float *sG = reinterpret_cast<float *>(sm + OFF_G);
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                 st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
             }
         }
-#pragma unroll
+#pragma unroll 1
         for (int h = 0; h < 2; ++h) {
             float4 xs[8], xd[8];
 #pragma unroll
@@ -465,40 +468,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         // ---- 9. dv = dR w, dw = dR v, staged [t][v] over dS~ (free since step 8) for one
         //      bulk store each; -dR^T -> the left half of the [-dR^T | dO^T] tile ----
         {
-            float x[32], vt[32], wt[32];
-            {
-                float pv[16], pw[16];
-                tmem_ld16(tmem + lane_base + TM_VB + j0 / 2, pv);
-                tmem_ld16(tmem + lane_base + TM_WB + j0 / 2, pw);
-                tmem_ld32(tmem + lane_base + TM_X + j0, x);
+            __nv_bfloat16 *sdv = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_DSB);
+#pragma unroll 1
+            for (int g8 = 0; g8 < 4; ++g8) {
+                const int tb = j0 + 8 * g8;
+                float x[8], pv[4], pw[4];
+                tmem_ld8(tmem + lane_base + TM_X + tb, x);
+                tmem_ld4(tmem + lane_base + TM_VB + tb / 2, pv);
+                tmem_ld4(tmem + lane_base + TM_WB + tb / 2, pw);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const uint32_t u = __float_as_uint(pv[j]), w = __float_as_uint(pw[j]);
-                    vt[2 * j] = __uint_as_float(u << 16);
-                    vt[2 * j + 1] = __uint_as_float(u & 0xFFFF0000u);
-                    wt[2 * j] = __uint_as_float(w << 16);
-                    wt[2 * j + 1] = __uint_as_float(w & 0xFFFF0000u);
+                for (int j = 0; j < 8; ++j) {
+                    const int t = tb + j;
+                    const uint32_t u = __float_as_uint(pv[j / 2]), w = __float_as_uint(pw[j / 2]);
+                    const float vt = __uint_as_float((j & 1) ? (u & 0xFFFF0000u) : (u << 16));
+                    const float wt = __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
+                    const float gw = t < n ? x[j] * vt : 0.f;
+                    sdv[t * DV + r] = __float2bfloat16_rn(x[j] * wt);
+                    if (vec_w) sdv[C * DV + t * DV + r] = __float2bfloat16_rn(gw);
+                    if (!vec_w) {   // t is the same across the warp: fold over the value channels
+                        const float s = warp_sum(gw);
+                        if (lane == 0 && t < n) atomicAdd(&sFw[t], s);
+                    }
                 }
-            }
-            __nv_bfloat16 *sdv = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_DSB);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int t = j0 + j;
-                const float gw = t < n ? x[j] * vt[j] : 0.f;
-                sdv[t * DV + r] = __float2bfloat16_rn(x[j] * wt[j]);
-                if (vec_w) sdv[C * DV + t * DV + r] = __float2bfloat16_rn(gw);
-                if (!vec_w) {   // t is the same across the warp: fold over the value channels
-                    const float s = warp_sum(gw);
-                    if (lane == 0 && t < n) atomicAdd(&sFw[t], s);
-                }
-            }
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
                 float f[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = -x[h * 8 + j];
-                st_chunk(sbase + OFF_DOR + tile_chunk(128, r, j0 / 8 + h), f);
+                for (int j = 0; j < 8; ++j) f[j] = -x[j];
+                st_chunk(sbase + OFF_DOR + tile_chunk(128, r, tb / 8), f);
             }
         }
         fence_async_smem();
@@ -590,16 +586,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             __nv_bfloat16 *sdb = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_QK);
             float ske = 0.f, sdg = 0.f;   // sum_t dKe Kb, sum_t dgamma over this thread's tokens
 #pragma unroll 1
-            for (int g16 = 0; g16 < 2; ++g16) {
-                const int tb = j0 + 16 * g16;
-                float dkh[16], dqg[16], dkb[16], dke[16];
-                tmem_ld16(tmem + lane_base + TM_DQK + tb, dkh);
-                tmem_ld16(tmem + lane_base + TM_DQK + 64 + tb, dqg);
-                tmem_ld16(tmem + lane_base + TM_DKB + tb, dkb);
-                tmem_ld16(tmem + lane_base + TM_DKE + tb, dke);
+            for (int g8 = 0; g8 < 4; ++g8) {
+                const int tb = j0 + 8 * g8;
+                float dkh[8], dqg[8], dkb[8], dke[8];
+                tmem_ld8(tmem + lane_base + TM_DQK + tb, dkh);
+                tmem_ld8(tmem + lane_base + TM_DQK + 64 + tb, dqg);
+                tmem_ld8(tmem + lane_base + TM_DKB + tb, dkb);
+                tmem_ld8(tmem + lane_base + TM_DKE + tb, dke);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     const int t = tb + i;
                     const bool in = t < n;
                     const float e = sG[t * DK + d], ei = rcp_approx(e);
@@ -653,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         if (tid < n) {
             const size_t tk = tok0 + tid;
             if (!vec_b) dBo[tk] = __float2bfloat16_rn(tied ? sFb[tid] + sFw[tid] : sFb[tid]);
-            if (mode == GDR_MODE_BONLY) dWo[tk] = __float2bfloat16_rn(sFw[tid]);
+            if (MODE == GDR_MODE_BONLY) dWo[tk] = __float2bfloat16_rn(sFw[tid]);
             if (!vec_g) a.dg[tk] = sFg[tid];
         }
     } while (0);
@@ -682,10 +678,15 @@ bool bwd_tc_supported(const BwdArgs &a) { return a.dtype == GDR_BF16 && a.dk_ ==
 
 gdr_status_t launch_bwd_tc(const BwdArgs &a, cudaStream_t s) {
     static_assert(2 * kBwdChunk == C, "a chunk here is two of the backward's 32-token chunks");
-    if (cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+    auto kern = a.mode == GDR_MODE_GDN2  ? bwd_tc_kernel<GDR_MODE_GDN2>
+              : a.mode == GDR_MODE_KDA   ? bwd_tc_kernel<GDR_MODE_KDA>
+              : a.mode == GDR_MODE_GDN   ? bwd_tc_kernel<GDR_MODE_GDN>
+              : a.mode == GDR_MODE_BONLY ? bwd_tc_kernel<GDR_MODE_BONLY>
+                                         : bwd_tc_kernel<GDR_MODE_WONLY>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     const unsigned grid = (unsigned)((size_t)a.B * a.H * ((a.T + C - 1) / C));
-    bwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(a);
+    kern<<<grid, kThreads, SMEM_BYTES, s>>>(a);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

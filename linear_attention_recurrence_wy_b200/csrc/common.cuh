@@ -54,12 +54,12 @@ struct DecodeArgs {
 
 // Gate shapes per mode: the erase gate b and the write gate w are per channel or one
 // scalar per token; the scalar write gate is w itself (b-only) or beta in b (tied modes).
-__host__ __device__ inline bool mode_b_vec(int m) { return m == GDR_MODE_GDN2 || m == GDR_MODE_BONLY; }
-__host__ __device__ inline bool mode_w_vec(int m) { return m == GDR_MODE_GDN2 || m == GDR_MODE_WONLY; }
-__host__ __device__ inline bool mode_uses_w(int m) {
+__host__ __device__ constexpr bool mode_b_vec(int m) { return m == GDR_MODE_GDN2 || m == GDR_MODE_BONLY; }
+__host__ __device__ constexpr bool mode_w_vec(int m) { return m == GDR_MODE_GDN2 || m == GDR_MODE_WONLY; }
+__host__ __device__ constexpr bool mode_uses_w(int m) {
     return m == GDR_MODE_GDN2 || m == GDR_MODE_BONLY || m == GDR_MODE_WONLY;
 }
-__host__ __device__ inline bool mode_g_vec(int m) { return m != GDR_MODE_GDN; }
+__host__ __device__ constexpr bool mode_g_vec(int m) { return m != GDR_MODE_GDN; }
 
 __device__ __forceinline__ float ld_elem(const void *p, size_t i, int dtype) {
     if (dtype == GDR_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i]);
