@@ -73,7 +73,7 @@ constexpr int OFF_DAP = OFF_P;            // [dA; dP] bf16 [128][64 j] (over P a
 // small arrays
 constexpr int OFF_GC = OFF_T + 8192;      // gamma_C fp32 [128]
 constexpr int OFF_EGC = OFF_GC + 512;     // exp(gamma_C) [128]
-constexpr int OFF_DGC = OFF_EGC + 512;    // sum_v S dS~ per key channel [128]
+constexpr int OFF_DGC = OFF_EGC + 512;    // sum_v S dS' per key channel [128]
 constexpr int OFF_CAR = OFF_DGC + 512;    // the epilogue's exchange between token halves [3][128]
 constexpr int OFF_BETA = OFF_CAR + 1536;  // scalar erase gate of the chunk's tokens [64]
 constexpr int OFF_GS = OFF_BETA + 256;    // scalar g_log (GDN) [64]
@@ -222,23 +222,44 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         // Per-thread global loads below read a clamped row (the chunk's last) for tokens past
         // the end and discard the value: no load sits behind a branch, so each batch costs
         // one memory latency.
-        // S -> bf16 tile (warp w: rows 16 w .. 16 w + 15; lane: columns 4 lane .. + 3), and
-        // dO^T of this thread's value channel and tokens -> bf16 in TMEM (zero past the end)
+        // S -> bf16 tile and sum_v S dS' per key channel (warp w: rows 16 w .. 16 w + 15;
+        // lane: columns 4 lane .. + 3); dS' stays in registers until gamma_C is known.  dO^T,
+        // v and w of this thread's value channel and tokens -> bf16 in TMEM (v and w in the
+        // [dKh | dQg] columns, first written in step 10)
+        float4 dsr[16];
         {
             float4 x[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                x[i] = *reinterpret_cast<const float4 *>(Sg + (size_t)(warp * 16 + i) * DV + 4 * lane);
+            for (int i = 0; i < 16; ++i) {
+                const size_t o = (size_t)(warp * 16 + i) * DV + 4 * lane;
+                x[i] = *reinterpret_cast<const float4 *>(Sg + o);
+                dsr[i] = *reinterpret_cast<const float4 *>(dSg + o);
+            }
             float y[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) y[j] = bf(dOg, (tok0 + min(j0 + j, n - 1)) * DV + r);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
+            for (int i = 0; i < 16; ++i) {
                 st_shared_v2(sbase + OFF_SB + tile_off(128, warp * 16 + i, 4 * lane), pack_bf16(x[i].x, x[i].y),
                              pack_bf16(x[i].z, x[i].w));
+                const float sd = warp_sum(x[i].x * dsr[i].x + x[i].y * dsr[i].y + x[i].z * dsr[i].z +
+                                          x[i].w * dsr[i].w);
+                if (lane == 0) sDGC[warp * 16 + i] = sd;
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) y[j] = (j0 + j < n) ? y[j] : 0.f;
             st_tmem_bf16(tmem + lane_base + TM_DOB + j0 / 2, y);
+        }
+        {
+            float vt[32], wt[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const size_t tk = tok0 + min(j0 + j, n - 1);
+                vt[j] = bf(V, tk * DV + r);
+                wt[j] = vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk);
+            }
+            st_tmem_bf16(tmem + lane_base + TM_VB + j0 / 2, vt);
+            st_tmem_bf16(tmem + lane_base + TM_WB + j0 / 2, wt);
         }
         if (!wait_bar(bar_raw, (uint32_t)((raw_copies - 1) & 1))) break;
         raw_pending = false;
@@ -271,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             break;
         }
         // ---- 3. operands: Kh, Qg, Kb (thread (tg, cg): tokens 4 tg .. + 3, channels
-        //      8 cg .. + 7), and dS~ with sum_v S dS~ per key channel ----
+        //      8 cg .. + 7), and dS~ = diag(e^gamma_C) dS' ----
         {
             const int tg = tid >> 4, cg = tid & 15;
 #pragma unroll 1
@@ -303,24 +324,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                 st_chunk(sbase + OFF_KB + tile_chunk(64, t, cg), kb);
             }
         }
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-            float4 xs[8], xd[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const size_t o = (size_t)(warp * 16 + h * 8 + i) * DV + 4 * lane;
-                xs[i] = *reinterpret_cast<const float4 *>(Sg + o);
-                xd[i] = *reinterpret_cast<const float4 *>(dSg + o);
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int d = warp * 16 + h * 8 + i;
-                const float eg = sEGC[d];
-                const float y0 = xd[i].x * eg, y1 = xd[i].y * eg, y2 = xd[i].z * eg, y3 = xd[i].w * eg;
-                st_shared_v2(sbase + OFF_DSB + tile_off(128, d, 4 * lane), pack_bf16(y0, y1), pack_bf16(y2, y3));
-                const float s = warp_sum(xs[i].x * y0 + xs[i].y * y1 + xs[i].z * y2 + xs[i].w * y3);
-                if (lane == 0) sDGC[d] = s;
-            }
+        for (int i = 0; i < 16; ++i) {
+            const int d = warp * 16 + i;
+            const float eg = sEGC[d];
+            st_shared_v2(sbase + OFF_DSB + tile_off(128, d, 4 * lane), pack_bf16(dsr[i].x * eg, dsr[i].y * eg),
+                         pack_bf16(dsr[i].z * eg, dsr[i].w * eg));
         }
         fence_async_smem();
         tmem_wait_st();
@@ -343,22 +352,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             mma_commit(bar_mma);
         }
         ++commits;
-        // W = w.v of this thread's value channel and tokens, while the MMAs run; v and w
-        // themselves wait in TMEM (the [dKh | dQg] columns, first written in step 10) for step 9
-        float wv[32];
-        {
-            float vt[32], wt[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const size_t tk = tok0 + min(j0 + j, n - 1);
-                vt[j] = bf(V, tk * DV + r);
-                wt[j] = vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk);
-            }
-            st_tmem_bf16(tmem + lane_base + TM_VB + j0 / 2, vt);
-            st_tmem_bf16(tmem + lane_base + TM_WB + j0 / 2, wt);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) wv[j] = (j0 + j < n) ? vt[j] * wt[j] : 0.f;
-        }
         if (!wait_mma()) break;
         tc_fence_after();
         // ---- 5. A (fp32, strictly lower) -> inverse scratch; P (lower incl.) -> bf16 tile;
@@ -386,10 +379,18 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                     st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
                 }
             }
+            float pv[16], pw[16];
+            tmem_ld16(tmem + lane_base + TM_VB + j0 / 2, pv);
+            tmem_ld16(tmem + lane_base + TM_WB + j0 / 2, pw);
             tmem_ld32(tmem + lane_base + TM_X + j0, x);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[j] = wv[j] - x[j];
+            for (int j = 0; j < 32; ++j) {   // W = w.v (zero past the end) from the packed pairs
+                const uint32_t u = __float_as_uint(pv[j / 2]), w = __float_as_uint(pw[j / 2]);
+                const float vt = __uint_as_float((j & 1) ? (u & 0xFFFF0000u) : (u << 16));
+                const float wt = __uint_as_float((j & 1) ? (w & 0xFFFF0000u) : (w << 16));
+                x[j] = (j0 + j < n ? vt * wt : 0.f) - x[j];
+            }
             st_tmem_bf16(tmem + lane_base + TM_RB + j0 / 2, x);
         }
         fence_async_smem();
@@ -622,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             if (j0) sCar[d] = sdg;
             sCar[128 * (1 + (j0 >> 5)) + d] = ske;
             __syncthreads();
-            float acc = sDGC[d] + sCar[128 + d] + sCar[256 + d] + (j0 ? 0.f : sCar[d]);
+            float acc = sEGC[d] * sDGC[d] + sCar[128 + d] + sCar[256 + d] + (j0 ? 0.f : sCar[d]);
 #pragma unroll 4
             for (int i = 31; i >= 0; --i) {
                 const int t = j0 + i;
