@@ -70,6 +70,9 @@ constexpr int OFF_X = OFF_A32 + 64 * tri::LD * 4;   // the inverse's scratch, 4 
 constexpr int OFF_DOR = OFF_RQ;           // [-dR^T | dO^T] bf16 [128 v][128] (after the inverse)
 constexpr int OFF_ET = OFF_RB;            // E^T bf16 [128 v][64 t]                      16 KB
 constexpr int OFF_DAP = OFF_P;            // [dA; dP] bf16 [128][64 j] (over P and T)    16 KB
+constexpr int OFF_RDO = OFF_QK;           // raw dO, v, w bf16 [64][128] each (until the build)
+constexpr int OFF_RV = OFF_QK + 16384;
+constexpr int OFF_RW = OFF_KB;
 // small arrays
 constexpr int OFF_GC = OFF_T + 8192;      // gamma_C fp32 [128]
 constexpr int OFF_EGC = OFF_GC + 512;     // exp(gamma_C) [128]
@@ -204,28 +207,25 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     auto wait_mma = [&]() -> bool { return wait_bar(bar_mma, (uint32_t)((commits - 1) & 1)); };
 
     do {
-        // ---- 1. raw q, k, b, g_log of the chunk: one bulk copy per tensor ----
+        // ---- 1. raw q, k, b, g_log, dO, v, w of the chunk: one bulk copy per tensor (dO, v
+        //      and w into the operand tiles, which the build fills only after they are read) ----
         if (tid == 0) {
             const uint32_t row16 = (uint32_t)n * DK * 2;
             fence_async_smem();
-            mbar_arrive_expect_tx(bar_raw, 2 * row16 + (vec_b ? row16 : 0) + (vec_g ? 2 * row16 : 0));
+            mbar_arrive_expect_tx(bar_raw, (4 + (vec_b ? 1 : 0) + (vec_g ? 2 : 0) + (vec_w ? 1 : 0)) * row16);
             bulk_g2s(sbase + OFF_RQ, Q + tok0 * DK, row16, bar_raw);
             bulk_g2s(sbase + OFF_RK, K + tok0 * DK, row16, bar_raw);
             if (vec_b) bulk_g2s(sbase + OFF_RB, Bg + tok0 * DK, row16, bar_raw);
             if (vec_g) bulk_g2s(sbase + OFF_G, a.g + tok0 * DK, 2 * row16, bar_raw);
-            // the value-side rows read by every thread later on
-            prefetch_l2(V + tok0 * DV, row16);
-            if (vec_w) prefetch_l2(Wg + tok0 * DV, row16);
+            bulk_g2s(sbase + OFF_RDO, dOg + tok0 * DV, row16, bar_raw);
+            bulk_g2s(sbase + OFF_RV, V + tok0 * DV, row16, bar_raw);
+            if (vec_w) bulk_g2s(sbase + OFF_RW, Wg + tok0 * DV, row16, bar_raw);
         }
         ++raw_copies;
         raw_pending = true;
-        // Per-thread global loads below read a clamped row (the chunk's last) for tokens past
-        // the end and discard the value: no load sits behind a branch, so each batch costs
-        // one memory latency.
         // S -> bf16 tile and sum_v S dS' per key channel (warp w: rows 16 w .. 16 w + 15;
-        // lane: columns 4 lane .. + 3); dS' stays in registers until gamma_C is known.  dO^T,
-        // v and w of this thread's value channel and tokens -> bf16 in TMEM (v and w in the
-        // [dKh | dQg] columns, first written in step 10)
+        // lane: columns 4 lane .. + 3); dS' stays in registers until gamma_C is known.  The
+        // loads are batched: no load sits behind a branch, so the batch costs one latency.
         float4 dsr[16];
         {
             float4 x[16];
@@ -235,9 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                 x[i] = *reinterpret_cast<const float4 *>(Sg + o);
                 dsr[i] = *reinterpret_cast<const float4 *>(dSg + o);
             }
-            float y[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = bf(dOg, (tok0 + min(j0 + j, n - 1)) * DV + r);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 st_shared_v2(sbase + OFF_SB + tile_off(128, warp * 16 + i, 4 * lane), pack_bf16(x[i].x, x[i].y),
@@ -246,23 +243,31 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
                                           x[i].w * dsr[i].w);
                 if (lane == 0) sDGC[warp * 16 + i] = sd;
             }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) y[j] = (j0 + j < n) ? y[j] : 0.f;
-            st_tmem_bf16(tmem + lane_base + TM_DOB + j0 / 2, y);
         }
-        {
-            float vt[32], wt[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const size_t tk = tok0 + min(j0 + j, n - 1);
-                vt[j] = bf(V, tk * DV + r);
-                wt[j] = vec_w ? bf(Wg, tk * DV + r) : bf(Wsc, tk);
-            }
-            st_tmem_bf16(tmem + lane_base + TM_VB + j0 / 2, vt);
-            st_tmem_bf16(tmem + lane_base + TM_WB + j0 / 2, wt);
-        }
+        // the scalar write gate of the chunk's tokens, if there is one (zero past the end)
+        float wsc = 0.f;
+        if (!vec_w) wsc = bf(Wsc, tok0 + min(j0 + (lane & 31), n - 1));
         if (!wait_bar(bar_raw, (uint32_t)((raw_copies - 1) & 1))) break;
         raw_pending = false;
+        // dO^T, v and w of this thread's value channel and tokens -> bf16 in TMEM (v and w in
+        // the [dKh | dQg] columns, first written in step 10); rows past the end are zero
+        {
+            const __nv_bfloat16 *rdo = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_RDO);
+            const __nv_bfloat16 *rv = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_RV);
+            const __nv_bfloat16 *rw = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_RW);
+            float x[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = (j0 + j < n) ? __bfloat162float(rdo[(j0 + j) * DV + r]) : 0.f;
+            st_tmem_bf16(tmem + lane_base + TM_DOB + j0 / 2, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[j] = (j0 + j < n) ? __bfloat162float(rv[(j0 + j) * DV + r]) : 0.f;
+            st_tmem_bf16(tmem + lane_base + TM_VB + j0 / 2, x);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                x[j] = vec_w ? ((j0 + j < n) ? __bfloat162float(rw[(j0 + j) * DV + r]) : 0.f)
+                             : __shfl_sync(0xffffffffu, wsc, j);
+            st_tmem_bf16(tmem + lane_base + TM_WB + j0 / 2, x);
+        }
         // ---- 2. cumulative log-decay: thread d < 128 scans key channel d and leaves e^gamma
         //      in place of g_log; any |gamma| > 60 sends the chunk to the exact path ----
         if (tid < DK) {

@@ -146,8 +146,9 @@ def test_t4k_workload_sampled_heads(cuda_ok):
         check_grad(f"t4k {n}", got, ref[n][:, 0], "bf16")
 
 
-# ---- the tensor-core shape (bf16, dk = dv = 128): checkpoints and the state gradient run on
-#      tcgen05 (the forward kernel and its reverse-order instantiation) -------------------------
+# ---- the tensor-core shape (bf16, dk = dv = 128): checkpoints, the state gradient and the
+#      per-chunk gradients run on tcgen05; 64-token chunks whose cumulative decay passes e^-60
+#      are listed for the CUDA-core per-chunk kernel ------------------------------------------
 @pytest.mark.parametrize("mode", ["gdn2", "kda", "gdn", "bonly", "wonly"])
 @pytest.mark.parametrize("T", [20, 64, 96, 150])
 def test_tensor_core_state_gradient(cuda_ok, mode, T):
@@ -170,3 +171,32 @@ def test_tensor_core_state_gradient_strong_decay(cuda_ok, g_const):
 def test_tensor_core_state_gradient_without_state_gradient_input(cuda_ok):
     d, dO, dST = make_case(2, 2, 130, 128, 128, "gdn2", "bf16", seed=43, s0=0.0, dst=False)
     run_case(d, dO, dST, "bf16")
+
+
+def test_tensor_core_backward_mixed_fast_and_exact_chunks(cuda_ok):
+    # strong decay in the first two 64-token chunks (CUDA-core kernel, exact pair decays), mild
+    # decay in the last two (tensor-core kernel), in one call
+    d, dO, dST = make_case(1, 2, 256, 128, 128, "gdn2", "bf16", seed=47, s0=0.05, g_scale=0.1)
+    d["g"][:, :, :128] = -2.0
+    run_case(d, dO, dST, "bf16")
+
+
+def test_tensor_core_backward_many_listed_chunks(cuda_ok):
+    # every chunk past the factorisation limit: 16 heads x 41 chunks = 656 listed spans, more
+    # than the CUDA-core kernel's grid (4 x 148 CTAs), so its CTAs walk the list; two heads
+    # are checked against the oracle
+    B, H, T = 1, 16, 2600
+    d, dO, dST = make_case(B, H, T, 128, 128, "kda", "bf16", seed=53, s0=0.05)
+    d["g"] = torch.full_like(d["g"], -2.0)
+    dd = to_dev(d)
+    out = gdr.chunk_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["b"], dd["w"], dd["S0"], dO.cuda(), dST.cuda(),
+                        mode="kda")
+    torch.cuda.synchronize()
+    assert gdr.gdr_last_device_error(torch.cuda.current_stream().cuda_stream) == 0
+    heads = [0, 15]
+    pick = lambda x: None if x is None else x[:, heads]
+    ref = oracle.bwd(*(pick(d[n]) for n in ("q", "k", "v", "g", "b", "w", "S0")), pick(dO), pick(dST), mode="kda")
+    for n in NAMES:
+        if ref[n] is None:
+            continue
+        check_grad(f"listed {n}", np64(out[n][:, heads]), ref[n], "bf16")
