@@ -50,6 +50,11 @@ __device__ __forceinline__ float ld_w(const BwdArgs &a, size_t tk, int j) {   //
     if (mode_w_vec(a.mode)) return ld_elem(a.w, tk * a.dv_ + j, a.dtype);
     return ld_elem(a.mode == GDR_MODE_BONLY ? a.w : a.b, tk, a.dtype);
 }
+// element idx of a state slot: fp32, or bf16 [dk][dv] at the slot's start (the tensor-core
+// passes' checkpoints and span-end state gradients)
+__device__ __forceinline__ float ld_state(const float *slot, size_t idx, bool bf) {
+    return bf ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(slot)[idx]) : slot[idx];
+}
 __device__ __forceinline__ float ld_g(const BwdArgs &a, size_t tk, int c) {
     return a.mode == GDR_MODE_GDN ? a.g[tk] : a.g[tk * a.dk_ + c];
 }
@@ -289,7 +294,8 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
             const int t = idx / dv, j = idx - t * dv;
             X1[idx] = t < n1 ? ld_elem(a.dO, (tk1 + t) * dv + j, a.dtype) : 0.f;
         }
-        for (int idx = tid; idx < dk * dv; idx += nth) Ss[(idx / dv) * SLD + idx % dv] = dSe[idx];
+        for (int idx = tid; idx < dk * dv; idx += nth)
+            Ss[(idx / dv) * SLD + idx % dv] = ld_state(dSe, idx, a.ckpt_bf16);
         chunk_core(a, tk1, n1, qq, kk, bb, gm, gC, Am, Tm, Pm);
         for (int idx = tid; idx < C * dk; idx += nth) {   // Ke, Qg, Kh
             const int d = idx % dk;
@@ -370,6 +376,10 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     float *fg = fw + C;              // [C]: folded scalar decay gradient
     float *Sg = a.ws_states + ((size_t)bh * nc + c_idx) * dk * dv;
     const float *dSg = a.ws_dstates + ((size_t)bh * nc + c_idx) * dk * dv;
+    // slots the tensor-core passes wrote (bf16): the span's start state, and the state
+    // gradient at the span's end (slot 2 span + 1, or 2 span for a one-chunk last span)
+    const bool s_bf = a.ckpt_bf16 && hf == 0;
+    const bool ds_bf = a.ckpt_bf16 && (hf == 1 || c_idx + 1 >= nc);
 
     float aq[RPG], ak[RPG], ab[RPG], ag[RPG];
 #pragma unroll
@@ -388,7 +398,7 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     }
     for (int idx = tid; idx < dk * dv; idx += nth) {
         const int d = idx / dv, j = idx - d * dv;
-        Ss[d * SLD + j] = Sg[idx];
+        Ss[d * SLD + j] = ld_state(Sg, idx, s_bf);
     }
     for (int i = tid; i < C; i += nth) fb[i] = fw[i] = fg[i] = 0.f;
     for (int d = tid; d < dk; d += nth) dgC[d] = 0.f;
@@ -478,11 +488,12 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     }
     for (int idx = tid; idx < dk * dv; idx += nth) {
         const int d = idx / dv, j = idx - d * dv;
-        Ss[d * SLD + j] = dSg[idx];
+        Ss[d * SLD + j] = ld_state(dSg, idx, ds_bf);
     }
     if (tid < dk) {
         float acc = 0.f;
-        for (int j = 0; j < dv; ++j) acc = fmaf(Sg[(size_t)tid * dv + j], dSg[(size_t)tid * dv + j], acc);
+        for (int j = 0; j < dv; ++j)
+            acc = fmaf(ld_state(Sg, (size_t)tid * dv + j, s_bf), ld_state(dSg, (size_t)tid * dv + j, ds_bf), acc);
         dgC[tid] = __expf(gC[tid]) * acc;
     }
     __syncthreads();
@@ -576,7 +587,7 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     }
     for (int idx = tid; idx < dk * dv; idx += nth) {
         const int d = idx / dv, j = idx - d * dv;
-        Ss[d * SLD + j] = Sg[idx];
+        Ss[d * SLD + j] = ld_state(Sg, idx, s_bf);
     }
     __syncthreads();
     // ---- DX = dR S^T (through Kh = b k e^gamma, with a minus sign: R = w.v - Kh S) ----
@@ -703,6 +714,7 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
         r.dO = a.dO;
         if ((st = launch_chunk_tc(r, s)) != GDR_OK) return st;
         b.mid_grad = 1;
+        b.ckpt_bf16 = 1;
         // 3. per-chunk gradients on the tensor cores; spans with a strong cumulative decay
         //    are listed for the CUDA-core kernel below
         b.tc_list = reinterpret_cast<int *>(reinterpret_cast<unsigned char *>(a.ws_states) +

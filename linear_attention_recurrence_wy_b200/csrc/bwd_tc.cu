@@ -113,10 +113,6 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-__device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_t b) {
-    asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
-}
-
 // One instantiation per mode (the gate shapes are compile-time: the kernel's code is run
 // once per chunk, so every branch left in it costs instruction fetch).
 template <int MODE>
@@ -136,8 +132,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     const int bh = blockIdx.x / nchunk, c = blockIdx.x - bh * nchunk;
     const int t0 = c * C, n = min(C, T - t0);
     const size_t tok0 = (size_t)bh * T + t0;            // row of the chunk's first token
-    // the workspace holds one fp32 state per 32-token chunk: S at this chunk's start is in
-    // the slot of its first 32-token chunk, dS' at its end in the slot of its last one
+    // the workspace has one fp32-sized state slot per 32-token chunk: S at this chunk's start
+    // is in the slot of its first 32-token chunk, dS' at its end in the slot of its last one,
+    // both as bf16 [dk][dv] (the tensor-core passes write them so)
     const int nslot = (T + kBwdChunk - 1) / kBwdChunk;
     const float *Sg = a.ws_states + ((size_t)bh * nslot + 2 * c) * DK * DV;
     const float *dSg = a.ws_dstates + ((size_t)bh * nslot + min(2 * c + 1, nslot - 1)) * DK * DV;
@@ -223,25 +220,34 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         }
         ++raw_copies;
         raw_pending = true;
-        // S -> bf16 tile and sum_v S dS' per key channel (warp w: rows 16 w .. 16 w + 15;
-        // lane: columns 4 lane .. + 3); dS' stays in registers until gamma_C is known.  The
-        // loads are batched: no load sits behind a branch, so the batch costs one latency.
-        float4 dsr[16];
+        // S -> bf16 tile and sum_v S dS' per key channel (both stored as bf16 [dk][dv]; warp w:
+        // rows 16 w .. 16 w + 15, two per load, 16 lanes of eight channels each); dS' stays in
+        // registers until gamma_C is known.  The loads are batched: no load sits behind a
+        // branch, so the batch costs one latency.
+        uint4 dsr[8];
         {
-            float4 x[16];
+            const __nv_bfloat16 *Sb = reinterpret_cast<const __nv_bfloat16 *>(Sg);
+            const __nv_bfloat16 *dSb = reinterpret_cast<const __nv_bfloat16 *>(dSg);
+            uint4 x[8];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const size_t o = (size_t)(warp * 16 + i) * DV + 4 * lane;
-                x[i] = *reinterpret_cast<const float4 *>(Sg + o);
-                dsr[i] = *reinterpret_cast<const float4 *>(dSg + o);
+            for (int i = 0; i < 8; ++i) {
+                const size_t o = (size_t)(warp * 16 + 2 * i + (lane >> 4)) * DV + 8 * (lane & 15);
+                x[i] = *reinterpret_cast<const uint4 *>(Sb + o);
+                dsr[i] = *reinterpret_cast<const uint4 *>(dSb + o);
             }
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                st_shared_v2(sbase + OFF_SB + tile_off(128, warp * 16 + i, 4 * lane), pack_bf16(x[i].x, x[i].y),
-                             pack_bf16(x[i].z, x[i].w));
-                const float sd = warp_sum(x[i].x * dsr[i].x + x[i].y * dsr[i].y + x[i].z * dsr[i].z +
-                                          x[i].w * dsr[i].w);
-                if (lane == 0) sDGC[warp * 16 + i] = sd;
+            for (int i = 0; i < 8; ++i) {
+                const int d = warp * 16 + 2 * i + (lane >> 4);
+                st_shared_v4(sbase + OFF_SB + tile_chunk(128, d, lane & 15), x[i].x, x[i].y, x[i].z, x[i].w);
+                float fs[8], fd[8];
+                bf16x8_to_f32(x[i], fs);
+                bf16x8_to_f32(dsr[i], fd);
+                float sd = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sd = fmaf(fs[j], fd[j], sd);
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) sd += __shfl_xor_sync(0xffffffffu, sd, o);   // 16 lanes of row d
+                if ((lane & 15) == 0) sDGC[d] = sd;
             }
         }
         // the scalar write gate of the chunk's tokens, if there is one (zero past the end)
@@ -330,11 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             }
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int d = warp * 16 + i;
+        for (int i = 0; i < 8; ++i) {
+            const int d = warp * 16 + 2 * i + (lane >> 4);
             const float eg = sEGC[d];
-            st_shared_v2(sbase + OFF_DSB + tile_off(128, d, 4 * lane), pack_bf16(dsr[i].x * eg, dsr[i].y * eg),
-                         pack_bf16(dsr[i].z * eg, dsr[i].w * eg));
+            float f[8];
+            bf16x8_to_f32(dsr[i], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] *= eg;
+            st_chunk(sbase + OFF_DSB + tile_chunk(128, d, lane & 15), f);
         }
         fence_async_smem();
         tmem_wait_st();

@@ -267,8 +267,8 @@ struct TokenMaps {
 
 // kMixer: the token-mixer instantiation (activations on load, output epilogue, either
 // layout; ChunkArgs::mixer).  kStates: the backward's checkpoint pass, which also writes
-// the fp32 state at the start of every chunk to ChunkArgs::chunk_states (slot 2c of the
-// backward's 32-token chunk slots).  kReverse: the backward's state-gradient pass
+// the state at the start of every chunk, rounded to bf16, to ChunkArgs::chunk_states (slot
+// 2c of the backward's 32-token chunk slots).  kReverse: the backward's state-gradient pass
 // (ChunkArgs::reverse), chunks in reverse order; see the state group.  The plain
 // instantiation is the recurrence alone.
 template <bool kMixer, bool kStates, bool kReverse>
@@ -725,15 +725,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             const float *egc = sEGC + (c & 3) * 128;
             if (kStates) {
                 // checkpoint: S_c (S^T columns [64 half, +64) of this lane), before this
-                // chunk's update; coalesced over the value channels (lanes)
-                float *dst = a.chunk_states + ((size_t)bh * ((a.T + 31) / 32) + 2 * c) * DK * DV + v;
+                // chunk's update, as bf16 [dk][dv] at the start of the slot; coalesced over
+                // the value channels (lanes)
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(
+                                         a.chunk_states + ((size_t)bh * ((a.T + 31) / 32) + 2 * c) * DK * DV) + v;
 #pragma unroll 1
                 for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
                     float x[32];
                     tmem_ld32(tmem + lane_base + TM_S + d0, x);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[(size_t)(d0 + j) * DV] = x[j];
+                    for (int j = 0; j < 32; ++j) dst[(size_t)(d0 + j) * DV] = __float2bfloat16_rn(x[j]);
                 }
             }
             // (w.v)^T for this thread's lane and token columns, read from global memory
@@ -968,14 +970,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             const float *egc = sEGC + (c & 3) * 128;
             {
                 const int nslot = (T + 31) / 32;
-                float *dst = a.chunk_states + ((size_t)bh * nslot + min(2 * cd + 1, nslot - 1)) * DK * DV + v;
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(
+                                         a.chunk_states + ((size_t)bh * nslot + min(2 * cd + 1, nslot - 1)) * DK * DV) + v;
 #pragma unroll 1
                 for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
                     float x[32];
                     tmem_ld32(tmem + lane_base + TM_S + d0, x);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) dst[(size_t)(d0 + j) * DV] = x[j];
+                    for (int j = 0; j < 32; ++j) dst[(size_t)(d0 + j) * DV] = __float2bfloat16_rn(x[j]);
                 }
             }
             {   // dO^T of this lane and token columns -> bf16 in TMEM; tokens past the end give zero

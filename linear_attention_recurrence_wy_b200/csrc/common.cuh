@@ -34,12 +34,14 @@ struct ChunkArgs {
     const float *nw;
     float b_range, eps;
     // The backward's checkpoints: when set, the state at the start of every chunk is written
-    // to chunk_states[B*H][ceil(T/32)][dk][dv] (fp32), in the slot of the chunk's first
-    // 32-token chunk (a 64-token chunk c fills slot 2c), and o may be NULL.
+    // to chunk_states[B*H][ceil(T/32)][dk][dv] (fp32 slots), in the slot of the chunk's
+    // first 32-token chunk (a 64-token chunk c fills slot 2c), and o may be NULL.  The
+    // CUDA-core kernel writes fp32; the tensor-core kernel writes the state rounded to bf16
+    // ([dk][dv] bf16 at the start of the slot), its MMA operands' precision.
     float *chunk_states;
     // The backward's state-gradient pass (tensor-core kernel, reverse != 0): S0 holds dS_T,
     // ST receives dS0, dO is the output gradient [B,H,T,dv], and chunk_states receives the
-    // gradient at every 64-token chunk's end (slot of its last 32-token chunk).
+    // gradient at every 64-token chunk's end (slot of its last 32-token chunk), as bf16.
     int reverse;
     const void *dO;
 };
@@ -95,6 +97,10 @@ struct BwdArgs {
     // the tensor-core per-chunk kernel left to the CUDA-core one; NULL: that kernel takes
     // every span
     int *tc_list;
+    // 1: the tensor-core passes wrote the checkpoints (ws_states slot 2 span) and the span-end
+    // state gradients (ws_dstates slot min(2 span + 1, last)) as bf16 [dk][dv]; the slots the
+    // CUDA-core kernel writes itself stay fp32
+    int ckpt_bf16;
 };
 constexpr int kBwdChunk = 32;   // tokens per chunk of the backward
 // the two state arrays, then tc_list (16-byte multiple)
