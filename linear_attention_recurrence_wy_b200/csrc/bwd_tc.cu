@@ -671,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
 
     tmem_wait_st();   // an early exit can leave this thread's dO^T store in flight
     tc_fence_before();
-    if (tid == 0) bulk_wait_all();   // the bulk stores have read their staging and landed
+    if (tid == 0) bulk_wait_read_all();   // the bulk stores have read their shared-memory staging
     __syncthreads();
     if (sFlag[1] && tid == 0) {
         // drain: the raw copies and every committed tensor-core operation
