@@ -631,6 +631,9 @@ TRAFFIC = {
     ("gdn2_t4k", "chunk_tc"): (948.307712e6 + 124.674048e6, "01c4f4a7"),
     ("decode", "decode"): (275.810304e6 + 212.322560e6, "6e1ae928"),
     ("mixer_t4k", "chunk_tc"): (1090.264320e6 + 124.702720e6, "01c4f4a7"),
+    # the backward's step (its four launches: checkpoints, state gradient, per-chunk
+    # gradients, the strong-decay list): the inputs are read by each of the first three
+    ("bwd_t4k", "bwd"): (4774.238208e6, "34699f72"),
 }
 
 
@@ -647,6 +650,8 @@ def traffic_for(name, kname):
         return None   # the recorded figures are for the workloads' own sizes
     if name == "decode":
         key, files = ("decode", "decode"), ["decode.cu"]
+    elif name == "bwd_t4k":
+        key, files = ("bwd_t4k", "bwd"), ["chunk_tc.cu", "tri_inverse.cuh", "tc_util.cuh", "bwd_tc.cu", "bwd.cu"]
     elif "chunk_tc" in kname and "split" not in kname:
         key, files = (name, "chunk_tc"), ["chunk_tc.cu", "tri_inverse.cuh", "tc_util.cuh"]
     else:

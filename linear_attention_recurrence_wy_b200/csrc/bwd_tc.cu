@@ -100,7 +100,7 @@ constexpr uint32_t TM_DKE = 448;   // dKe^T; before it, R^T and dO^T bf16 (packe
 constexpr uint32_t TM_DEB = TM_DKB;
 constexpr uint32_t TM_RB = TM_DKE;
 constexpr uint32_t TM_DOB = TM_DKE + 32;
-constexpr uint32_t TM_VB = TM_DQK;         // v and w bf16 (packed), steps 4 to 9
+constexpr uint32_t TM_VB = TM_DQK;         // v and w bf16 (packed), steps 1 to 9
 constexpr uint32_t TM_WB = TM_DQK + 32;
 constexpr uint32_t TM_COLS = 512;
 
