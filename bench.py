@@ -629,7 +629,7 @@ def run_ours(args, rank, world, local):
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
     ("gdn2_t4k", "chunk_tc"): (948.307712e6 + 124.674048e6, "01c4f4a7"),
-    ("decode", "decode"): (275.810304e6 + 212.322560e6, "6e1ae928"),
+    ("decode", "decode"): (275.802368e6 + 209.808384e6, "131f9490"),
     ("mixer_t4k", "chunk_tc"): (1090.264320e6 + 124.702720e6, "01c4f4a7"),
     # the backward's step (its four launches: checkpoints, state gradient, per-chunk
     # gradients, the strong-decay list): the inputs are read by each of the first three
