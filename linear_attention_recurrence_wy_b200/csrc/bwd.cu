@@ -698,7 +698,9 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
                 a.B, a.H, a.T, a.dk_, a.dv_, 2 * C, a.mode, a.dtype,
                 1, a.T, 0, nullptr, nullptr, nullptr,
                 0, 1, nullptr, nullptr, 1.f, 0.f, a.ws_states, 0, nullptr};
-    const bool tc = chunk_tc_supported(f);
+    // the tensor-core path needs both the forward kernel (checkpoints, state gradient) and the
+    // per-chunk kernel to take the shape
+    const bool tc = chunk_tc_supported(f) && bwd_tc_supported(a);
     gdr_status_t st = tc ? launch_chunk_tc(f, s) : launch_chunk_simt(f, s);
     if (st != GDR_OK) return st;
     BwdArgs b = a;
