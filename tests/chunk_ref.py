@@ -79,3 +79,38 @@ def chunk_fwd(q, k, v, g, b, w=None, S0=None, mode="gdn2", C=64):
                 S = np.exp(gam[-1])[:, None] * S + (kc * np.exp(gam[-1][None, :] - gam)).T @ E
             ST[bi, hi] = S
     return o, ST
+
+
+def chunk_fwd_factorised(q, k, v, g, b, w=None, S0=None, mode="gdn2", C=64):
+    """The same forward in the factorised form the tensor-core kernel runs on chunks whose
+    cumulative decay stays within e^+-60: no per-pair decays, the decay folded into three
+    operands instead (Kh = b.k.e^gamma, Qg = q.e^gamma, Kb = k.e^-gamma) and the state scaled
+    after its update:
+
+      [A; P] = [Kh; Qg] Kb^T  (A strictly lower, P lower incl.)    T = (I + A)^-1
+      E = T (w.v - Kh S)      O = Qg S + P E      S' = diag(e^gamma_C) (S + Kb^T E)
+    """
+    q, k, v, g, b, w, S0 = map(_f64, (q, k, v, g, b, w, S0))
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    g, b, w = expand_gates(g, b, w, mode, dk, dv)
+    o = np.zeros((B, H, T, dv))
+    ST = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for hi in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else S0[bi, hi].copy()
+            for c0 in range(0, T, C):
+                sl = slice(c0, min(T, c0 + C))
+                n = min(T, c0 + C) - c0
+                e = np.exp(np.cumsum(g[bi, hi, sl], axis=0))
+                Kh = b[bi, hi, sl] * k[bi, hi, sl] * e
+                Qg = q[bi, hi, sl] * e
+                Kb = k[bi, hi, sl] / e
+                AP = np.vstack([Kh, Qg]) @ Kb.T
+                A, P = np.tril(AP[:n], -1), np.tril(AP[n:])
+                Tm = solve_triangular(np.eye(n) + A, np.eye(n), lower=True, unit_diagonal=True)
+                E = Tm @ (w[bi, hi, sl] * v[bi, hi, sl] - Kh @ S)
+                o[bi, hi, sl] = Qg @ S + P @ E
+                S = e[-1][:, None] * (S + Kb.T @ E)
+            ST[bi, hi] = S
+    return o, ST
