@@ -1,4 +1,5 @@
-// bwd.cu -- chunkwise backward of the gated delta rule on CUDA cores (fp32 arithmetic).
+// bwd.cu -- chunkwise backward of the gated delta rule: the launch sequence, and the
+// CUDA-core kernels (fp32 arithmetic) for the shapes and chunks the tensor cores do not take.
 //
 // The gradient of L = sum_t <o_t, dO_t> + <S_T, dS_T> with respect to q, k, v, the decay,
 // both gates and S0 (the gate-aware backward of Gated DeltaNet-2 Review §4-3 and the
@@ -17,18 +18,22 @@
 //   Kh, E dS'^T through Ke, dP and dA through the pair decays F; the decay gradient is
 //   the reverse cumulative sum of the gamma gradient over the chunk.
 //
-// Three launches:
+// The launches:
 //   1. the states at every 64-token boundary (the forward kernel of the shape, tcgen05 or
 //      CUDA cores, writing checkpoints and no output) -> workspace;
 //   2. the state gradient dS' entering chunks from above, walking the chunks backwards ->
 //      workspace, and dS0: for bf16 with dk = dv = 128 the tcgen05 kernel's reverse
 //      instantiation (64-token chunks; gradients at the span ends), else bwd_dstate_kernel
 //      (CUDA cores, 32-token chunks, every chunk's end);
-//   3. bwd_chunk_kernel: every 64-token span in parallel (its two chunks in turn; the first
-//      forms the middle state for the second), from S_c and dS' -> dq, dk, dv, dg, db, dw.
+//   3. for bf16 with dk = dv = 128: bwd_tc_kernel (bwd_tc.cu), the per-chunk gradients of
+//      every 64-token chunk on the tensor cores, listing the chunks whose cumulative decay
+//      is too strong for its factorised form;
+//   4. bwd_chunk_kernel: every 64-token span in parallel, or only the listed ones (its two
+//      32-token chunks in turn; the first forms the middle state for the second), from S_c
+//      and dS' -> dq, dk, dv, dg, db, dw.
 // Pair decays are formed as exp(gamma_i - gamma_j) with i >= j, never as a product of two
 // exponentials, so no factor overflows for a forgetting decay.  The CUDA-core kernels are
-// fp32 throughout.
+// fp32 throughout (states the tensor-core passes wrote are read as stored, in bf16).
 #include <algorithm>
 #include <type_traits>
 
