@@ -633,7 +633,7 @@ TRAFFIC = {
     ("mixer_t4k", "chunk_tc"): (1090.264320e6 + 124.702720e6, "01c4f4a7"),
     # the backward's step (its four launches: checkpoints, state gradient, per-chunk
     # gradients, the strong-decay list): the inputs are read by each of the first three
-    ("bwd_t4k", "bwd"): (4774.238208e6, "34699f72"),
+    ("bwd_t4k", "bwd"): (4774.238208e6, "18a6549f"),
 }
 
 
