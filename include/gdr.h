@@ -152,9 +152,15 @@ gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const void *v, co
  *   - Limit: the split's workspace, gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg),
  *     must fit in 24 MiB (e.g. B*H*nseg <= 128 at dk = dv = 128); larger requests
  *     return GDR_ERR_WORKSPACE before anything is launched.
- *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any stream
- *     capture begins.
+ *   - Arguments are checked first, exactly as gdr_chunk_fwd_split checks them; a call
+ *     that needs no workspace (one segment, or no sequence-head) runs unsplit and never
+ *     touches the array.
+ *   - The array's device address belongs to the CUDA context that loaded the library's
+ *     module.  A call made outside a stream capture looks it up afresh in the current
+ *     context (so calls after a cudaDeviceReset, or in another context, use the right
+ *     one); a call made while its stream is being captured makes no lookup and uses the
+ *     address the last uncaptured call in the same context found, so make at least one
+ *     call in each context before any stream capture begins (else GDR_ERR_CUDA).
  *   - Every call shares the one array, which keeps the previous call's contents; the
  *     split reads only what the same call wrote, so nothing needs clearing.  Calls
  *     that overlap on the GPU (for example on two streams) race on the array and must

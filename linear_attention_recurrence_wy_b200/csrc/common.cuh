@@ -108,5 +108,8 @@ unsigned long long bwd_states_bytes(int B, int H, int T, int dk, int dv);
 unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
 gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s);
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);
+// Segments the sequence split actually runs for a request of nseg (segments of whole
+// chunks, none empty); 1 for T <= 0.
+int split_effective_segments(int T, int chunk, int nseg);
 
 }  // namespace gdr

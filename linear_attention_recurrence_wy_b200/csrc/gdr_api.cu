@@ -103,6 +103,13 @@ void split_geometry(int nchunks, int nseg, int *seg_chunks, int *nseg_eff) {
 
 }  // namespace
 
+int gdr::split_effective_segments(int T, int chunk, int nseg) {
+    if (T <= 0 || chunk <= 0) return 1;
+    int sc = 1, ne = 1;
+    split_geometry((T + chunk - 1) / chunk, nseg, &sc, &ne);
+    return ne;
+}
+
 extern "C" int gdr_chunk_fwd_split_segments(int B, int H, int T, int dk, int dv, int chunk,
                                             gdr_dtype_t dtype) {
     if (B <= 0 || H <= 0 || T <= 0 || dtype != GDR_BF16 || dk != 128 || dv != 128 || chunk != 64)

@@ -21,3 +21,23 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With GDR_PARITY_TABLE=<path>, write every achieved parity error of the session
+    (whole tensor, worst sequence-head, tolerance, margin) as a markdown table."""
+    path = os.environ.get("GDR_PARITY_TABLE")
+    if not path:
+        return
+    import util
+    if not util.RECORDS:
+        return
+    lines = ["| test | tensor | metric | whole tensor | worst head | tolerance | margin |",
+             "|---|---|---|---|---|---|---|"]
+    for test, name, what, err, worst, tol in util.RECORDS:
+        top = max(err, worst or 0.0)
+        margin = f"{tol / top:.1f}x" if top > 0 else "exact"
+        w = "" if worst is None else f"{worst:.2e}"
+        lines.append(f"| {test} | {name} | {what} | {err:.2e} | {w} | {tol:g} | {margin} |")
+    with open(path, "w") as f:
+        f.write("\n".join(lines) + "\n")

@@ -3,14 +3,15 @@ against the fp64 adjoint oracle (oracle.bwd).
 
 Tolerances for the gradients: fp32 storage, max |x - x_oracle| <= 1e-4 * max(1, max |x_oracle|)
 per tensor (the forward's 1e-4, scaled to the gradient's size: a gradient sums over up to
-T tokens and d channels); bf16 storage, relative L2 <= 2e-2 per tensor, as for the forward."""
+T tokens and d channels); bf16 storage, relative L2 <= 2e-2 per tensor and per
+sequence-head, as for the forward."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import workload
-from util import assert_close, np64, rel_l2, to_dev, worst_head
+from util import assert_close, np64, record, rel_l2, to_dev, worst_head
 
 gdr = pytest.importorskip("linear_attention_recurrence_wy_b200")
 pytestmark = pytest.mark.gpu
@@ -26,12 +27,16 @@ def check_grad(name, x, ref, dtype):
         scale = max(1.0, float(np.abs(ref).max()) if ref.size else 1.0)
         err = float(np.abs(x - ref).max()) / scale if x.size else 0.0
         print(f"{name}: max abs err / scale {err:.3e} (scale {scale:.2e})")
+        record(name, "max abs / scale", err, None, 1e-4)
         assert err <= 1e-4, f"{name}: {err:.3e} > 1e-4"
     else:
         err = rel_l2(x, ref)
         worst = worst_head(x, ref, rel_l2)
         print(f"{name}: rel L2 err {err:.3e}" + ("" if worst is None else f" (worst head {worst:.3e})"))
+        record(name, "rel L2", err, worst, 2e-2)
         assert err <= 2e-2, f"{name}: {err:.3e} > 2e-2"
+        if worst is not None:
+            assert worst <= 2e-2, f"{name}: worst head {worst:.3e} > 2e-2"
 
 
 def make_case(B, H, T, dk, dv, mode, dtype, seed, s0=0.1, dst=True, g_scale=0.5):
@@ -120,11 +125,8 @@ def test_gradient_matches_finite_difference_of_the_gpu_forward(cuda_ok):
     assert abs(fd - ad) <= 2e-3 * max(1.0, abs(ad)), (fd, ad)
 
 
-SAMPLE = 3
-
-
-def test_t4k_workload_sampled_heads(cuda_ok):
-    # the T=4K workload's shape (B=8, H=16, T=4096, d=128, bf16), sampled sequence-heads
+def test_t4k_workload_all_heads(cuda_ok):
+    # the T=4K workload's shape (B=8, H=16, T=4096, d=128, bf16), every sequence-head
     wl = workload.CONFIGS["gdn2_t4k"]
     d = workload.make_inputs(wl)
     gen = torch.Generator().manual_seed(77)
@@ -134,16 +136,19 @@ def test_t4k_workload_sampled_heads(cuda_ok):
     out = gdr.chunk_bwd(dd["q"], dd["k"], dd["v"], dd["g"], dd["b"], dd["w"], dd["S0"], dO.cuda(), dST.cuda(),
                         mode="gdn2")
     torch.cuda.synchronize()
+    assert gdr.gdr_last_device_error(torch.cuda.current_stream().cuda_stream) == 0
     for n in NAMES:
         assert torch.isfinite(out[n].float()).all(), n
-    rng = np.random.default_rng(5)
-    flat = rng.choice(wl.B * wl.H, size=SAMPLE, replace=False)
-    heads = [(int(i) // wl.H, int(i) % wl.H) for i in flat]
-    pick = lambda x: None if x is None else torch.stack([x[b, h] for b, h in heads])[:, None]
-    ref = oracle.bwd(*(pick(d[n]) for n in ("q", "k", "v", "g", "b", "w", "S0")), pick(dO), pick(dST), mode="gdn2")
+    # one sequence (its 16 heads, threaded) at a time bounds the fp64 copies' host memory
+    refs = {n: [] for n in NAMES}
+    for i in range(wl.B):
+        one = lambda x: None if x is None else x[i:i + 1]
+        r = oracle.bwd(*(one(d[n]) for n in ("q", "k", "v", "g", "b", "w", "S0")), one(dO), one(dST),
+                       mode="gdn2")
+        for n in NAMES:
+            refs[n].append(r[n])
     for n in NAMES:
-        got = np.stack([np64(out[n][b, h]) for b, h in heads])
-        check_grad(f"t4k {n}", got, ref[n][:, 0], "bf16")
+        check_grad(f"t4k {n}", np64(out[n]), np.concatenate(refs[n]), "bf16")
 
 
 # ---- the tensor-core shape (bf16, dk = dv = 128): checkpoints, the state gradient and the

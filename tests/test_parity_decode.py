@@ -75,7 +75,7 @@ def test_decode_workload_1000_steps(cuda_ok):
     # sampled (sequence, head) pairs; each is independent of the others
     rng = np.random.default_rng(5)
     N, H = cfg["N"], cfg["H"]
-    flat = rng.choice(N * H, size=24, replace=False)
+    flat = rng.choice(N * H, size=256, replace=False)
     ns, hs = flat // H, flat % H
     Sr = pool["S0"][ns, hs][:, None].double().numpy()
     for s in range(steps):
@@ -84,7 +84,7 @@ def test_decode_workload_1000_steps(cuda_ok):
         o_ref, Sr = oracle.decode(sel(st["q"]), sel(st["k"]), sel(st["v"]), sel(st["g"]),
                                   sel(st["b"]), sel(st["w"]), S=Sr, mode="gdn2")
         if s < P:
-            assert_close(f"o step {s}", np64(outs[s][ns, hs]), o_ref[:, 0], "bf16")
-    assert_close("S after 1000 steps", np64(S[ns, hs]), Sr[:, 0], "bf16")
+            assert_close(f"o step {s}", np64(outs[s][ns, hs]), o_ref[:, 0], "bf16", head_axes=1)
+    assert_close("S after 1000 steps", np64(S[ns, hs]), Sr[:, 0], "bf16", head_axes=1)
     # the fp32 state itself is carried in fp32 on both sides: check it tightly too
     assert np.max(np.abs(np64(S[ns, hs]) - Sr[:, 0])) < 1e-4
