@@ -273,6 +273,22 @@ gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *v, const fl
  */
 gdr_status_t gdr_last_device_error(void *stream);
 
+/*
+ * gdr_test_set_first_wait_limit -- test hook for the bounded-wait expiry path.  The pages
+ * have no counterpart to it.
+ *
+ * polls != 0: in every call enqueued afterwards, the first mbarrier wait of each CTA of the
+ * tensor-core forward (its state group's wait for the first chunk's operands), of the
+ * streaming decode kernel (its first state copy) and of the tensor-core per-chunk backward
+ * kernel (its raw input copies) gives up after `polls` non-blocking polls instead of the
+ * normal bound of 2^24.  The producer is then merely still working, so the expiry path
+ * (abort flag, drain of the kernel's own copies and tensor-core work, TMEM released)
+ * runs for real and gdr_last_device_error() reports GDR_ERR_TIMEOUT; the outputs of such a
+ * call are unspecified.  polls = 0 (the default) restores the normal bound.  Host-side
+ * state of the library, not thread-safe; for tests only.
+ */
+void gdr_test_set_first_wait_limit(unsigned polls);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *gdr_status_string(gdr_status_t status);
 

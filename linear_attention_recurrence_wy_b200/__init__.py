@@ -8,7 +8,7 @@ PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raise
 Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
 gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
 gdr_mixer_fwd, gdr_chunk_bwd, gdr_chunk_bwd_workspace, gdr_decode_step,
-gdr_last_device_error, gdr_status_string.
+gdr_last_device_error, gdr_status_string, gdr_test_set_first_wait_limit.
 Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
 chunk_bwd, decode_step.
 """
@@ -62,6 +62,8 @@ def lib():
         L.gdr_decode_step.restype = ci
         L.gdr_last_device_error.argtypes = [vp]
         L.gdr_last_device_error.restype = ci
+        L.gdr_test_set_first_wait_limit.argtypes = [ctypes.c_uint]
+        L.gdr_test_set_first_wait_limit.restype = None
         L.gdr_status_string.argtypes = [ci]
         L.gdr_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -116,6 +118,12 @@ def gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, strea
 
 def gdr_last_device_error(stream=None):
     return lib().gdr_last_device_error(stream)
+
+
+def gdr_test_set_first_wait_limit(polls: int) -> None:
+    """Test hook: the first bounded wait of each CTA gives up after `polls` non-blocking
+    polls (0 restores the normal bound); see include/gdr.h."""
+    lib().gdr_test_set_first_wait_limit(polls)
 
 
 def gdr_status_string(code: int) -> str:

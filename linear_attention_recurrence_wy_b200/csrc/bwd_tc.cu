@@ -50,7 +50,6 @@ using namespace tc;
 
 constexpr int C = 64, DK = 128, DV = 128;
 constexpr int kThreads = 256;
-constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kFastLimit = 60.f;
 
 // shared memory map (byte offsets from a 1024-aligned base)
@@ -196,8 +195,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     int raw_copies = 0;       // rounds of raw input copies issued on bar_raw
     bool raw_pending = false;
     // Bounded wait for a phase of an mbarrier: thread 0 polls, the block meets at a barrier.
+    // test hook (see BwdArgs): the first wait, on the raw copies, polls them right after they
+    // are issued, a few non-blocking times, and gives up while they are still in flight
+    bool first_expired = false;
     auto wait_bar = [&](uint32_t bar, uint32_t parity) -> bool {
-        if (tid == 0 && !mbar_wait(bar, parity, kWaitLimit)) sFlag[1] = 1;
+        if (tid == 0 && (first_expired || !mbar_wait(bar, parity, a.wait_limit))) sFlag[1] = 1;
+        first_expired = false;
         __syncthreads();
         return sFlag[1] == 0;
     };
@@ -217,6 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
             bulk_g2s(sbase + OFF_RDO, dOg + tok0 * DV, row16, bar_raw);
             bulk_g2s(sbase + OFF_RV, V + tok0 * DV, row16, bar_raw);
             if (vec_w) bulk_g2s(sbase + OFF_RW, Wg + tok0 * DV, row16, bar_raw);
+            if (a.first_wait_limit != 0) {
+                bool got = false;
+                for (uint32_t i = 0; i < a.first_wait_limit && !got; ++i) got = mbar_test_wait(bar_raw, 0u);
+                first_expired = !got;
+            }
         }
         ++raw_copies;
         raw_pending = true;
@@ -676,11 +684,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     if (sFlag[1] && tid == 0) {
         // drain: the raw copies and every committed tensor-core operation
         atomicExch(&g_bwd_tc_error, 1);
-        if (raw_pending) mbar_wait(bar_raw, (uint32_t)((raw_copies - 1) & 1), kWaitLimit);
+        if (raw_pending) mbar_wait(bar_raw, (uint32_t)((raw_copies - 1) & 1), a.wait_limit);
         mma_commit(bar_mma);
         const int k = commits + 1;
-        if (k >= 2) mbar_wait(bar_mma, (uint32_t)((k - 2) & 1), kWaitLimit);
-        mbar_wait(bar_mma, (uint32_t)((k - 1) & 1), kWaitLimit);
+        if (k >= 2) mbar_wait(bar_mma, (uint32_t)((k - 2) & 1), a.wait_limit);
+        mbar_wait(bar_mma, (uint32_t)((k - 1) & 1), a.wait_limit);
     }
     __syncthreads();
     tc_fence_after();

@@ -71,7 +71,6 @@ using namespace tc;
 
 constexpr int C = 64, DK = 128, DV = 128;
 constexpr int kThreads = 512;
-constexpr uint32_t kWaitLimit = 1u << 24;
 constexpr float kFastLimit = 60.f;
 constexpr float kFastProd = 8.7565108e-27f;   // e^-60: the same limit on e^gamma
 constexpr int kAS = tri::LD;   // fp32 row stride of the A / T scratch
@@ -180,9 +179,9 @@ __device__ __forceinline__ float sigmoid_gate(float x) { return fmaf(0.5f, tanh_
 // After an abort: wait (bounded) until every commit issued on bar has arrived.  The
 // commits complete in order; n of them were issued, so phases n-2 and n-1 are waited
 // for in turn (a parity wait alone cannot tell phase n-1 from phase n-3).
-__device__ __forceinline__ void drain_commits(uint32_t bar, int n) {
-    if (n >= 2) mbar_wait(bar, (uint32_t)((n - 2) & 1), kWaitLimit);
-    if (n >= 1) mbar_wait(bar, (uint32_t)((n - 1) & 1), kWaitLimit);
+__device__ __forceinline__ void drain_commits(uint32_t bar, int n, uint32_t limit) {
+    if (n >= 2) mbar_wait(bar, (uint32_t)((n - 2) & 1), limit);
+    if (n >= 1) mbar_wait(bar, (uint32_t)((n - 1) & 1), limit);
 }
 
 // Exact path, strong-decay chunks only: A (fp32, strictly lower) and P (bf16 tile, lower
@@ -359,8 +358,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
     // barrier (bar.red), which also carries the outcome and orders their later reads
     // after the phase completed.  Polling by every thread would steal shared-memory and
     // issue bandwidth from the other group.
+    const uint32_t wait_limit = a.wait_limit;
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        for (uint32_t i = 0; i < kWaitLimit; ++i) {
+        for (uint32_t i = 0; i < wait_limit; ++i) {
             if (mbar_try_wait(bar, parity)) return true;
             if ((i & 255) == 255 && sAbort[0]) return false;
         }
@@ -698,6 +698,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         const float nwv = kMixer ? a.nw[v] : 0.f;
         const float wact = (mode == GDR_MODE_KDA || mode == GDR_MODE_GDN) ? a.b_range : 1.f;
         bool ok = true;
+        if (a.first_wait_limit != 0) {
+            // test hook: the group's first wait (for chunk 0's operands) happens at once and
+            // gives up after a few non-blocking polls, while the WY group is still loading
+            bool got = stid != 0;
+            for (uint32_t i = 0; i < a.first_wait_limit && !got; ++i) got = mbar_test_wait(bar_h1, 0u);
+            if (!got) sAbort[0] = 1;
+            ok = group_and(BAR_ST, got);
+        }
         // initial state -> TMEM: fp32 S^T and its bf16 operand copy
         for (int d0 = half * 64; d0 < half * 64 + 64; d0 += 32) {
             float x[32];
@@ -717,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         tmem_wait_st();
         tc_fence_before();
         group_sync(BAR_ST);
-        for (int c = 0; !kReverse && c < nchunks; ++c) {
+        for (int c = 0; ok && !kReverse && c < nchunks; ++c) {
             const int t0 = dch(c) * C, n = min(C, T - t0);
             const int pb = c & 1;
             const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
@@ -961,7 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         //        G^T <- G^T diag(e^gamma_C) + dO^T Qg - dR^T Kh
         //      Before each chunk's update G is the gradient at the chunk's end: it goes to the
         //      checkpoint slot of the chunk's last 32-token chunk. ----
-        for (int c = 0; kReverse && c < nchunks; ++c) {
+        for (int c = 0; ok && kReverse && c < nchunks; ++c) {
             const int cd = dch(c);
             const int t0 = cd * C, n = min(C, T - t0);
             const int pb = c & 1;
@@ -1112,12 +1120,12 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         if (tid == 0) {
             atomicExch(&g_tc_error, 1);
             mma_commit(bar_wy);
-            drain_commits(bar_wy, mma_wy + 1);
-            if (raw_issued > raw_done) mbar_wait(bar_raw, (uint32_t)(raw_done & 1), kWaitLimit);
+            drain_commits(bar_wy, mma_wy + 1, wait_limit);
+            if (raw_issued > raw_done) mbar_wait(bar_raw, (uint32_t)(raw_done & 1), wait_limit);
         }
         if (tid == 256) {
             mma_commit(bar_st);
-            drain_commits(bar_st, mma_st + 1);
+            drain_commits(bar_st, mma_st + 1, wait_limit);
         }
     }
     __syncthreads();
@@ -1131,10 +1139,8 @@ bool chunk_tc_supported(const ChunkArgs &a) {
     return a.dtype == GDR_BF16 && a.dk == DK && a.dv == DV && a.chunk == C;
 }
 
-namespace {
-
 // cuTensorMapEncodeTiled from the driver, looked up once (no link against libcuda)
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
     std::call_once(once, [] {
@@ -1148,6 +1154,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     });
     return fn;
 }
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tensor_map_encode_fn(); }
 
 // Map of a token-major [B, T, H, D] tensor (D = 128 elements of esize bytes): dims
 // {D, H, T, B}, box {D, 1, C, 1}, no swizzle, zero fill out of range.

@@ -44,6 +44,12 @@ struct ChunkArgs {
     // gradient at every 64-token chunk's end (slot of its last 32-token chunk), as bf16.
     int reverse;
     const void *dO;
+    // Bounded waits: polls of an mbarrier before a kernel gives up and reports
+    // GDR_ERR_TIMEOUT.  first_wait_limit != 0 is a test hook: the tensor-core forward's state
+    // group then gives up its very first wait after that many non-blocking polls, so the
+    // expiry path runs while the WY group is merely still working.
+    unsigned wait_limit = 1u << 24;
+    unsigned first_wait_limit = 0;
 };
 
 struct DecodeArgs {
@@ -52,6 +58,10 @@ struct DecodeArgs {
     float *S;
     void *o;
     int N, H, dk, dv, mode, dtype;
+    // bounded waits of the streaming kernel, as in ChunkArgs (first_wait_limit: a test hook
+    // that makes each CTA's first wait give up after that many non-blocking polls)
+    unsigned wait_limit = 1u << 24;
+    unsigned first_wait_limit = 0;
 };
 
 // Gate shapes per mode: the erase gate b and the write gate w are per channel or one
@@ -101,6 +111,10 @@ struct BwdArgs {
     // state gradients (ws_dstates slot min(2 span + 1, last)) as bf16 [dk][dv]; the slots the
     // CUDA-core kernel writes itself stay fp32
     int ckpt_bf16;
+    // bounded waits of the tensor-core per-chunk kernel, as in ChunkArgs (first_wait_limit: a
+    // test hook that makes each CTA's first wait give up after that many non-blocking polls)
+    unsigned wait_limit = 1u << 24;
+    unsigned first_wait_limit = 0;
 };
 constexpr int kBwdChunk = 32;   // tokens per chunk of the backward
 // the two state arrays, then tc_list (16-byte multiple)

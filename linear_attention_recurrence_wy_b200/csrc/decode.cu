@@ -132,7 +132,6 @@ constexpr int kBufs = 3;                      // state buffers
 constexpr int kStateBytes = SD * SD * 4;      // 64 KB
 constexpr int kVecSlot = 512;                 // one per-head vector, bf16 or fp32
 constexpr int kVecBytes = 6 * kVecSlot;       // q, k, b, w, v, g
-constexpr uint32_t kStreamWaitLimit = 1u << 24;
 // dynamic shared memory map
 constexpr int SO_BUF = 0;
 constexpr int SO_VEC = kBufs * kStateBytes;                 // [2][kVecBytes]
@@ -210,10 +209,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
         if (!vec_w) vb[3 * kVecSlot / 4] = pend_w;   // scalar write gate in slot 3
         if (!vec_g) vb[5 * kVecSlot / 4] = pend_g;   // scalar g_log in slot 5
     };
+    bool first_expired = false;   // thread 0: the test hook's first wait gave up
     // bounded wait on a state buffer; gives up early once another thread has aborted
     auto wait_full = [&](int i) -> bool {
         const uint32_t bar = bar_full + 8 * (i % kBufs), parity = (uint32_t)((i / kBufs) & 1);
-        for (uint32_t n = 0; n < kStreamWaitLimit; ++n) {
+        if (i == 0 && a.first_wait_limit != 0 && first_expired) {
+            *s_abort = 1;   // test hook: see the first load below
+            return false;
+        }
+        for (uint32_t n = 0; n < a.wait_limit; ++n) {
             if (tc::mbar_try_wait(bar, parity)) return true;
             if ((n & 255) == 255 && *s_abort) return false;
         }
@@ -236,6 +240,13 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
     int loads = 0;
     if (tid == 0) {
         for (; loads < 2 && loads < iters; ++loads) issue_load(loads);
+        if (a.first_wait_limit != 0 && iters > 0) {
+            // test hook: the first wait on a state copy polls it right after the issue, a few
+            // non-blocking times, and gives up while the copy is still in flight
+            bool got = false;
+            for (uint32_t n = 0; n < a.first_wait_limit && !got; ++n) got = tc::mbar_test_wait(bar_full, 0u);
+            first_expired = !got;
+        }
     }
     if (iters > 0) {
         fetch_vectors(0);
@@ -336,7 +347,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
             atomicExch(&g_decode_error, 1);
             // drain: the loads issued but not consumed, at most the last two (bounded)
             for (int i = loads > 2 ? loads - 2 : 0; i < loads; ++i)
-                tc::mbar_wait(bar_full + 8 * (i % kBufs), (uint32_t)((i / kBufs) & 1), kStreamWaitLimit);
+                tc::mbar_wait(bar_full + 8 * (i % kBufs), (uint32_t)((i / kBufs) & 1), a.wait_limit);
         }
         cp_async_wait_all();
     }

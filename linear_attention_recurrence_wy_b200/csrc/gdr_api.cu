@@ -43,6 +43,10 @@ gdr_status_t check_chunk(const void *q, const void *k, const void *v, const floa
     return GDR_OK;
 }
 
+// Test hook (gdr_test_set_first_wait_limit): 0, the default, leaves every wait at its
+// normal bound.
+unsigned g_first_wait_limit = 0;
+
 ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_log, const void *b,
                     const void *w, const float *S0, void *o, float *S_T, int B, int H, int T,
                     int dk, int dv, int chunk, int mode, int dtype) {
@@ -50,6 +54,7 @@ ChunkArgs make_args(const void *q, const void *k, const void *v, const float *g_
                 B, H, T, dk, dv, chunk, mode, dtype,
                 1, T, 0, nullptr, nullptr, nullptr,
                 0, 1, nullptr, nullptr, 1.f, 0.f, nullptr, 0, nullptr};
+    a.first_wait_limit = g_first_wait_limit;
     return a;
 }
 
@@ -234,6 +239,7 @@ extern "C" gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *
               dq, dk_, dv_, db, mode_uses_w(mode) ? dw : nullptr, dg, dS0,
               B, H, T, dk, dv, (int)mode, (int)dtype,
               static_cast<float *>(workspace), static_cast<float *>(workspace) + per, 0, nullptr};
+    a.first_wait_limit = g_first_wait_limit;
     return launch_bwd(a, s);
 }
 
@@ -252,6 +258,7 @@ extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void
         return GDR_ERR_ALIGN;
     DecodeArgs a{q, k, v, b, mode_uses_w(mode) ? w : nullptr, g_log, S, o,
                  N, H, dk, dv, (int)mode, (int)dtype};
+    a.first_wait_limit = g_first_wait_limit;
     return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -264,6 +271,8 @@ extern "C" gdr_status_t gdr_last_device_error(void *stream) {
     if (bwd_tc_read_and_clear_error(&berr) != cudaSuccess) return GDR_ERR_CUDA;
     return (err || derr || berr) ? GDR_ERR_TIMEOUT : GDR_OK;
 }
+
+extern "C" void gdr_test_set_first_wait_limit(unsigned polls) { g_first_wait_limit = polls; }
 
 extern "C" const char *gdr_status_string(gdr_status_t status) {
     switch (status) {

@@ -189,6 +189,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t saddr, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking test of the phase with the given parity (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t saddr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(saddr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase with the given parity; false if the limit was reached.
 __device__ __forceinline__ bool mbar_wait(uint32_t saddr, uint32_t parity, uint32_t limit) {
     for (uint32_t i = 0; i < limit; ++i)
@@ -221,6 +233,21 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst_saddr, const void *tmap
         "%4, %5}], [%6];" ::"r"(dst_saddr),
         "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(mbar_saddr)
         : "memory");
+}
+// Tiled tensor copy (TMA) of one box of a 2-D tensor map into shared memory, completing on
+// mbar.  The innermost coordinate c0 must be a multiple of 16 bytes' worth of elements.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst_saddr, const void *tmap, int c0, int c1,
+                                            uint32_t mbar_saddr) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(dst_saddr),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(mbar_saddr)
+        : "memory");
+}
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t saddr) {
+    uint2 r;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(saddr) : "memory");
+    return r;
 }
 // Tiled tensor store (TMA) of one box from shared memory; out-of-range rows are clipped.
 // Completion is tracked by the issuing thread's bulk async-groups.
@@ -259,6 +286,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
                                              uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
 }
 
 // ---- element conversions and tile stores ------------------------------------------------

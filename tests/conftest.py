@@ -23,21 +23,55 @@ def cuda_ok():
     return True
 
 
+WORKLOAD_TESTS = ("full_size", "all_heads", "1000_steps", "long_context")
+
+
+def parity_table(records):
+    """Markdown summary of the parity records (util.RECORDS): the measured workloads at full
+    size (every sequence-head; a decode run's per-step rows folded into one), then the
+    tightest check of each test file, then the totals."""
+    def margin(err, worst, tol):
+        top = max(err, worst or 0.0)
+        return tol / top if top > 0 else float("inf")
+
+    def fmt_row(test, name, what, err, worst, tol):
+        m = margin(err, worst, tol)
+        w = "" if worst is None else f"{worst:.2e}"
+        return f"| {test} | {name} | {what} | {err:.2e} | {w} | {tol:g} | {'exact' if m == float('inf') else f'{m:.1f}x'} |"
+
+    head = ["| test | tensor | metric | whole tensor | worst head | tolerance | margin |",
+            "|---|---|---|---|---|---|---|"]
+    out = ["## Measured workloads at full size (every sequence-head compared)", ""] + head
+    folded = {}
+    for test, name, what, err, worst, tol in records:
+        if not any(k in test for k in WORKLOAD_TESTS):
+            continue
+        key = (test, "o (every step)" if name.startswith("o step") else name, what, tol)
+        e0, w0, n0 = folded.get(key, (0.0, None, 0))
+        folded[key] = (max(e0, err), None if worst is None and w0 is None else max(w0 or 0.0, worst or 0.0), n0 + 1)
+    for (test, name, what, tol), (err, worst, n) in folded.items():
+        out.append(fmt_row(test.split("::")[-1], name + (f" ({n} checks, max)" if n > 1 else ""), what, err, worst, tol))
+    out += ["", "## Tightest check of each test file", ""] + head
+    tight = {}
+    for r in records:
+        f = r[0].split("::")[0]
+        if f not in tight or margin(*r[3:]) < margin(*tight[f][3:]):
+            tight[f] = r
+    for f, r in sorted(tight.items()):
+        out.append(fmt_row(r[0].split("/")[-1], *r[1:]))
+    out += ["", f"{len(records)} checks in all; tightest margin "
+            f"{min(margin(*r[3:]) for r in records):.1f}x of its tolerance."]
+    return "\n".join(out) + "\n"
+
+
 def pytest_sessionfinish(session, exitstatus):
-    """With GDR_PARITY_TABLE=<path>, write every achieved parity error of the session
-    (whole tensor, worst sequence-head, tolerance, margin) as a markdown table."""
+    """With GDR_PARITY_TABLE=<path>, write the achieved parity errors of the session (whole
+    tensor, worst sequence-head, tolerance, margin) as a markdown summary."""
     path = os.environ.get("GDR_PARITY_TABLE")
     if not path:
         return
     import util
     if not util.RECORDS:
         return
-    lines = ["| test | tensor | metric | whole tensor | worst head | tolerance | margin |",
-             "|---|---|---|---|---|---|---|"]
-    for test, name, what, err, worst, tol in util.RECORDS:
-        top = max(err, worst or 0.0)
-        margin = f"{tol / top:.1f}x" if top > 0 else "exact"
-        w = "" if worst is None else f"{worst:.2e}"
-        lines.append(f"| {test} | {name} | {what} | {err:.2e} | {w} | {tol:g} | {margin} |")
     with open(path, "w") as f:
-        f.write("\n".join(lines) + "\n")
+        f.write(parity_table(util.RECORDS))
