@@ -369,16 +369,15 @@ def config_of(name, world):
             else "L2 flushed between steps", "parallelism": f"replicas{world}"}
 
 
-def run_ours(args, rank, world, local):
+def setup_workload(name, rank, dev, decode_steps=None):
+    """Inputs resident on `dev` and the callables of one bench step of workload `name`.
+    Returns a dict: step (one whole step, L2 flush included), fwd (the timed launches),
+    flush (a buffer written between timed launches, or None), units, unit,
+    bytes_per_launch, launches_per_step, kernel (name of the timed kernels), flops (tensor
+    products per step, or None), nseg, and the host-side inputs for the end-to-end leg."""
     import linear_attention_recurrence_wy_b200 as gdr
-    gdr.lib()
-    name = args.workload
-    dev = torch.device("cuda", local)
-    hbm, tf_burst, tf_sust, peak_src = load_peaks()
     wl, mode = rank_workload(name, rank)
-    stream = torch.cuda.current_stream(dev)
-    flush = None
-
+    r = dict(name=name, wl=wl, mode=mode, flush=None, flops=None, nseg=1, unit="token-heads/s")
     if name == "mixer_t4k":
         c = wl
         inp = workload.make_mixer_inputs(c["B"], c["H"], c["T"], c["dk"], c["dv"], mode=c["mode"],
@@ -391,12 +390,9 @@ def run_ours(args, rank, world, local):
         def fwd():
             gdr.mixer_fwd(d["q"], d["k"], d["v"], d["xg"], d["xb"], d["xw"], d["z"], d["weight"], d["S0"],
                           mode=c["mode"], layout=c["layout"], y=y, S_T=ST)
-        step = fwd
-        units = c["B"] * c["H"] * c["T"]
-        bytes_per_launch = mixer_bytes(c)
-        launches_per_step = 1
-        unit = "token-heads/s"
-        nseg = 1
+        r.update(fwd=fwd, step=fwd, units=c["B"] * c["H"] * c["T"], bytes_per_launch=mixer_bytes(c),
+                 launches_per_step=1, inp=inp, out=(y, ST),
+                 kernel="gdr chunk_tc_kernel<mixer> (tcgen05, fused prologue/epilogue)")
     elif name == "bwd_t4k":
         inp = workload.make_inputs(wl, mode=mode)
         d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
@@ -412,33 +408,33 @@ def run_ours(args, rank, world, local):
         def fwd():
             gdr.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], dO, dST, mode=mode,
                           workspace=ws, out=grads)
-        step = fwd
-        units = wl.units
-        bytes_per_launch = bwd_bytes(wl)
-        launches_per_step = 4
-        unit = "token-heads/s"
-        nseg = 1
+        # one step = the whole backward (states, state gradient, per-chunk gradients, and the
+        # CUDA-core kernel for strong-decay spans, none here), the unit of the roofline
+        r.update(fwd=fwd, step=fwd, units=wl.units, bytes_per_launch=bwd_bytes(wl), launches_per_step=4,
+                 flops=bwd_flops(wl), inp=inp, dO=dO, dST=dST, ws=ws, grads=grads,
+                 kernel="gdr chunk_tc_kernel (checkpoints) + chunk_tc_kernel (state gradient) + "
+                        "bwd_tc_kernel + bwd_chunk_kernel (backward, 4 launches, tcgen05)")
     elif name == "decode":
         pool = workload.make_decode_pool(wl)
         d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in pool.items()}
         S = d["S0"].clone()
         P = wl["pool"]
-        n_inner = args.decode_steps or wl["steps"]
+        n_inner = decode_steps or wl["steps"]
 
         def step():
-            for s in range(n_inner):
-                p = s % P
-                gdr.decode_step(d["q"][p], d["k"][p], d["v"][p], d["g"][p], d["b"][p], d["w"][p], S,
+            for s_ in range(n_inner):
+                p_ = s_ % P
+                gdr.decode_step(d["q"][p_], d["k"][p_], d["v"][p_], d["g"][p_], d["b"][p_], d["w"][p_], S,
                                 mode="gdn2")
-        units = wl["N"] * wl["H"] * n_inner
-        bytes_per_launch = decode_bytes(wl)
-        launches_per_step = n_inner
-        unit = "step-heads/s"
+        r.update(fwd=step, step=step, units=wl["N"] * wl["H"] * n_inner, bytes_per_launch=decode_bytes(wl),
+                 launches_per_step=n_inner, unit="step-heads/s",
+                 kernel="gdr decode_stream_kernel" if wl["dk"] == wl["dv"] == 128 else "gdr decode_kernel")
     else:
         inp = workload.make_inputs(wl, mode=mode)
         d = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in inp.items()}
         o = torch.empty(wl.B, wl.H, wl.T, wl.dv, dtype=d["q"].dtype, device=dev)
         ST = torch.empty(wl.B, wl.H, wl.dk, wl.dv, dtype=torch.float32, device=dev)
+        flush = None
         if chunk_bytes(wl, mode) <= 126e6:
             flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         dt_code = 1 if wl.dtype == "bf16" else 0
@@ -460,58 +456,111 @@ def run_ours(args, rank, world, local):
             if flush is not None:
                 flush.zero_()
             fwd()
-        units = wl.units
-        bytes_per_launch = chunk_bytes(wl, mode)
-        launches_per_step = 3 if nseg > 1 else 1
-        unit = "token-heads/s"
+        # one step = the whole forward; with a sequence split it is three launches (state
+        # pass, combine, output pass) and the step is the unit of the roofline
+        r.update(fwd=fwd, step=step, flush=flush, units=wl.units, bytes_per_launch=chunk_bytes(wl, mode),
+                 launches_per_step=3 if nseg > 1 else 1, flops=chunk_flops(wl), nseg=nseg, inp=inp,
+                 out=(o, ST), kernel=kernel_name(wl, mode) if nseg <= 1 else
+                 f"gdr chunk_tc_kernel x2 + split_combine_kernel (sequence split, {nseg} segments)")
+    return r
 
-    for _ in range(args.warmup):
-        step()
+
+def time_device(r, steps, warmup, world, local, stream):
+    """W untimed steps, then `steps` timed ones: CUDA events on the launching stream around
+    each step's launches (the L2 flush, if any, between them), clocks sampled meanwhile,
+    barrier + synchronize on both sides.  Returns (mean ms per step, total ms, clocks)."""
+    import linear_attention_recurrence_wy_b200 as gdr
+    dev = torch.device("cuda", local)
+    for _ in range(warmup):
+        r["step"]()
     torch.cuda.synchronize(dev)
     rc = gdr.gdr_last_device_error(stream.cuda_stream)
     if rc != 0:
         raise RuntimeError(f"device error after warm-up: {gdr.gdr_status_string(rc)}")
-
-    # kernel-only timing: events around each step on the launching stream
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         t_start.record(stream)
-        for i in range(args.steps):
-            if flush is not None:
-                flush.zero_()
+        for i in range(steps):
+            if r["flush"] is not None:
+                r["flush"].zero_()
             ev[i][0].record(stream)
-            if name == "decode":
-                step()
-            else:
-                fwd()
+            r["fwd"]()
             ev[i][1].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = t_start.elapsed_time(t_end)
-    kern_ms = sum(step_ms) / len(step_ms)
-    ms_per_step = max_over_ranks(kern_ms, world)
-    value = units * world / (ms_per_step * 1e-3)
     rc = gdr.gdr_last_device_error(stream.cuda_stream)
     if rc != 0:
         raise RuntimeError(f"device error in timed region: {gdr.gdr_status_string(rc)}")
+    return sum(step_ms) / len(step_ms), t_start.elapsed_time(t_end), clk.summary()
+
+
+def roofline_of(r, ms, hbm, tf_burst, peak_src):
+    achieved = r["bytes_per_launch"] / (ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+            "traffic": traffic_for(r["name"], r["kernel"]), "peak_source": f"{peak_src} hbm_gbs",
+            "kernel": r["kernel"]}
+    if r["flops"] is not None:
+        roof["tensor_context"] = {"flops_per_launch": r["flops"],
+                                  "achieved_tflops": r["flops"] / (ms * 1e-3) / 1e12,
+                                  "peak_tflops": tf_burst,
+                                  "frac": r["flops"] / (ms * 1e-3) / 1e12 / tf_burst}
+    return roof
+
+
+# Workloads timed beside the headline on a one-GPU run (the `secondary` object): the decode
+# target, the other chunked shapes, the fused token mixer and the backward.
+SECONDARY = ("decode", "gdn_t2k", "gdn2_t16k", "gdn2_t16k_kda", "mixer_t4k", "bwd_t4k")
+
+
+def run_secondary(names, steps, local, stream, hbm, tf_burst, peak_src):
+    out = {}
+    dev = torch.device("cuda", local)
+    for name in names:
+        r = setup_workload(name, 0, dev)
+        ms, _, clk = time_device(r, steps, 3, 1, local, stream)
+        roof = roofline_of(r, ms / (r["launches_per_step"] if name == "decode" else 1), hbm, tf_burst, peak_src)
+        out[name] = {"ms_per_step": ms, "value": r["units"] / (ms * 1e-3), "unit": r["unit"],
+                     "steps": steps, "launches_per_step": r["launches_per_step"],
+                     "config": config_of(name, 1), "roofline": roof, "clocks": clk}
+        if name == "decode":
+            out[name]["us_per_decode_step"] = 1e3 * ms / r["launches_per_step"]
+        del r
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local):
+    import linear_attention_recurrence_wy_b200 as gdr
+    gdr.lib()
+    name = args.workload
+    dev = torch.device("cuda", local)
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    r = setup_workload(name, rank, dev, decode_steps=args.decode_steps)
+    wl, mode, units, unit = r["wl"], r["mode"], r["units"], r["unit"]
+    kern_ms, total_ms, clk = time_device(r, args.steps, args.warmup, world, local, stream)
+    ms_per_step = max_over_ranks(kern_ms, world)
+    value = units * world / (ms_per_step * 1e-3)
 
     # end to end through the public API with host buffers (pinned), copies inside
     e2e = None
     if not args.no_e2e and name == "bwd_t4k":
+        inp = r["inp"]
         hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
-        dOh, dSTh = dO.cpu().pin_memory(), dST.cpu().pin_memory()
-        outh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in grads.items()}
+        dOh, dSTh = r["dO"].cpu().pin_memory(), r["dST"].cpu().pin_memory()
+        outh = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in r["grads"].items()}
         h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v)) + \
             dOh.numel() * dOh.element_size() + dSTh.numel() * dSTh.element_size()
         d2h = sum(x.numel() * x.element_size() for x in outh.values())
         n_e2e = max(1, min(args.steps, 3))
+        ws = r["ws"]
 
         def call():
             x = {k: (v.to(dev, non_blocking=True) if torch.is_tensor(v) else v) for k, v in hin.items()}
@@ -534,8 +583,10 @@ def run_ours(args, rank, world, local):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     elif not args.no_e2e and name == "mixer_t4k":
         c = wl
+        inp = r["inp"]
         hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
         h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v))
+        y, ST = r["out"]
         outh = (torch.empty(y.shape, dtype=y.dtype, pin_memory=True),
                 torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True))
         d2h = sum(x.numel() * x.element_size() for x in outh)
@@ -556,69 +607,53 @@ def run_ours(args, rank, world, local):
         e2e = {"value": units * world / (e2e_ms * 1e-3), "unit": unit,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     elif not args.no_e2e and name != "decode":
+        inp = r["inp"]
         hin = {k: (v.pin_memory() if torch.is_tensor(v) else v) for k, v in inp.items()}
         h2d = sum(v.numel() * v.element_size() for v in hin.values() if torch.is_tensor(v))
+        o, ST = r["out"]
         outh = (torch.empty(o.shape, dtype=o.dtype, pin_memory=True),
                 torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True))
         d2h = sum(x.numel() * x.element_size() for x in outh)
         n_e2e = max(1, min(args.steps, 5))
-        gdr.chunk_fwd_host(hin["q"], hin["k"], hin["v"], hin["g"], hin["b"], hin["w"], hin["S0"],
-                           mode=mode, chunk=wl.chunk, device=dev, out=outh)
+        call = lambda: gdr.chunk_fwd_host(hin["q"], hin["k"], hin["v"], hin["g"], hin["b"], hin["w"],
+                                          hin["S0"], mode=mode, chunk=wl.chunk, device=dev, out=outh)
+        call()
         torch.cuda.synchronize(dev)
         barrier(world)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(n_e2e):
-            gdr.chunk_fwd_host(hin["q"], hin["k"], hin["v"], hin["g"], hin["b"], hin["w"], hin["S0"],
-                               mode=mode, chunk=wl.chunk, device=dev, out=outh)
+            call()
         b.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, world)
         e2e = {"value": units * world / (e2e_ms * 1e-3), "unit": unit,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
-    elif name == "decode":
-        e2e = None
 
+    launches_per_step = r["launches_per_step"]
+    # the roofline's unit: one decode launch, else the whole step
+    launch_ms = kern_ms / launches_per_step if name == "decode" else kern_ms
+    roof = roofline_of(r, launch_ms, hbm, tf_burst, peak_src)
+    del r
+    torch.cuda.empty_cache()
+    secondary = None
+    if world == 1 and not args.no_secondary and BATCH is None:
+        secondary = run_secondary([n for n in SECONDARY if n != name], args.secondary_steps, local, stream,
+                                  hbm, tf_burst, peak_src)
     if rank != 0:
         return
-    if name == "decode":
-        launch_ms = kern_ms / launches_per_step
-        kname = "gdr decode_stream_kernel" if wl["dk"] == wl["dv"] == 128 else "gdr decode_kernel"
-    elif name == "mixer_t4k":
-        launch_ms = kern_ms
-        kname = "gdr chunk_tc_kernel<mixer> (tcgen05, fused prologue/epilogue)"
-    elif name == "bwd_t4k":
-        # one step = the whole backward (states, state gradient, per-chunk gradients, and the
-        # CUDA-core kernel for strong-decay spans, none here), the unit of the roofline
-        launch_ms = kern_ms
-        kname = ("gdr chunk_tc_kernel (checkpoints) + chunk_tc_kernel (state gradient) + bwd_tc_kernel"
-                 " + bwd_chunk_kernel (backward, 4 launches, tcgen05)")
-    else:
-        # one step = the whole forward; with a sequence split it is three launches
-        # (state pass, combine, output pass) and the step is the unit of the roofline
-        launch_ms = kern_ms
-        kname = kernel_name(wl, mode) if nseg <= 1 else \
-            f"gdr chunk_tc_kernel x2 + split_combine_kernel (sequence split, {nseg} segments)"
-    achieved = bytes_per_launch / (launch_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-            "frac": achieved / hbm, "traffic": traffic_for(name, kname), "peak_source": f"{peak_src} hbm_gbs",
-            "kernel": kname}
-    if name not in ("decode", "mixer_t4k"):
-        fl = bwd_flops(wl) if name == "bwd_t4k" else chunk_flops(wl)
-        roof["tensor_context"] = {"flops_per_launch": fl,
-                                  "achieved_tflops": fl / (launch_ms * 1e-3) / 1e12,
-                                  "peak_tflops": tf_burst,
-                                  "frac": fl / (launch_ms * 1e-3) / 1e12 / tf_burst}
     line = {"metric": metric_name(name), "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if (name in ("decode", "mixer_t4k", "bwd_t4k") or wl.dtype == "bf16") else "f32",
             "data": "synthetic", "config": config_of(name, world), "roofline": roof,
-            "clocks": clk.summary(), "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk, "gpu_launches": launches_per_step * args.steps,
             "e2e": e2e, "wall_total_ms": total_ms}
     if name != "decode":
         # the same throughput for a whole layer of H heads: B*T / step time
         line["layer_tokens_per_s"] = value / (wl["H"] if name == "mixer_t4k" else wl.H)
+    if secondary is not None:
+        line["secondary"] = secondary
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(name, target_cpu_s=args.ref_cpu_s)
     print(json.dumps(line), flush=True)
@@ -680,6 +715,9 @@ def main():
                              "gdn2_t4k_bonly", "gdn2_t4k_wonly", "mixer_t4k", "bwd_t4k"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads timed beside the headline on a one-GPU run")
+    ap.add_argument("--secondary-steps", type=int, default=10)
     ap.add_argument("--ref-cpu-s", type=float, default=15.0)
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="decode steps per bench step (default: the workload's 1000); fewer keep an "

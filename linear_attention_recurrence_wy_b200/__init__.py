@@ -234,19 +234,66 @@ def chunk_fwd_split(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, ns
     return o, S_T
 
 
+def _pipelined_host_call(inputs, outputs, groups, run, device):
+    """Run `run(lo, hi, dev_inputs, dev_outputs)` on groups [lo, hi) of the leading unit axis
+    of host tensors, overlapping the host-to-device copies of group i+1 (a copy stream), the
+    library call on group i (the current stream) and the device-to-host copies of group i-1
+    (a second copy stream).  inputs / outputs: lists of host tensors (None allowed) viewed
+    with the unit axis first; returns nothing (the outputs are filled).  The current stream
+    waits for every copy before this returns, so work queued after it sees the results."""
+    dev = torch.device(device)
+    cur = torch.cuda.current_stream(dev)
+    d_in = [None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev) for t in inputs]
+    d_out = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in outputs]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_in.wait_stream(cur)
+    s_out.wait_stream(cur)
+    n = inputs[0].shape[0]
+    bounds = [(n * i // groups, n * (i + 1) // groups) for i in range(groups)]
+    for lo, hi in bounds:
+        if hi == lo:
+            continue
+        with torch.cuda.stream(s_in):
+            for h, d in zip(inputs, d_in):
+                if h is not None:
+                    d[lo:hi].copy_(h[lo:hi], non_blocking=True)
+        cur.wait_stream(s_in)
+        run(lo, hi, d_in, d_out)
+        s_out.wait_stream(cur)
+        with torch.cuda.stream(s_out):
+            for h, d in zip(outputs, d_out):
+                h[lo:hi].copy_(d[lo:hi], non_blocking=True)
+    cur.wait_stream(s_out)
+
+
 def chunk_fwd_host(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, device="cuda",
-                   out=None):
-    """End-to-end call on host tensors: copies the inputs (pinned host memory is
-    copied asynchronously) to the device, runs chunk_fwd and copies o and S_T back
-    into host tensors (`out` = (o_host, S_T_host) to reuse pinned buffers)."""
-    nb = q.is_pinned()
-    to = lambda t: None if t is None else t.to(device, non_blocking=nb)
-    o_d, S_d = chunk_fwd(to(q), to(k), to(v), to(g), to(b), to(w), to(S0), mode=mode, chunk=chunk)
+                   out=None, groups=None):
+    """End-to-end call on host tensors: copies the inputs to the device, runs chunk_fwd and
+    copies o and S_T back into host tensors (`out` = (o_host, S_T_host) to reuse pinned
+    buffers).  With pinned inputs the (sequence, head) pairs are processed in `groups`
+    (default: up to 8) contiguous groups whose copies in both directions overlap the
+    computation of the neighbouring groups."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
     if out is None:
-        out = (torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True),
-               torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True))
-    out[0].copy_(o_d, non_blocking=True)
-    out[1].copy_(S_d, non_blocking=True)
+        out = (torch.empty(B, H, T, dv, dtype=q.dtype, pin_memory=True),
+               torch.empty(B, H, dk, dv, dtype=torch.float32, pin_memory=True))
+    units = B * H
+    ng = min(units, 8) if groups is None else max(1, min(int(groups), units))
+    if not q.is_pinned() or ng <= 1:
+        to = lambda t: None if t is None else t.to(device, non_blocking=q.is_pinned())
+        o_d, S_d = chunk_fwd(to(q), to(k), to(v), to(g), to(b), to(w), to(S0), mode=mode, chunk=chunk)
+        out[0].copy_(o_d, non_blocking=True)
+        out[1].copy_(S_d, non_blocking=True)
+        return out
+    flat = lambda t: None if t is None else t.reshape(units, *t.shape[2:])
+    ins = [flat(t) for t in (q, k, v, g, b, w, S0)]
+    outs = [flat(out[0]), flat(out[1])]
+
+    def run(lo, hi, d, dout):
+        one = lambda t: None if t is None else t[lo:hi].unsqueeze(0)
+        chunk_fwd(*(one(t) for t in d), mode=mode, chunk=chunk, o=one(dout[0]), S_T=one(dout[1]))
+    _pipelined_host_call(ins, outs, ng, run, device)
     return out
 
 
@@ -292,18 +339,33 @@ def mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0=None, *, mode="gdn2", layo
 
 
 def mixer_fwd_host(q, k, v, xg, xb, xw, z, norm_weight, S0=None, *, mode="gdn2", layout="bhtd",
-                   b_range=1.0, eps=1e-5, device="cuda", out=None):
-    """mixer_fwd end to end from host tensors (pinned host memory is copied
-    asynchronously); y and S_T come back into host tensors (`out` to reuse them)."""
-    nb = q.is_pinned()
-    to = lambda t: None if t is None else t.to(device, non_blocking=nb)
-    y_d, S_d = mixer_fwd(to(q), to(k), to(v), to(xg), to(xb), to(xw), to(z), to(norm_weight), to(S0),
-                         mode=mode, layout=layout, b_range=b_range, eps=eps)
+                   b_range=1.0, eps=1e-5, device="cuda", out=None, groups=None):
+    """mixer_fwd end to end from host tensors; y and S_T come back into host tensors (`out`
+    to reuse them).  With pinned inputs the sequences are processed in `groups` (default: up
+    to 8) contiguous groups whose copies overlap the computation of the neighbouring
+    groups."""
+    B = q.shape[0]
     if out is None:
-        out = (torch.empty(y_d.shape, dtype=y_d.dtype, pin_memory=True),
-               torch.empty(S_d.shape, dtype=S_d.dtype, pin_memory=True))
-    out[0].copy_(y_d, non_blocking=True)
-    out[1].copy_(S_d, non_blocking=True)
+        dv = v.shape[-1]
+        H = q.shape[1] if layout == "bhtd" else q.shape[2]
+        out = (torch.empty(v.shape[:-1] + (dv,), dtype=q.dtype, pin_memory=True),
+               torch.empty(B, H, q.shape[-1], dv, dtype=torch.float32, pin_memory=True))
+    ng = min(B, 8) if groups is None else max(1, min(int(groups), B))
+    if not q.is_pinned() or ng <= 1:
+        to = lambda t: None if t is None else t.to(device, non_blocking=q.is_pinned())
+        y_d, S_d = mixer_fwd(to(q), to(k), to(v), to(xg), to(xb), to(xw), to(z), to(norm_weight), to(S0),
+                             mode=mode, layout=layout, b_range=b_range, eps=eps)
+        out[0].copy_(y_d, non_blocking=True)
+        out[1].copy_(S_d, non_blocking=True)
+        return out
+    nw = norm_weight.to(device, non_blocking=True)
+
+    def run(lo, hi, d, dout):
+        sl = lambda t: None if t is None else t[lo:hi]
+        q_, k_, v_, xg_, xb_, xw_, z_, S0_ = (sl(t) for t in d)
+        mixer_fwd(q_, k_, v_, xg_, xb_, xw_, z_, nw, S0_, mode=mode, layout=layout, b_range=b_range, eps=eps,
+                  y=sl(dout[0]), S_T=sl(dout[1]))
+    _pipelined_host_call([q, k, v, xg, xb, xw, z, S0], list(out), ng, run, device)
     return out
 
 

@@ -123,3 +123,15 @@ def test_mixer_workload_full_size(cuda_ok):
         y_np = np64(y)
     assert_close("mixer_t4k y", y_np, y_ref, "bf16")
     assert_close("mixer_t4k S_T", np64(ST), S_ref, "bf16")
+
+
+@pytest.mark.parametrize("layout", ["bhtd", "bthd"])
+def test_host_call_pipelined_in_groups_equals_device_call(cuda_ok, layout):
+    d = workload.make_mixer_inputs(3, 2, 150, 128, 128, mode="gdn2", layout=layout, seed=9, s0_std=0.05)
+    pin = lambda t: None if t is None else t.pin_memory()
+    y_h, S_h = gdr.mixer_fwd_host(pin(d["q"]), pin(d["k"]), pin(d["v"]), pin(d["xg"]), pin(d["xb"]),
+                                  pin(d["xw"]), pin(d["z"]), d["weight"], pin(d["S0"]), mode="gdn2",
+                                  layout=layout, eps=EPS, groups=2)
+    torch.cuda.synchronize()
+    y_d, S_d = run_gpu(d)
+    assert torch.equal(y_h, y_d.cpu()) and torch.equal(S_h, S_d.cpu())
