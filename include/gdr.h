@@ -173,6 +173,49 @@ gdr_status_t gdr_chunk_fwd_split_noalloc(const void *q, const void *k, const voi
                                          gdr_dtype_t dtype, int nseg, void *stream);
 
 /*
+ * Sequence split across GPUs (one state hand-off per segment).
+ *
+ * Only the state crosses chunk borders (Gated DeltaNet-2 Review §3-2.5, "Chunkwise WY
+ * training"), and the recurrence is affine in it: over a segment of the sequence,
+ * S_end = M S_start + S_local (Gated DeltaNet-2 Q&A page, Q3 update equation).  R holders
+ * (ranks, one per GPU) each take one contiguous range of the tokens of every
+ * sequence-head, in order.  Holder r computes its segment's maps, the holders exchange
+ * them (one all-gather, done by the caller's communication library), each chains them to
+ * its own start state and runs gdr_chunk_fwd on its range from that state: it owns o of
+ * its range, and the last holder's end state is S_T.  The Python binding's
+ * chunk_fwd_seqpar does all of this over torch.distributed.
+ *
+ * gdr_chunk_fwd_segment_maps -- the maps of one segment held on its own.
+ *   q .. w        the segment's tokens, laid out as for gdr_chunk_fwd with T = its length
+ *   S0            start state of the segment if known (holder 0: the sequence's S0), else
+ *                 NULL: S_local is then the end state reached from a zero state
+ *   S_local       [B,H,dk,dv] fp32 (written): the end state reached from S0
+ *   M             [B,H,dk,dk] fp32 (written) or NULL: the segment's transition map, the
+ *                 end state reached from the identity with the write term (w.v) dropped;
+ *                 holders 1 .. R-2 need it, holders 0 and R-1 do not
+ * bf16 with dk = dv = 128 and chunk 64 only (else GDR_ERR_DIM); T >= 1.  Asynchronous on
+ * `stream`; the caller owns every buffer.
+ */
+gdr_status_t gdr_chunk_fwd_segment_maps(const void *q, const void *k, const void *v, const float *g_log,
+                                        const void *b, const void *w, const float *S0, float *S_local,
+                                        float *M, int B, int H, int T, int dk, int dv, int chunk,
+                                        gdr_mode_t mode, gdr_dtype_t dtype, void *stream);
+
+/*
+ * gdr_chain_segment_states -- the start state of holder r from every holder's maps.
+ *   M_all         [R][B,H,dk,dk] fp32: the gathered transition maps (entries of holders 0
+ *                 and R-1 are not read; may be NULL when r < 2)
+ *   S_local_all   [R][B,H,dk,dv] fp32: the gathered end states, holder 0's from S0 (may be
+ *                 NULL when r = 0)
+ *   S0            [B,H,dk,dv] fp32 or NULL (zero): the sequence's start state, read when r = 0
+ *   S_start       [B,H,dk,dv] fp32 (written)
+ * r = 0: S_start = S0; r >= 1: S = S_local_all[0], then S <- M_all[i] S + S_local_all[i] for
+ * i = 1 .. r-1, in fp32 on the GPU.  dk = dv = 128; 0 <= r < R.
+ */
+gdr_status_t gdr_chain_segment_states(const float *M_all, const float *S_local_all, const float *S0,
+                                      float *S_start, int R, int r, int B, int H, int dk, int dv, void *stream);
+
+/*
  * gdr_decode_step -- one-token recurrent update for N sequences x H heads.
  *
  * The recurrent form used for constant-memory decoding (Gated DeltaNet-2 Q&A page,

@@ -8,9 +8,11 @@ PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raise
 Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
 gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
 gdr_mixer_fwd, gdr_chunk_bwd, gdr_chunk_bwd_workspace, gdr_decode_step,
-gdr_last_device_error, gdr_status_string, gdr_test_set_first_wait_limit.
+gdr_chunk_fwd_segment_maps, gdr_chain_segment_states, gdr_last_device_error,
+gdr_status_string, gdr_test_set_first_wait_limit.
 Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
-chunk_bwd, decode_step.
+chunk_bwd, decode_step, segment_maps, chain_segment_states; the sequence split across GPUs
+(torch.distributed): seqpar.chunk_fwd_seqpar.
 """
 from __future__ import annotations
 
@@ -62,6 +64,10 @@ def lib():
         L.gdr_decode_step.restype = ci
         L.gdr_last_device_error.argtypes = [vp]
         L.gdr_last_device_error.restype = ci
+        L.gdr_chunk_fwd_segment_maps.argtypes = [vp] * 9 + [ci] * 8 + [vp]
+        L.gdr_chunk_fwd_segment_maps.restype = ci
+        L.gdr_chain_segment_states.argtypes = [vp] * 4 + [ci] * 6 + [vp]
+        L.gdr_chain_segment_states.restype = ci
         L.gdr_test_set_first_wait_limit.argtypes = [ctypes.c_uint]
         L.gdr_test_set_first_wait_limit.restype = None
         L.gdr_status_string.argtypes = [ci]
@@ -118,6 +124,61 @@ def gdr_decode_step(q, k, v, g_log, b, w, S, o, N, H, dk, dv, mode, dtype, strea
 
 def gdr_last_device_error(stream=None):
     return lib().gdr_last_device_error(stream)
+
+
+def gdr_chunk_fwd_segment_maps(q, k, v, g_log, b, w, S0, S_local, M, B, H, T, dk, dv, chunk, mode, dtype,
+                               stream=None):
+    return lib().gdr_chunk_fwd_segment_maps(q, k, v, g_log, b, w, S0, S_local, M, B, H, T, dk, dv, chunk, mode,
+                                            dtype, stream)
+
+
+def gdr_chain_segment_states(M_all, S_local_all, S0, S_start, R, r, B, H, dk, dv, stream=None):
+    return lib().gdr_chain_segment_states(M_all, S_local_all, S0, S_start, R, r, B, H, dk, dv, stream)
+
+
+def segment_maps(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, want_M=False):
+    """Maps of one segment of the sequence held on its own (gdr_chunk_fwd_segment_maps):
+    returns (S_local, M) -- the end state reached from S0 (zero if None) and, when want_M,
+    the transition map [B,H,dk,dk] (else None).  bf16, dk = dv = 128, chunk 64."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    gshape, bshape, wshape = _gate_shapes(mode, (B, H, T), dk, dv)
+    for t, name, shape, tdt in ((q, "q", (B, H, T, dk), dt), (k, "k", (B, H, T, dk), dt),
+                                (v, "v", (B, H, T, dv), dt), (g, "g", gshape, torch.float32),
+                                (b, "b", bshape, dt)):
+        _check(t, name, shape, tdt, dev)
+    if wshape is not None:
+        _check(w, "w", wshape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    S_local = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    M = torch.empty(B, H, dk, dk, dtype=torch.float32, device=dev) if want_M else None
+    rc = gdr_chunk_fwd_segment_maps(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
+                                    _ptr(w) if wshape is not None else None, _ptr(S0), _ptr(S_local), _ptr(M),
+                                    B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_segment_maps")
+    return S_local, M
+
+
+def chain_segment_states(M_all, S_local_all, S0, r):
+    """Start state of holder r (gdr_chain_segment_states) from the gathered maps
+    M_all [R,B,H,dk,dk] (may be None when r < 2) and S_local_all [R,B,H,dk,dv]; S0 is read
+    when r = 0 (None: zero)."""
+    R, B, H, dk, dv = S_local_all.shape
+    dev = S_local_all.device
+    _check(S_local_all, "S_local_all", (R, B, H, dk, dv), torch.float32, dev)
+    if M_all is not None:
+        _check(M_all, "M_all", (R, B, H, dk, dk), torch.float32, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    S_start = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    rc = gdr_chain_segment_states(_ptr(M_all), _ptr(S_local_all), _ptr(S0), _ptr(S_start), R, r, B, H, dk, dv,
+                                  _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_chain_segment_states")
+    return S_start
 
 
 def gdr_test_set_first_wait_limit(polls: int) -> None:

@@ -280,10 +280,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
     // ---- this CTA's job: one sequence-head, one segment of it, one role ----
-    const int roles = a.pass ? max(1, 2 * a.nseg - 3) : a.nseg;
+    const bool maps = a.seg_maps != 0;                        // a whole segment's maps
+    const int roles = chunk_roles(a);
     const int bh = blockIdx.x / roles, role = blockIdx.x % roles;
-    const bool transfer = a.pass && role > a.nseg - 2;       // transition-matrix run
-    const int seg = transfer ? role - (a.nseg - 2) : role;
+    const bool transfer = maps ? role == 1 : (a.pass && role > a.nseg - 2);   // transition-matrix run
+    const int seg = maps ? 0 : transfer ? role - (a.nseg - 2) : role;
     const int t_begin = seg * a.seg_len;
     const int T = min(a.seg_len, a.T - t_begin);              // tokens of this segment
     const int mode = a.mode;
@@ -298,7 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
     const size_t sidx = ((size_t)bh * a.nseg + seg) * DK * DV;
     const float *S0p = nullptr;        // initial state (NULL: zero, unless the identity)
     float *STp = nullptr;              // end state destination (NULL: not written)
-    if (!a.pass) {
+    if (maps) {
+        S0p = (!transfer && a.S0) ? a.S0 + (size_t)bh * DK * DV : nullptr;
+        STp = (transfer ? a.ws_m : a.ws_send) + (size_t)bh * DK * DV;
+    } else if (!a.pass) {
         S0p = a.nseg == 1 ? (a.S0 ? a.S0 + (size_t)bh * DK * DV : nullptr) : a.ws_sstart + sidx;
         STp = seg == a.nseg - 1 ? (a.ST ? a.ST + (size_t)bh * DK * DV : nullptr) : nullptr;
     } else {
@@ -1220,8 +1224,7 @@ gdr_status_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
                             : encode_head_major(&tm.y, a.o, a.B, a.T, a.H, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2);
         if (!ok) return GDR_ERR_CUDA;
     }
-    const int roles = a.pass ? (2 * a.nseg - 3 > 1 ? 2 * a.nseg - 3 : 1) : a.nseg;
-    kern<<<(unsigned)(a.B * a.H * roles), kThreads, SMEM_BYTES, s>>>(a, tm);
+    kern<<<(unsigned)(a.B * a.H * chunk_roles(a)), kThreads, SMEM_BYTES, s>>>(a, tm);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -50,7 +50,21 @@ struct ChunkArgs {
     // expiry path runs while the WY group is merely still working.
     unsigned wait_limit = 1u << 24;
     unsigned first_wait_limit = 0;
+    // The maps of one whole segment held on its own (the sequence split across GPUs;
+    // tensor-core kernel, pass 1 semantics, no output): seg_maps != 0 writes the end state
+    // reached from S0 (NULL: zero) to ws_send[B*H][dk][dv] and, when want_m, the segment's
+    // transition map (the end state from the identity with the write term dropped) to
+    // ws_m[B*H][dk][dk].
+    int seg_maps = 0, want_m = 0;
 };
+
+// CTAs per sequence-head of a tensor-core forward launch: its roles (whole sequence, the
+// split's segments and transfer runs, or a segment's maps).
+__host__ __device__ inline int chunk_roles(const ChunkArgs &a) {
+    if (a.seg_maps) return a.want_m ? 2 : 1;
+    if (a.pass) return 2 * a.nseg - 3 > 1 ? 2 * a.nseg - 3 : 1;
+    return a.nseg;
+}
 
 struct DecodeArgs {
     const void *q, *k, *v, *b, *w;
@@ -122,6 +136,12 @@ unsigned long long bwd_states_bytes(int B, int H, int T, int dk, int dv);
 unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
 gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s);
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);
+// Start state of segment r of a sequence split across R holders (ranks), from every
+// segment's maps gathered as M_all[R][BH][dk][dk] and S_all[R][BH][dk][dv] (fp32; the end
+// state of segment 0 is taken from S0 already):  r = 0: S0 (zero if NULL);  r >= 1:
+// S = S_all[0];  S <- M_all[i] S + S_all[i] for i = 1 .. r-1.  dk = dv = 128.
+gdr_status_t launch_segment_chain(const float *M_all, const float *S_all, const float *S0, float *S_start, int R,
+                                  int r, int BH, cudaStream_t s);
 // Segments the sequence split actually runs for a request of nseg (segments of whole
 // chunks, none empty); 1 for T <= 0.
 int split_effective_segments(int T, int chunk, int nseg);

@@ -176,6 +176,40 @@ extern "C" gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const 
     return launch_chunk_tc(a, s);
 }
 
+extern "C" gdr_status_t gdr_chunk_fwd_segment_maps(const void *q, const void *k, const void *v,
+                                                   const float *g_log, const void *b, const void *w,
+                                                   const float *S0, float *S_local, float *M, int B, int H,
+                                                   int T, int dk, int dv, int chunk, gdr_mode_t mode,
+                                                   gdr_dtype_t dtype, void *stream) {
+    gdr_status_t st = check_chunk(q, k, v, g_log, b, w, S0, S_local, S_local, B, H, T, dk, dv, chunk, mode, dtype);
+    if (st != GDR_OK) return st;
+    if (!S_local) return GDR_ERR_NULL;
+    if (!aligned16(M)) return GDR_ERR_ALIGN;
+    if (T < 1) return GDR_ERR_DIM;
+    ChunkArgs a = make_args(q, k, v, g_log, b, w, S0, nullptr, nullptr, B, H, T, dk, dv, chunk, mode, dtype);
+    if (!chunk_tc_supported(a)) return GDR_ERR_DIM;
+    if ((int64_t)B * H * 2 > INT32_MAX) return GDR_ERR_DIM;
+    if ((int64_t)B * H == 0) return GDR_OK;
+    a.pass = 1;   // no output
+    a.seg_maps = 1;
+    a.want_m = M != nullptr;
+    a.seg_len = T;
+    a.ws_send = S_local;
+    a.ws_m = M;
+    return launch_chunk_tc(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" gdr_status_t gdr_chain_segment_states(const float *M_all, const float *S_local_all, const float *S0,
+                                                 float *S_start, int R, int r, int B, int H, int dk, int dv,
+                                                 void *stream) {
+    if (B < 0 || H < 0 || R < 1 || r < 0 || r >= R || dk != 128 || dv != 128) return GDR_ERR_DIM;
+    if ((int64_t)B * H * (dv / 16) > INT32_MAX) return GDR_ERR_DIM;
+    if (!S_start || (r >= 1 && !S_local_all) || (r >= 2 && !M_all)) return GDR_ERR_NULL;
+    if (!aligned16(M_all) || !aligned16(S_local_all) || !aligned16(S0) || !aligned16(S_start)) return GDR_ERR_ALIGN;
+    if ((int64_t)B * H == 0) return GDR_OK;
+    return launch_segment_chain(M_all, S_local_all, S0, S_start, R, r, B * H, reinterpret_cast<cudaStream_t>(stream));
+}
+
 extern "C" gdr_status_t gdr_mixer_fwd(const void *q, const void *k, const void *v, const float *xg,
                                       const void *xb, const void *xw, const void *z,
                                       const float *norm_weight, const float *S0, void *y,
