@@ -54,7 +54,8 @@ typedef enum {
     GDR_ERR_CUDA = -6,     /* a CUDA launch or attribute call failed */
     GDR_ERR_TIMEOUT = -7,  /* a bounded device-side wait gave up (tensor-core path) */
     GDR_ERR_WORKSPACE = -8,/* workspace missing, misaligned or smaller than required */
-    GDR_ERR_VALUE = -9     /* a scalar argument is out of range (eps, b_range, layout) */
+    GDR_ERR_VALUE = -9,    /* a scalar argument is out of range (eps, b_range, layout) */
+    GDR_ERR_BOUNDS = -10   /* debug build only: an in-kernel bounds check failed */
 } gdr_status_t;
 
 typedef enum {
@@ -315,6 +316,21 @@ gdr_status_t gdr_chunk_bwd(const void *q, const void *k, const void *v, const fl
  * its tensor memory), GDR_ERR_CUDA if the stream reports a CUDA error, else GDR_OK.
  */
 gdr_status_t gdr_last_device_error(void *stream);
+
+/*
+ * The debug build (libgdr_debug.so, compiled with -DGDR_DEBUG; the pages have no
+ * counterpart).  Its kernels check that every bulk copy's source range, every clamped tail
+ * load, every output row and every workspace or checkpoint slot they touch lies inside the
+ * extents the call's arguments imply; a failed check skips the access and records its site
+ * (no trap), gdr_last_device_error() then returns GDR_ERR_BOUNDS and
+ * gdr_debug_bounds_site() the site (1xx tensor-core forward, 2xx decode, 3xx tensor-core
+ * backward, 4xx CUDA-core backward, 5xx split chaining, 6xx CUDA-core forward).  It stands
+ * in for a memory sanitizer, which is not available; results are identical otherwise.
+ * gdr_debug_build() is 1 in that library and 0 in the release build, where the bounds
+ * site is always 0.
+ */
+int gdr_debug_build(void);
+int gdr_debug_bounds_site(void);
 
 /*
  * gdr_test_set_first_wait_limit -- test hook for the bounded-wait expiry path.  The pages

@@ -9,7 +9,7 @@ Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
 gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
 gdr_mixer_fwd, gdr_chunk_bwd, gdr_chunk_bwd_workspace, gdr_decode_step,
 gdr_chunk_fwd_segment_maps, gdr_chain_segment_states, gdr_last_device_error,
-gdr_status_string, gdr_test_set_first_wait_limit.
+gdr_status_string, gdr_test_set_first_wait_limit, gdr_debug_build, gdr_debug_bounds_site.
 Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
 chunk_bwd, decode_step, segment_maps, chain_segment_states; the sequence split across GPUs
 (torch.distributed): seqpar.chunk_fwd_seqpar.
@@ -22,7 +22,8 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libgdr.so")
+# GDR_DEBUG=1 loads the debug build (in-kernel bounds checks, build.py --debug) instead
+LIB_PATH = os.path.join(_PKG, "libgdr_debug.so" if os.environ.get("GDR_DEBUG") == "1" else "libgdr.so")
 MODES = {"gdn2": 0, "kda": 1, "gdn": 2, "bonly": 3, "wonly": 4}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 LAYOUTS = {"bhtd": 0, "bthd": 1}
@@ -36,12 +37,13 @@ class GdrError(RuntimeError):
 
 
 def lib():
-    """Load libgdr.so (built in-tree by build.py); raises if it is absent."""
+    """Load libgdr.so (built in-tree by build.py; libgdr_debug.so when GDR_DEBUG=1); raises if
+    it is absent."""
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libgdr.so not built: run python -m linear_attention_recurrence_wy_b200.build "
-                              f"(expected at {LIB_PATH})")
+            raise ImportError(f"{os.path.basename(LIB_PATH)} not built: run python -m "
+                              f"linear_attention_recurrence_wy_b200.build (expected at {LIB_PATH})")
         L = ctypes.CDLL(LIB_PATH)
         vp, ci = ctypes.c_void_p, ctypes.c_int
         L.gdr_chunk_fwd.argtypes = [vp] * 9 + [ci] * 8 + [vp]
@@ -68,6 +70,10 @@ def lib():
         L.gdr_chunk_fwd_segment_maps.restype = ci
         L.gdr_chain_segment_states.argtypes = [vp] * 4 + [ci] * 6 + [vp]
         L.gdr_chain_segment_states.restype = ci
+        L.gdr_debug_build.argtypes = []
+        L.gdr_debug_build.restype = ci
+        L.gdr_debug_bounds_site.argtypes = []
+        L.gdr_debug_bounds_site.restype = ci
         L.gdr_test_set_first_wait_limit.argtypes = [ctypes.c_uint]
         L.gdr_test_set_first_wait_limit.restype = None
         L.gdr_status_string.argtypes = [ci]
@@ -179,6 +185,14 @@ def chain_segment_states(M_all, S_local_all, S0, r):
     if rc != 0:
         raise GdrError(rc, "gdr_chain_segment_states")
     return S_start
+
+
+def gdr_debug_build() -> int:
+    return lib().gdr_debug_build()
+
+
+def gdr_debug_bounds_site() -> int:
+    return lib().gdr_debug_bounds_site()
 
 
 def gdr_test_set_first_wait_limit(polls: int) -> None:

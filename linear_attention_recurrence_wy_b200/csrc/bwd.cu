@@ -39,6 +39,7 @@
 
 #include "bwd_tc.cuh"
 #include "chunk_tc.cuh"
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace gdr {
@@ -178,6 +179,8 @@ __global__ void __launch_bounds__(kThreadsS, 1) bwd_dstate_kernel(BwdArgs a) {
     float *dR = dE + C * VS;         // [C][VS]
     const int nc = (T + C - 1) / C;
     const size_t tok0 = (size_t)bh * T;
+    // debug build: this job's sequence-head and value slice exist (uniform: return before any barrier)
+    if (!GDR_IN_BOUNDS(bh < a.B * a.H && v0 + VS <= dv, 401)) return;
 
     for (int idx = tid; idx < dk * VS; idx += nth) {
         const int d = idx / VS, j = idx - d * VS;
@@ -277,9 +280,13 @@ __global__ void __launch_bounds__(kThreadsC, 1) bwd_chunk_kernel(BwdArgs a) {
     const int tid = threadIdx.x, nth = blockDim.x;
     // this CTA's span, or with tc_list every gridDim.x-th listed span
     const int njobs = a.tc_list ? a.tc_list[0] : (int)gridDim.x;
+  // debug build: the span list holds no more entries than there are spans
+  if (!GDR_IN_BOUNDS(njobs <= a.B * a.H * nspan, 403)) return;
   for (int job = blockIdx.x; job < njobs; job += gridDim.x) {
     const int blk = a.tc_list ? a.tc_list[1 + job] : job;
     const int bh = blk / nspan, span = blk - bh * nspan;
+    // debug build: a valid span (the same for every thread of the CTA: skipped together)
+    if (!GDR_IN_BOUNDS(blk >= 0 && blk < a.B * a.H * nspan, 402)) continue;
     __syncthreads();   // the previous span's shared-memory reads are done
     if (a.mid_grad && 2 * span + 1 < nc) {
         // The state gradient at the span's middle, from its end by one step of the reverse
@@ -760,4 +767,8 @@ gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s) {
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
+}  // namespace gdr
+
+namespace gdr {
+GDR_BOUNDS_READER(bwd_bounds_site)
 }  // namespace gdr

@@ -36,6 +36,7 @@
 // Every wait on an mbarrier is bounded; on expiry the CTA records the failure in
 // g_bwd_tc_error, waits (bounded) for its own tensor-core work and copies, frees its TMEM
 // and returns.
+#include "bounds.cuh"
 #include "bwd_tc.cuh"
 #include "tc_util.cuh"
 #include "tri_inverse.cuh"
@@ -137,6 +138,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
     const int nslot = (T + kBwdChunk - 1) / kBwdChunk;
     const float *Sg = a.ws_states + ((size_t)bh * nslot + 2 * c) * DK * DV;
     const float *dSg = a.ws_dstates + ((size_t)bh * nslot + min(2 * c + 1, nslot - 1)) * DK * DV;
+    // debug build: this chunk and its two state slots lie inside what the arguments imply
+    // (a uniform condition: a failing CTA returns before its first barrier)
+    if (!GDR_IN_BOUNDS(bh < a.B * a.H && n >= 1 && t0 + n <= T && 2 * c < nslot, 301)) return;
 
     const __nv_bfloat16 *Q = (const __nv_bfloat16 *)a.q, *K = (const __nv_bfloat16 *)a.k;
     const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
@@ -307,7 +311,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         }
         __syncthreads();
         if (sFlag[0]) {
-            if (tid == 0) a.tc_list[1 + atomicAdd(a.tc_list, 1)] = blockIdx.x;
+            if (tid == 0) {
+                const int k = atomicAdd(a.tc_list, 1);
+                // the list holds one entry per 64-token span of every sequence-head
+                if (GDR_IN_BOUNDS(k < a.B * a.H * nchunk, 302)) a.tc_list[1 + k] = blockIdx.x;
+            }
             break;
         }
         // ---- 3. operands: Kh, Qg, Kb (thread (tg, cg): tokens 4 tg .. + 3, channels
@@ -720,4 +728,8 @@ cudaError_t bwd_tc_read_and_clear_error(int *err) {
     return cudaMemcpyToSymbol(g_bwd_tc_error, &zero, sizeof(int));
 }
 
+}  // namespace gdr
+
+namespace gdr {
+GDR_BOUNDS_READER(bwd_tc_bounds_site)
 }  // namespace gdr

@@ -16,6 +16,7 @@
 // for a forgetting decay, so no factor can overflow however strong the decay is.
 // Everything is fp32 FFMA; this kernel carries the fp32 path and every shape the
 // tensor-core kernel does not take.
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace gdr {
@@ -36,6 +37,9 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkArgs a) {
     const int v0 = blockIdx.y * VS;
     const int tid = threadIdx.x;
     const int nth = blockDim.x;
+    // debug build: this job's sequence-head and value slice exist (uniform: the barriers below
+    // are reached by every thread or by none)
+    if (!GDR_IN_BOUNDS(bh < a.B * a.H && v0 + VS <= dv, 601)) return;
 
     extern __shared__ float sm[];
     float *kk = sm;               // [C][dk]  k, later k . exp(gamma_C - gamma)
@@ -225,4 +229,8 @@ gdr_status_t launch_state_copy(const ChunkArgs &a, cudaStream_t s) {
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
+}  // namespace gdr
+
+namespace gdr {
+GDR_BOUNDS_READER(simt_bounds_site)
 }  // namespace gdr

@@ -57,6 +57,7 @@
 
 #include <mutex>
 
+#include "bounds.cuh"
 #include "chunk_tc.cuh"
 #include "tc_util.cuh"
 #include "tri_inverse.cuh"
@@ -310,6 +311,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         STp = transfer ? a.ws_m + sidx : a.ws_send + sidx;
     }
     const bool write_o = !a.pass && !kStates && !kReverse;
+    // debug build: this job's rows and state slots lie inside what the arguments imply (a
+    // uniform condition: a failing CTA returns before its first barrier)
+    const size_t rows_total = (size_t)a.B * a.H * a.T;
+    (void)rows_total;   // read by the debug build's checks only
+    if (!GDR_IN_BOUNDS(bh < a.B * a.H && t_begin >= 0 && T >= 1 && tok0 + (size_t)(T - 1) * ts < rows_total &&
+                           (maps || a.nseg == 1 || sidx + (size_t)DK * DV <= (size_t)a.B * a.H * a.nseg * DK * DV),
+                       101))
+        return;
 
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
@@ -437,6 +446,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             const int t0 = dch(c) * C, n = min(C, T - t0);
             const size_t e = (tok0 + t0) * DK;
             const uint32_t row16 = (uint32_t)n * DK * 2;
+            // debug build: the chunk's rows lie inside this head (the copies then stay in the tensors)
+            if (!GDR_IN_BOUNDS(n >= 1 && t0 >= 0 && t_begin + t0 + n <= a.T && tok0 + t0 + n <= rows_total, 102))
+                return;
             fence_async_smem();
             if (warp == 4) {
                 uint32_t bytes = 2 * row16;
@@ -735,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
             const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
             const float *egc = sEGC + (c & 3) * 128;
-            if (kStates) {
+            if (kStates && GDR_IN_BOUNDS(2 * c < (a.T + 31) / 32 && bh < a.B * a.H, 105)) {
                 // checkpoint: S_c (S^T columns [64 half, +64) of this lane), before this
                 // chunk's update, as bf16 [dk][dv] at the start of the slot; coalesced over
                 // the value channels (lanes)
@@ -755,8 +767,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             float wvt[32];
             uint32_t zp[16];   // mixer: the output gate z of the same lane and tokens, bf16 pairs
             {
-                const int last = transfer ? -1 : min(31, n - 1 - j0);   // last token column in range
+                int last = transfer ? -1 : min(31, n - 1 - j0);   // last token column in range
                 const size_t row = tok0 + (size_t)(t0 + j0) * ts;
+                // debug build: the rows read (v, w, z) lie inside the segment and the tensors
+                if (!GDR_IN_BOUNDS(last < 0 || (t0 + j0 + last < T && row + (size_t)last * ts < rows_total), 103))
+                    last = -1;
                 const __nv_bfloat16 *vp = V + row * DV + v;
                 const __nv_bfloat16 *wp = vec_w ? Wg + row * DV + v : Wsc + row;
                 const size_t ws = vec_w ? vs : (size_t)ts;
@@ -884,7 +899,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             float xo[32];
             tmem_ld32(tmem + lane_base + TM_XO + 64 + j0, xo);
             tmem_wait_ld();
-            if (!kMixer && write_o) {
+            if (!kMixer && write_o &&
+                GDR_IN_BOUNDS(n - j0 <= 0 || tok0 + (size_t)(t0 + n - 1) * ts < rows_total, 104)) {
                 __nv_bfloat16 *op = O + (tok0 + (size_t)(t0 + j0) * ts) * DV + v;
                 const int lim = n - j0;
 #pragma unroll
@@ -980,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
             const uint32_t kb_tile = sbase + OFF_KB + pb * 16384;
             const uint32_t p_tile = sbase + OFF_P + pb * 8192, t_tile = sbase + OFF_T + pb * 8192;
             const float *egc = sEGC + (c & 3) * 128;
-            {
+            if (GDR_IN_BOUNDS(2 * cd < (T + 31) / 32 && bh < a.B * a.H, 106)) {
                 const int nslot = (T + 31) / 32;
                 __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(
                                          a.chunk_states + ((size_t)bh * nslot + min(2 * cd + 1, nslot - 1)) * DK * DV) + v;
@@ -994,8 +1010,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
                 }
             }
             {   // dO^T of this lane and token columns -> bf16 in TMEM; tokens past the end give zero
-                const int last = min(31, n - 1 - j0);
+                int last = min(31, n - 1 - j0);
                 const __nv_bfloat16 *op = reinterpret_cast<const __nv_bfloat16 *>(a.dO) + (tok0 + t0 + j0) * DV + v;
+                if (!GDR_IN_BOUNDS(last < 0 || (t0 + j0 + last < T && tok0 + t0 + j0 + last < rows_total), 107))
+                    last = -1;
                 float x[32];
                 if (last >= 0) {   // rows past the end re-read the last row and give zero
 #pragma unroll
@@ -1227,6 +1245,8 @@ gdr_status_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t s) {
     kern<<<(unsigned)(a.B * a.H * chunk_roles(a)), kThreads, SMEM_BYTES, s>>>(a, tm);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
+
+GDR_BOUNDS_READER(chunk_tc_bounds_site)
 
 cudaError_t chunk_tc_read_and_clear_error(int *err) {
     cudaError_t e = cudaMemcpyFromSymbol(err, g_tc_error, sizeof(int));

@@ -136,6 +136,14 @@ unsigned long long bwd_states_bytes(int B, int H, int T, int dk, int dv);
 unsigned long long bwd_workspace_bytes(int B, int H, int T, int dk, int dv);
 gdr_status_t launch_bwd(const BwdArgs &a, cudaStream_t s);
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s);
+// Debug build (GDR_DEBUG): the first failed bounds-check site of each translation unit's
+// kernels, read and cleared (0: none; always 0 in the release build).  See bounds.cuh.
+int chunk_tc_bounds_site();
+int bwd_tc_bounds_site();
+int bwd_bounds_site();
+int simt_bounds_site();
+int decode_bounds_site();
+int split_bounds_site();
 // Start state of segment r of a sequence split across R holders (ranks), from every
 // segment's maps gathered as M_all[R][BH][dk][dk] and S_all[R][BH][dk][dv] (fp32; the end
 // state of segment 0 is taken from S0 already):  r = 0: S0 (zero if NULL);  r >= 1:

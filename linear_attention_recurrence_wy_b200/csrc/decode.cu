@@ -21,6 +21,7 @@
 // Other shapes (decode_kernel): one CTA of 256 threads per head; each thread holds
 // float4 column groups of several rows, the loads are 16-byte coalesced and all issued
 // before any arithmetic.
+#include "bounds.cuh"
 #include "common.cuh"
 #include "tc_util.cuh"
 
@@ -226,6 +227,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
     };
     auto issue_load = [&](int i) {   // state of iteration i -> buffer i % kBufs (thread 0)
         const int h = blockIdx.x + i * G;
+        if (!GDR_IN_BOUNDS(h < NH, 201)) return;   // debug build: a head of this call
         const uint32_t bar = bar_full + 8 * (i % kBufs);
         tc::mbar_arrive_expect_tx(bar, kStateBytes);
         tc::bulk_g2s(sbase + SO_BUF + (i % kBufs) * kStateBytes, a.S + (size_t)h * SD * SD, kStateBytes, bar);
@@ -330,7 +332,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) decode_stream_kernel(Decode
         if (tid == kStreamThreads - 1 && i + 1 < iters) put_scalars(i + 1);
         tc::fence_async_smem();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && GDR_IN_BOUNDS(h < NH, 202)) {
             bulk_s2g(a.S + (size_t)h * SD * SD, sbase + SO_BUF + (i % kBufs) * kStateBytes, kStateBytes);
             bulk_commit();
             if (loads < iters) {
@@ -400,4 +402,8 @@ cudaError_t decode_read_and_clear_error(int *err) {
     const int zero = 0;
     return cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(int));
 }
+}  // namespace gdr
+
+namespace gdr {
+GDR_BOUNDS_READER(decode_bounds_site)
 }  // namespace gdr

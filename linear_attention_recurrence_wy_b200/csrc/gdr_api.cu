@@ -296,9 +296,39 @@ extern "C" gdr_status_t gdr_decode_step(const void *q, const void *k, const void
     return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+namespace {
+int g_last_bounds_site = 0;   // debug build: the site gdr_last_device_error last reported
+}  // namespace
+
+extern "C" int gdr_debug_build(void) {
+#ifdef GDR_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+extern "C" int gdr_debug_bounds_site(void) { return g_last_bounds_site; }
+
 extern "C" gdr_status_t gdr_last_device_error(void *stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_CUDA;
+    // debug build: a failed bounds check comes first (it can also starve a bounded wait)
+    const int sites[] = {chunk_tc_bounds_site(), bwd_tc_bounds_site(), bwd_bounds_site(),
+                         simt_bounds_site(),     decode_bounds_site(), split_bounds_site()};
+    int site = 0;
+    for (int x : sites) {
+        if (x < 0) return GDR_ERR_CUDA;
+        if (x && !site) site = x;
+    }
+    if (site) {
+        g_last_bounds_site = site;
+        int ignore = 0;   // clear the wait error words too
+        chunk_tc_read_and_clear_error(&ignore);
+        decode_read_and_clear_error(&ignore);
+        bwd_tc_read_and_clear_error(&ignore);
+        return GDR_ERR_BOUNDS;
+    }
     int err = 0, derr = 0, berr = 0;
     if (chunk_tc_read_and_clear_error(&err) != cudaSuccess) return GDR_ERR_CUDA;
     if (decode_read_and_clear_error(&derr) != cudaSuccess) return GDR_ERR_CUDA;
@@ -320,6 +350,7 @@ extern "C" const char *gdr_status_string(gdr_status_t status) {
         case GDR_ERR_TIMEOUT: return "GDR_ERR_TIMEOUT: a bounded device wait expired";
         case GDR_ERR_WORKSPACE: return "GDR_ERR_WORKSPACE: workspace missing, misaligned or too small";
         case GDR_ERR_VALUE: return "GDR_ERR_VALUE: scalar argument out of range";
+        case GDR_ERR_BOUNDS: return "GDR_ERR_BOUNDS: a bounds check of the debug build failed";
     }
     return "unknown gdr_status_t";
 }

@@ -9,6 +9,7 @@
 // in fp32:
 //     S_start(0) = S0,  S_start(1) = S_end(0),  S_start(s+1) = M_s S_start(s) + S_local(s)
 // and the second pass recomputes every segment from its S_start.
+#include "bounds.cuh"
 #include "common.cuh"
 
 namespace gdr {
@@ -21,6 +22,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
     const int bh = blockIdx.x / slices, c0 = (blockIdx.x % slices) * COLS;
     const int tid = threadIdx.x, i = tid >> 1, h = tid & 1;   // row i, columns c0 + 8h ..
     __shared__ float S[DK][COLS + 1];
+    if (!GDR_IN_BOUNDS(bh < a.B * a.H, 501)) return;   // debug build: uniform, before any barrier
     const size_t head = (size_t)bh * a.nseg * DK * DV;
     const size_t seg_sz = (size_t)DK * DV;
     float *sstart = a.ws_sstart + head;
@@ -65,6 +67,7 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *M_all, 
     __shared__ float S[DK][COLS + 1];
     const size_t st = (size_t)DK * DV;                       // one state
     const size_t per = (size_t)BH * st;                      // one holder's block of states
+    if (!GDR_IN_BOUNDS(bh < BH, 502)) return;                // debug build: uniform, before any barrier
     float *out = S_start + bh * st + (size_t)i * DV + c0 + 8 * h;
     if (r == 0) {
         for (int j = 0; j < 8; ++j) out[j] = S0 ? S0[bh * st + (size_t)i * DV + c0 + 8 * h + j] : 0.f;
@@ -108,4 +111,8 @@ gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s) {
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
+}  // namespace gdr
+
+namespace gdr {
+GDR_BOUNDS_READER(split_bounds_site)
 }  // namespace gdr

@@ -23,6 +23,22 @@ def cuda_ok():
     return True
 
 
+@pytest.fixture(autouse=True)
+def debug_build_bounds_clean(request):
+    """With GDR_DEBUG=1 (the debug library, in-kernel bounds checks), every GPU test ends by
+    checking that the debug library is the one loaded and that no bounds check failed."""
+    yield
+    if os.environ.get("GDR_DEBUG") != "1" or request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import linear_attention_recurrence_wy_b200 as gdr
+    assert gdr.gdr_debug_build() == 1
+    rc = gdr.gdr_last_device_error(torch.cuda.current_stream().cuda_stream)
+    assert rc != -10, f"bounds check failed at site {gdr.gdr_debug_bounds_site()}"
+
+
 WORKLOAD_TESTS = ("full_size", "all_heads", "1000_steps", "long_context")
 
 
