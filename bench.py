@@ -663,12 +663,13 @@ def run_ours(args, rank, world, local):
 # keyed by workload and by a digest of the kernel's sources at capture time (a changed
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
-    ("gdn2_t4k", "chunk_tc"): (948.307712e6 + 124.674048e6, "01c4f4a7"),
-    ("decode", "decode"): (275.802368e6 + 209.808384e6, "131f9490"),
-    ("mixer_t4k", "chunk_tc"): (1090.264320e6 + 124.702720e6, "01c4f4a7"),
+    ("gdn2_t4k", "chunk_tc"): (948.144384e6 + 125.184000e6, "e871ab82"),
+    ("decode", "decode"): (275.801088e6 + 210.006784e6, "e0c71d93"),
+    ("mixer_t4k", "chunk_tc"): (1093.413376e6 + 125.841408e6, "e871ab82"),
     # the backward's step (its four launches: checkpoints, state gradient, per-chunk
-    # gradients, the strong-decay list): the inputs are read by each of the first three
-    ("bwd_t4k", "bwd"): (4774.238208e6, "18a6549f"),
+    # gradients, the strong-decay list), captured one kernel at a time on one sequence of
+    # the workload and scaled by the 8 sequences: the inputs are read by three launches
+    ("bwd_t4k", "bwd"): (8 * (421.988736e6 + 110.801408e6), "e109afb9"),
 }
 
 
