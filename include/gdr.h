@@ -141,6 +141,48 @@ gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const void *v, co
                                  unsigned long long workspace_bytes, void *stream);
 
 /*
+ * Two-phase forward for few sequence-heads.
+ *
+ * The chunkwise WY form splits every chunk's work into a part that does not depend on the
+ * state and one that does (Gated DeltaNet-2 Review §3-2.5, "Chunkwise WY training": the
+ * WY factors W = T (decayed, b-scaled K) and U = T (w.V) with T = (I + A)^-1 are built
+ * inside a chunk, and only the state S crosses chunk borders).  gdr_chunk_fwd_two_phase
+ * runs them as separate phases on the stream:
+ *   (1) for every chunk of every sequence-head at once: the chunk-local cumulative decay,
+ *       A, T, W and U, the decayed queries Qg and keys Kb and the lower-triangular P; each
+ *       chunk's record goes to the workspace (73 KB per chunk, bf16 tiles);
+ *   (2) the recurrence over the records: per sequence-head (or per segment, when nseg >
+ *       1, chained exactly as gdr_chunk_fwd_split chains them) E = U - W S,
+ *       O = Qg S + P E, S' = diag(exp gamma_C) (S + Kb^T E).
+ * Phase one fills the GPU however few sequence-heads there are, and phase two's per-chunk
+ * chain is two tensor-core round trips.  It pays for that with memory traffic (each record
+ * is written once and read once per state pass), so it wins when the sequence-heads are
+ * fewer than the SMs; gdr_chunk_fwd_two_phase_segments says when.  Results equal
+ * gdr_chunk_fwd up to rounding (W and U are rounded to bf16 as operands).
+ *
+ * Shape: bf16, dk = dv = 128, chunk 64, head-major [B, H, T, D] as gdr_chunk_fwd (other
+ * shapes: GDR_ERR_DIM).  The workspace is caller-owned device memory of at least
+ * gdr_chunk_fwd_two_phase_workspace(B, H, T, dk, dv, chunk, nseg) bytes, 16-byte aligned;
+ * its contents are scratch and need no initialisation.  nseg is clamped and rounded to
+ * whole chunks as in gdr_chunk_fwd_split.  S_T may equal S0.  Errors: those of
+ * gdr_chunk_fwd_split, GDR_ERR_WORKSPACE for a missing, misaligned or short workspace.
+ * Bounded device waits report GDR_ERR_TIMEOUT through gdr_last_device_error().
+ */
+
+/* Segment count for phase two of the two-phase forward on this device and problem, or 0
+ * when the fused kernel (gdr_chunk_fwd / gdr_chunk_fwd_split) is expected to be faster. */
+int gdr_chunk_fwd_two_phase_segments(int B, int H, int T, int dk, int dv, int chunk, gdr_dtype_t dtype);
+
+/* Workspace bytes needed by gdr_chunk_fwd_two_phase (0 for invalid arguments). */
+unsigned long long gdr_chunk_fwd_two_phase_workspace(int B, int H, int T, int dk, int dv, int chunk, int nseg);
+
+gdr_status_t gdr_chunk_fwd_two_phase(const void *q, const void *k, const void *v, const float *g_log,
+                                     const void *b, const void *w, const float *S0, void *o,
+                                     float *S_T, int B, int H, int T, int dk, int dv, int chunk,
+                                     gdr_mode_t mode, gdr_dtype_t dtype, int nseg, void *workspace,
+                                     unsigned long long workspace_bytes, void *stream);
+
+/*
  * gdr_chunk_fwd_split_noalloc -- gdr_chunk_fwd_split without a caller workspace.
  *
  * The pages have no counterpart to this entry point; it exists for callers that cannot

@@ -7,10 +7,11 @@ PyTorch fallback: if libgdr.so is missing or a call fails, an exception is raise
 
 Raw C-ABI names (integer pointers):  gdr_chunk_fwd, gdr_chunk_fwd_split,
 gdr_chunk_fwd_split_noalloc, gdr_chunk_fwd_split_segments, gdr_chunk_fwd_split_workspace,
+gdr_chunk_fwd_two_phase, gdr_chunk_fwd_two_phase_segments, gdr_chunk_fwd_two_phase_workspace,
 gdr_mixer_fwd, gdr_chunk_bwd, gdr_chunk_bwd_workspace, gdr_decode_step,
 gdr_chunk_fwd_segment_maps, gdr_chain_segment_states, gdr_last_device_error,
 gdr_status_string, gdr_test_set_first_wait_limit, gdr_debug_build, gdr_debug_bounds_site.
-Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
+Tensor wrappers:  chunk_fwd, chunk_fwd_split, chunk_fwd_two_phase, chunk_fwd_auto, chunk_fwd_host, mixer_fwd, mixer_fwd_host,
 chunk_bwd, decode_step, segment_maps, chain_segment_states; the sequence split across GPUs
 (torch.distributed): seqpar.chunk_fwd_seqpar.
 """
@@ -56,6 +57,12 @@ def lib():
         L.gdr_chunk_fwd_split_segments.restype = ci
         L.gdr_chunk_fwd_split_workspace.argtypes = [ci] * 5
         L.gdr_chunk_fwd_split_workspace.restype = ctypes.c_ulonglong
+        L.gdr_chunk_fwd_two_phase.argtypes = [vp] * 9 + [ci] * 9 + [vp, ctypes.c_ulonglong, vp]
+        L.gdr_chunk_fwd_two_phase.restype = ci
+        L.gdr_chunk_fwd_two_phase_segments.argtypes = [ci] * 7
+        L.gdr_chunk_fwd_two_phase_segments.restype = ci
+        L.gdr_chunk_fwd_two_phase_workspace.argtypes = [ci] * 7
+        L.gdr_chunk_fwd_two_phase_workspace.restype = ctypes.c_ulonglong
         L.gdr_mixer_fwd.argtypes = [vp] * 11 + [ci] * 9 + [ctypes.c_float] * 2 + [vp]
         L.gdr_mixer_fwd.restype = ci
         L.gdr_chunk_bwd.argtypes = [vp] * 16 + [ci] * 7 + [vp, ctypes.c_ulonglong, vp]
@@ -106,6 +113,20 @@ def gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, dtype):
 
 def gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg):
     return lib().gdr_chunk_fwd_split_workspace(B, H, dk, dv, nseg)
+
+
+def gdr_chunk_fwd_two_phase(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype, nseg,
+                            workspace, workspace_bytes, stream):
+    return lib().gdr_chunk_fwd_two_phase(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode,
+                                         dtype, nseg, workspace, workspace_bytes, stream)
+
+
+def gdr_chunk_fwd_two_phase_segments(B, H, T, dk, dv, chunk, dtype):
+    return lib().gdr_chunk_fwd_two_phase_segments(B, H, T, dk, dv, chunk, dtype)
+
+
+def gdr_chunk_fwd_two_phase_workspace(B, H, T, dk, dv, chunk, nseg):
+    return lib().gdr_chunk_fwd_two_phase_workspace(B, H, T, dk, dv, chunk, nseg)
 
 
 def gdr_mixer_fwd(q, k, v, xg, xb, xw, z, norm_weight, S0, y, S_T, B, H, T, dk, dv, chunk, mode,
@@ -307,6 +328,63 @@ def chunk_fwd_split(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, ns
     if rc != 0:
         raise GdrError(rc, "gdr_chunk_fwd_split")
     return o, S_T
+
+
+def chunk_fwd_two_phase(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, nseg=None,
+                        workspace=None, o=None, S_T=None, return_state=True):
+    """chunk_fwd as two phases (gdr_chunk_fwd_two_phase): the WY records of every chunk in
+    parallel, then the recurrence over them, its sequences cut into `nseg` segments (None:
+    the library's recommendation, at least 1).  The workspace (uint8 CUDA tensor) is
+    allocated here when not given.  bf16, dk = dv = 128, chunk 64 only."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dt, dev = q.dtype, q.device
+    if dt not in DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    if nseg is None:
+        nseg = max(1, gdr_chunk_fwd_two_phase_segments(B, H, T, dk, dv, chunk, DTYPES[dt]))
+    gshape, bshape, wshape = _gate_shapes(mode, (B, H, T), dk, dv)
+    for t, name, shape, tdt in ((q, "q", (B, H, T, dk), dt), (k, "k", (B, H, T, dk), dt),
+                                (v, "v", (B, H, T, dv), dt), (g, "g", gshape, torch.float32),
+                                (b, "b", bshape, dt)):
+        _check(t, name, shape, tdt, dev)
+    if wshape is not None:
+        _check(w, "w", wshape, dt, dev)
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dk, dv), torch.float32, dev)
+    need = gdr_chunk_fwd_two_phase_workspace(B, H, T, dk, dv, chunk, nseg)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    if o is None:
+        o = torch.empty(B, H, T, dv, dtype=dt, device=dev)
+    if S_T is None and return_state:
+        S_T = torch.empty(B, H, dk, dv, dtype=torch.float32, device=dev)
+    rc = gdr_chunk_fwd_two_phase(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(b),
+                                 _ptr(w) if wshape is not None else None, _ptr(S0), _ptr(o), _ptr(S_T),
+                                 B, H, T, dk, dv, chunk, MODES[mode], DTYPES[dt], nseg,
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream())
+    if rc != 0:
+        raise GdrError(rc, "gdr_chunk_fwd_two_phase")
+    return o, S_T
+
+
+def chunk_fwd_auto(q, k, v, g, b, w=None, S0=None, *, mode="gdn2", chunk=64, o=None, S_T=None,
+                   return_state=True):
+    """chunk_fwd by the path the library expects to be fastest for this problem on this
+    device: the two-phase forward, the fused kernel with a sequence split, or the fused
+    kernel (workspaces allocated here)."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype in DTYPES:
+        code = DTYPES[q.dtype]
+        n2 = gdr_chunk_fwd_two_phase_segments(B, H, T, dk, dv, chunk, code)
+        if n2 > 0:
+            return chunk_fwd_two_phase(q, k, v, g, b, w, S0, mode=mode, chunk=chunk, nseg=n2, o=o, S_T=S_T,
+                                       return_state=return_state)
+        if gdr_chunk_fwd_split_segments(B, H, T, dk, dv, chunk, code) > 1:
+            return chunk_fwd_split(q, k, v, g, b, w, S0, mode=mode, chunk=chunk, o=o, S_T=S_T,
+                                   return_state=return_state)
+    return chunk_fwd(q, k, v, g, b, w, S0, mode=mode, chunk=chunk, o=o, S_T=S_T, return_state=return_state)
 
 
 def _pipelined_host_call(inputs, outputs, groups, run, device):

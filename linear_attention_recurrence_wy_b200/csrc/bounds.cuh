@@ -9,7 +9,8 @@
 //
 // Sites:  1xx chunk_tc_kernel (forward, mixer, checkpoints, reverse), 2xx decode kernels,
 //         3xx bwd_tc_kernel, 4xx backward CUDA-core kernels, 5xx split chaining kernels,
-//         6xx chunk_simt_kernel.
+//         6xx chunk_simt_kernel, 7xx the two-phase forward's phase one (wy_prep.cu),
+//         8xx its state pass (state_pass.cu).
 #pragma once
 
 #ifdef GDR_DEBUG

@@ -144,6 +144,8 @@ int bwd_bounds_site();
 int simt_bounds_site();
 int decode_bounds_site();
 int split_bounds_site();
+int wy_prep_bounds_site();
+int state_pass_bounds_site();
 // Start state of segment r of a sequence split across R holders (ranks), from every
 // segment's maps gathered as M_all[R][BH][dk][dk] and S_all[R][BH][dk][dv] (fp32; the end
 // state of segment 0 is taken from S0 already):  r = 0: S0 (zero if NULL);  r >= 1:

@@ -9,6 +9,7 @@
 #include "common.cuh"
 #include "bwd_tc.cuh"
 #include "chunk_tc.cuh"
+#include "two_phase.cuh"
 
 using namespace gdr;
 
@@ -115,13 +116,12 @@ int gdr::split_effective_segments(int T, int chunk, int nseg) {
     return ne;
 }
 
-extern "C" int gdr_chunk_fwd_split_segments(int B, int H, int T, int dk, int dv, int chunk,
-                                            gdr_dtype_t dtype) {
-    if (B <= 0 || H <= 0 || T <= 0 || dtype != GDR_BF16 || dk != 128 || dv != 128 || chunk != 64)
-        return 1;
-    const int units = B * H, sms = sm_count(), nchunks = (T + chunk - 1) / chunk;
-    // time model in chunk-steps: first pass (state only, ~0.9 of a chunk) in waves of
-    // units * (2 nseg - 3) CTAs, second pass in waves of units * nseg CTAs
+namespace {
+
+// Time models in steps of the fused kernel's chunk period (one chunk of one sequence-head
+// on one SM, ~10 K cycles).  The fused split: its first pass (state only, ~0.9 of a chunk)
+// in waves of units * (2 nseg - 3) CTAs, its second in waves of units * nseg CTAs.
+double fused_split_time(int units, int sms, int nchunks, int *nseg_out) {
     double best = (double)((units + sms - 1) / sms) * nchunks;
     int best_n = 1;
     for (int n = 2; n <= 64 && n <= nchunks; ++n) {
@@ -135,7 +135,65 @@ extern "C" int gdr_chunk_fwd_split_segments(int B, int H, int T, int dk, int dv,
             best_n = ne;
         }
     }
-    return best_n;
+    *nseg_out = best_n;
+    return best;
+}
+
+// The two-phase forward, in the same unit: phase one over every chunk at two CTAs per SM
+// (kPrep per chunk), or bound by its traffic (the inputs, at most 112 KB per chunk, and
+// the 73 KB record it writes); then the state pass, whole or split like the fused kernel,
+// each CTA kState per chunk plus kFix to start, or bound by the records it reads and the
+// output it writes.  kBytes: HBM bytes moved in one fused chunk period (~6 TB/s x 5 us).
+constexpr double kPrep = 1.2, kState = 0.3, kFix = 0.5, kBytes = 30e6;
+constexpr double kIn = 112.0 * 1024, kRec = 74752, kOut = 16.0 * 1024;
+double waves(long long ctas, int sms) { return (double)((ctas + sms - 1) / sms); }
+double two_phase_time(int units, int sms, int nchunks, int *nseg_out) {
+    const long long un = (long long)units * nchunks;
+    const double prep = fmax(kPrep * (double)((un + 2 * sms - 1) / (2 * sms)), un * (kIn + kRec) / kBytes);
+    const double out_pass = un * (kRec + kOut) / kBytes;   // the output pass's traffic
+    double best = prep + fmax(waves(units, sms) * (kState * nchunks + kFix), out_pass);
+    int best_n = 1;
+    for (int n = 2; n <= 64 && n <= nchunks; ++n) {
+        int sc, ne;
+        split_geometry(nchunks, n, &sc, &ne);
+        if (ne < 2) continue;
+        const int r1 = 2 * ne - 3 > 1 ? 2 * ne - 3 : 1;
+        const double pass1 = fmax(waves((long long)units * r1, sms) * (kState * sc + kFix),
+                                  (double)units * r1 * sc * kRec / kBytes);
+        const double pass0 = fmax(waves((long long)units * ne, sms) * (kState * sc + kFix), out_pass);
+        const double t = prep + pass1 + pass0;
+        if (t < best) {
+            best = t;
+            best_n = ne;
+        }
+    }
+    *nseg_out = best_n;
+    return best;
+}
+
+bool two_phase_shape(int B, int H, int T, int dk, int dv, int chunk, int dtype) {
+    return B > 0 && H > 0 && T > 0 && dtype == GDR_BF16 && dk == 128 && dv == 128 && chunk == 64;
+}
+
+}  // namespace
+
+extern "C" int gdr_chunk_fwd_split_segments(int B, int H, int T, int dk, int dv, int chunk,
+                                            gdr_dtype_t dtype) {
+    if (!two_phase_shape(B, H, T, dk, dv, chunk, dtype)) return 1;
+    int n = 1;
+    fused_split_time(B * H, sm_count(), (T + chunk - 1) / chunk, &n);
+    return n;
+}
+
+extern "C" int gdr_chunk_fwd_two_phase_segments(int B, int H, int T, int dk, int dv, int chunk,
+                                                gdr_dtype_t dtype) {
+    if (!two_phase_shape(B, H, T, dk, dv, chunk, dtype)) return 0;
+    if ((long long)B * H * ((T + chunk - 1) / chunk) > INT32_MAX) return 0;
+    const int units = B * H, sms = sm_count(), nchunks = (T + chunk - 1) / chunk;
+    int nf = 1, nt = 1;
+    const double fused = fused_split_time(units, sms, nchunks, &nf);
+    const double two = two_phase_time(units, sms, nchunks, &nt);
+    return two < 0.8 * fused ? nt : 0;   // only for a clear gain
 }
 
 extern "C" unsigned long long gdr_chunk_fwd_split_workspace(int B, int H, int dk, int dv, int nseg) {
@@ -174,6 +232,54 @@ extern "C" gdr_status_t gdr_chunk_fwd_split(const void *q, const void *k, const 
     if ((st = launch_split_combine(a, s)) != GDR_OK) return st;
     a.pass = 0;
     return launch_chunk_tc(a, s);
+}
+
+extern "C" unsigned long long gdr_chunk_fwd_two_phase_workspace(int B, int H, int T, int dk, int dv, int chunk,
+                                                                int nseg) {
+    if (B < 0 || H < 0 || T < 0 || dk != 128 || dv != 128 || chunk != 64 || nseg < 1) return 0;
+    int sc = 1, ne = 1;
+    if (T > 0) split_geometry((T + chunk - 1) / chunk, nseg, &sc, &ne);
+    return tp::records_bytes(B, H, T) + tp::list_bytes(B, H, T) +
+           (ne > 1 ? gdr_chunk_fwd_split_workspace(B, H, dk, dv, ne) : 0ull);
+}
+
+extern "C" gdr_status_t gdr_chunk_fwd_two_phase(const void *q, const void *k, const void *v,
+                                                const float *g_log, const void *b, const void *w,
+                                                const float *S0, void *o, float *S_T, int B, int H,
+                                                int T, int dk, int dv, int chunk, gdr_mode_t mode,
+                                                gdr_dtype_t dtype, int nseg, void *workspace,
+                                                unsigned long long workspace_bytes, void *stream) {
+    gdr_status_t st = check_chunk(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype);
+    if (st != GDR_OK) return st;
+    if (nseg < 1) return GDR_ERR_DIM;
+    ChunkArgs a = make_args(q, k, v, g_log, b, w, S0, o, S_T, B, H, T, dk, dv, chunk, mode, dtype);
+    if (!chunk_tc_supported(a)) return GDR_ERR_DIM;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((int64_t)B * H == 0) return GDR_OK;
+    if (T == 0) return launch_state_copy(a, s);
+    const int nchunks = (T + chunk - 1) / chunk;
+    if ((int64_t)B * H * nchunks > INT32_MAX || (int64_t)B * H * 2 * nseg > INT32_MAX) return GDR_ERR_DIM;
+    int seg_chunks = 1, nseg_eff = 1;
+    split_geometry(nchunks, nseg, &seg_chunks, &nseg_eff);
+    const unsigned long long need = gdr_chunk_fwd_two_phase_workspace(B, H, T, dk, dv, chunk, nseg);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return GDR_ERR_WORKSPACE;
+    unsigned char *records = static_cast<unsigned char *>(workspace);
+    int *list = reinterpret_cast<int *>(records + tp::records_bytes(B, H, T));
+    float *split_ws = reinterpret_cast<float *>(records + tp::records_bytes(B, H, T) + tp::list_bytes(B, H, T));
+    if (cudaMemsetAsync(list, 0, sizeof(int), s) != cudaSuccess) return GDR_ERR_CUDA;
+    if ((st = tp::launch_wy_prep(a, records, list, s)) != GDR_OK) return st;
+    if (nseg_eff <= 1) return tp::launch_state_pass(a, records, s);
+    const size_t per = (size_t)B * H * nseg_eff * dk * dv;
+    a.nseg = nseg_eff;
+    a.seg_len = seg_chunks * chunk;
+    a.ws_send = split_ws;
+    a.ws_m = split_ws + per;
+    a.ws_sstart = split_ws + 2 * per;
+    a.pass = 1;
+    if ((st = tp::launch_state_pass(a, records, s)) != GDR_OK) return st;
+    if ((st = launch_split_combine(a, s)) != GDR_OK) return st;
+    a.pass = 0;
+    return tp::launch_state_pass(a, records, s);
 }
 
 extern "C" gdr_status_t gdr_chunk_fwd_segment_maps(const void *q, const void *k, const void *v,
@@ -315,7 +421,8 @@ extern "C" gdr_status_t gdr_last_device_error(void *stream) {
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_CUDA;
     // debug build: a failed bounds check comes first (it can also starve a bounded wait)
     const int sites[] = {chunk_tc_bounds_site(), bwd_tc_bounds_site(), bwd_bounds_site(),
-                         simt_bounds_site(),     decode_bounds_site(), split_bounds_site()};
+                         simt_bounds_site(),     decode_bounds_site(), split_bounds_site(),
+                         wy_prep_bounds_site(),  state_pass_bounds_site()};
     int site = 0;
     for (int x : sites) {
         if (x < 0) return GDR_ERR_CUDA;
@@ -327,13 +434,15 @@ extern "C" gdr_status_t gdr_last_device_error(void *stream) {
         chunk_tc_read_and_clear_error(&ignore);
         decode_read_and_clear_error(&ignore);
         bwd_tc_read_and_clear_error(&ignore);
+        tp::two_phase_read_and_clear_error(&ignore);
         return GDR_ERR_BOUNDS;
     }
-    int err = 0, derr = 0, berr = 0;
+    int err = 0, derr = 0, berr = 0, terr = 0;
     if (chunk_tc_read_and_clear_error(&err) != cudaSuccess) return GDR_ERR_CUDA;
     if (decode_read_and_clear_error(&derr) != cudaSuccess) return GDR_ERR_CUDA;
     if (bwd_tc_read_and_clear_error(&berr) != cudaSuccess) return GDR_ERR_CUDA;
-    return (err || derr || berr) ? GDR_ERR_TIMEOUT : GDR_OK;
+    if (tp::two_phase_read_and_clear_error(&terr) != cudaSuccess) return GDR_ERR_CUDA;
+    return (err || derr || berr || terr) ? GDR_ERR_TIMEOUT : GDR_OK;
 }
 
 extern "C" void gdr_test_set_first_wait_limit(unsigned polls) { g_first_wait_limit = polls; }

@@ -1,0 +1,460 @@
+// wy_prep.cu -- phase one of the two-phase chunked forward: the WY factors of every chunk.
+//
+// One CTA (256 threads, two CTAs per SM) per chunk of a sequence-head; the chunks do not
+// depend on one another, so a call with few sequence-heads still fills the GPU.  Per chunk
+// (Gated DeltaNet-2 Review §3-2.5 "Chunkwise WY training"; Gated DeltaNet-2 Q&A page, Q4):
+//
+//   gamma   = chunk-local cumulative sum of g_log           fp32, per key channel
+//   Kh      = b.k.e^gamma,  Qg = q.e^gamma,  Kb = k.e^-gamma   bf16 tiles (shared memory)
+//   [A; P]  = [Kh; Qg] Kb^T        one M=128 tcgen05 MMA; A strictly lower, P lower incl.
+//   T       = (I + A)^-1           blocked substitution (tri_inverse.cuh)
+//   W^T     = Kh^T T^T             W = T Kh: the pages' W, with the decay and b folded in
+//   U^T     = (w.v)^T T^T          U = T (w.v)
+//
+// and the chunk's record (two_phase.cuh) goes to global memory by bulk copies.  Thread d of
+// each half of the CTA scans key channel d over its half of the chunk's tokens and builds
+// that channel's operands as it goes (the global loads of a warp are 64 contiguous bytes of
+// one token row).  Both factors of every product in [A; P] stay within e^+-60 when |gamma| <=
+// 60 on the whole chunk; a chunk with a stronger cumulative decay is listed instead and
+// wy_exact_kernel writes its record from per-pair decays exp(gamma_i - gamma_j) in fp32 on
+// CUDA cores (with K_end = k.e^(gamma_C - gamma) in place of Kb, and the flag set that tells
+// phase two to scale the state before its update).
+#include <cuda_bf16.h>
+
+#include "bounds.cuh"
+#include "tc_util.cuh"
+#include "tri_inverse.cuh"
+#include "two_phase.cuh"
+
+namespace gdr {
+namespace tp {
+
+__device__ int g_tp_error = 0;
+
+namespace {
+
+using namespace tc;
+
+constexpr int C = 64, DK = 128, DV = 128;
+constexpr int kThreads = 256;
+constexpr float kFastLimit = 60.f;
+
+// shared memory map of the tensor-core kernel (byte offsets from a 1024-aligned base)
+constexpr int OFF_QK = 0;                       // [Kh; Qg] bf16 [128][128]            32 KB
+constexpr int OFF_KB = OFF_QK + 32768;          // Kb bf16 [64 t][128 d]               16 KB
+constexpr int OFF_WV = OFF_KB + 16384;          // w.v bf16 [64 t][128 v], then U^T    16 KB
+constexpr int OFF_P = OFF_WV + 16384;           // P bf16 [64 t][64 j]                  8 KB
+constexpr int OFF_T = OFF_P + 8192;             // T bf16 [64 t][64 j]                  8 KB
+constexpr int OFF_A32 = OFF_T + 8192;           // A, then T, fp32 [64][68]; then W^T bf16
+constexpr int OFF_X = OFF_A32 + 64 * tri::LD * 4;   // the inverse's scratch, 4 x [16][20] fp32
+constexpr int OFF_HALF = OFF_X + 4 * 16 * tri::XLD * 4;   // sum of g over tokens 0..31 [128]
+constexpr int OFF_META = OFF_HALF + 512;        // the record's e^gamma_C [128] and flag
+constexpr int OFF_BAR = OFF_META + 528 + 16;    // mbarrier; TMEM slot
+constexpr int SMEM_BYTES = OFF_BAR + 16 + 1024; // + alignment slack
+static_assert(64 * tri::LD * 4 >= 16384, "W^T fits over the inverse's fp32 scratch");
+static_assert(OFF_A32 % 1024 == 0 && OFF_WV % 1024 == 0, "tiles on 1024-byte boundaries");
+static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
+
+// TMEM columns (fp32): lane = row of [A; P]; lane = key channel of W^T, value channel of U^T
+constexpr uint32_t TM_AP = 0, TM_W = 64, TM_U = 128, TM_COLS = 256;
+
+__device__ __forceinline__ void st_bf16(unsigned char *p, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    wy_prep_kernel(ChunkArgs a, unsigned char *records, int *list) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t sbase = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+
+    const int nch = (a.T + C - 1) / C;
+    const int unit = blockIdx.x, bh = unit / nch, c = unit % nch;
+    const int t0 = c * C, n = min(C, a.T - t0);
+    const size_t row0 = (size_t)bh * a.T + t0;   // token t of the chunk is row row0 + t
+    unsigned char *rec = records + (size_t)unit * REC_BYTES;
+    // debug build: the chunk lies inside the inputs (a uniform condition)
+    if (!GDR_IN_BOUNDS(bh < a.B * a.H && n >= 1, 701)) return;
+
+    const int mode = a.mode;
+    const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
+    const __nv_bfloat16 *Q = (const __nv_bfloat16 *)a.q, *K = (const __nv_bfloat16 *)a.k;
+    const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
+    const __nv_bfloat16 *Wg = (const __nv_bfloat16 *)a.w;
+    const __nv_bfloat16 *Wsc = mode == GDR_MODE_BONLY ? Wg : Bg;   // a scalar write gate
+    float *sHalf = reinterpret_cast<float *>(sm + OFF_HALF);
+    float *sEgc = reinterpret_cast<float *>(sm + OFF_META);
+    float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
+    float *sX = reinterpret_cast<float *>(sm + OFF_X);
+    const uint32_t bar = sbase + OFF_BAR;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8);
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tslot), TM_COLS);
+        tmem_relinquish();
+    }
+    // T's blocks above the diagonal are never written by the inverse
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4 *>(sm + OFF_T)[tid + kThreads] = make_uint4(0, 0, 0, 0);
+    static_assert(kThreads * 32 == 8192, "two 16-byte stores per thread clear the T tile");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+
+    // ---- gamma and the operands: thread (d, hh) takes key channel d, tokens 32 hh .. +31 ----
+    const int d = tid & 127, hh = tid >> 7;
+    float gv[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int t = 32 * hh + i;
+        gv[i] = t < n ? (vec_g ? a.g[(row0 + t) * DK + d] : a.g[row0 + t]) : 0.f;
+    }
+    {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s += gv[i];
+        if (hh == 0) sHalf[d] = s;
+    }
+    __syncthreads();
+    float acc = hh ? sHalf[d] : 0.f, mx = 0.f;
+#pragma unroll 1
+    for (int i0 = 0; i0 < 32; i0 += 8) {
+        float fq[8], fk[8], fb[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 32 * hh + i0 + i;
+            const bool in = t < n;
+            const size_t e = (row0 + t) * DK + d;
+            fq[i] = in ? __bfloat162float(Q[e]) : 0.f;
+            fk[i] = in ? __bfloat162float(K[e]) : 0.f;
+            fb[i] = in ? __bfloat162float(vec_b ? Bg[e] : Bg[row0 + t]) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int t = 32 * hh + i0 + i;
+            acc += gv[i0 + i];
+            mx = fmaxf(mx, fabsf(acc));
+            const float eg = __expf(acc);
+            st_bf16(sm + OFF_QK + tile_off(128, t, d), fb[i] * fk[i] * eg);
+            st_bf16(sm + OFF_QK + tile_off(128, 64 + t, d), fq[i] * eg);
+            st_bf16(sm + OFF_KB + tile_off(64, t, d), fk[i] * rcp_approx(eg));
+        }
+    }
+    if (hh == 1) sEgc[d] = __expf(acc);   // gamma at the chunk's end (tokens past it add zero)
+    if (tid == 0) reinterpret_cast<int4 *>(sm + OFF_META + 512)[0] = make_int4(0, 0, 0, 0);
+    if (__syncthreads_or(mx > kFastLimit)) {
+        // strong decay: listed for the exact kernel, which writes this chunk's record
+        if (tid == 0) list[1 + atomicAdd(list, 1)] = unit;
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+        return;
+    }
+    fence_async_smem();
+    __syncthreads();
+    // ---- [A; P] = [Kh; Qg] Kb^T ----
+    if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+        for (int s = 0; s < DK / 16; ++s)
+            mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s), desc_kmajor(sbase + OFF_KB, 64, 0, s),
+                     id, s > 0);
+        mma_commit(bar);
+    }
+    const uint32_t wait_limit = a.wait_limit;
+    bool ok = __syncthreads_and(tid != 0 || mbar_wait(bar, 0u, wait_limit));
+    if (ok) {
+        tc_fence_after();
+        // A (fp32, strictly lower) -> inverse scratch; P (bf16, lower incl.) -> its tile
+        const int r = quarter * 32 + lane, j0 = (warp >> 2) * 32;
+        float x[32];
+        tmem_ld32(tmem + lane_base + TM_AP + j0, x);
+        tmem_wait_ld();
+        if (r < 64) {
+            float4 *dst = reinterpret_cast<float4 *>(sA32 + r * tri::LD + j0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                float y[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
+                dst[q] = make_float4(y[0], y[1], y[2], y[3]);
+            }
+        } else {
+            const int t = r - 64;
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
+                st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+            }
+        }
+        __syncthreads();
+        if (warp < 4) {
+            // ---- T = (I + A)^-1 by warps 0-3, straight into the bf16 tile ----
+            tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
+        } else {
+            // ---- meanwhile warps 4-7: w.v (fp32 products, one bf16 rounding) ----
+            const int u = tid - 128, tg = u >> 4, cg = u & 15;   // tokens 8 tg .. +7, channels 8 cg .. +7
+#pragma unroll 1
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * tg + i;
+                float f[8];
+                if (t < n) {
+                    const size_t e = (row0 + t) * DV + 8 * cg;
+                    float fv[8], fw[8];
+                    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(V + e), fv);
+                    if (vec_w) {
+                        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Wg + e), fw);
+                    } else {
+                        const float ws = __bfloat162float(Wsc[row0 + t]);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) fw[j] = ws;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = fw[j] * fv[j];
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = 0.f;
+                }
+                st_chunk(sbase + OFF_WV + tile_chunk(64, t, cg), f);
+            }
+        }
+        fence_async_smem();
+        __syncthreads();
+        // ---- W^T = Kh^T T^T and U^T = (w.v)^T T^T (A operands MN-major) ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, true, false, false);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + TM_W, desc_mnmajor(sbase + OFF_QK, 128, 0, s), desc_kmajor(sbase + OFF_T, 64, 0, s),
+                         id, s > 0);
+#pragma unroll
+            for (int s = 0; s < C / 16; ++s)
+                mma_bf16(tmem + TM_U, desc_mnmajor(sbase + OFF_WV, 64, 0, s), desc_kmajor(sbase + OFF_T, 64, 0, s),
+                         id, s > 0);
+            mma_commit(bar);
+        }
+        ok = __syncthreads_and(tid != 0 || mbar_wait(bar, 1u, wait_limit));
+    }
+    if (ok) {
+        tc_fence_after();
+        // W^T rows (warps 0-3) over the inverse's dead scratch, U^T rows (warps 4-7) over w.v
+        const int r = quarter * 32 + lane;
+        const uint32_t col = warp < 4 ? TM_W : TM_U;
+        const uint32_t tile = sbase + (warp < 4 ? OFF_A32 : OFF_WV);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + col + 32 * h, x);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float f[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) f[j] = x[8 * q + j];
+                st_chunk(tile + tile_chunk(128, r, 4 * h + q), f);
+            }
+        }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_s2g(rec + REC_WT, sbase + OFF_A32, 16384);
+            bulk_s2g(rec + REC_UT, sbase + OFF_WV, 16384);
+            // Qg: rows 64..127 of each column block of the stacked tile = a 64-row tile
+            bulk_s2g(rec + REC_QG, sbase + OFF_QK + 8192, 8192);
+            bulk_s2g(rec + REC_QG + 8192, sbase + OFF_QK + 16384 + 8192, 8192);
+            bulk_s2g(rec + REC_KB, sbase + OFF_KB, 16384);
+            bulk_s2g(rec + REC_P, sbase + OFF_P, 8192);
+            bulk_s2g(rec + REC_EGC, sbase + OFF_META, 528);
+            bulk_commit();
+            bulk_wait_all();
+        }
+    } else if (tid == 0) {
+        // a bounded wait expired: record it and give the tensor cores a bounded time to finish
+        atomicExch(&g_tp_error, 1);
+        mma_commit(bar);
+        mbar_wait(bar, 0u, wait_limit);
+        mbar_wait(bar, 1u, wait_limit);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+}
+
+// ---- the exact path: chunks whose cumulative decay leaves the fast path's range ----------
+// One CTA per listed chunk (grid-stride over the list), fp32 on CUDA cores throughout, from
+// the inputs in global memory: gamma by a scan per key channel, then per-pair decays
+//   A_ij = sum_d b_id k_id k_jd e^(gamma_id - gamma_jd)   (i > j)
+//   P_ij = sum_d q_id k_jd e^(gamma_id - gamma_jd)         (i >= j)
+// T = (I + A)^-1 by forward substitution row by row, W = T Kh, U = T (w.v) with
+// Kh = b.k.e^gamma, and the record's tiles written element by element.  Rarely run.
+constexpr int XS = 129;   // padded fp32 row stride of the [64][128] arrays
+constexpr int XOFF_G = 0;                    // gamma [64][XS]
+constexpr int XOFF_K = XOFF_G + 64 * XS * 4; // k [64][XS]
+constexpr int XOFF_Q = XOFF_K + 64 * XS * 4; // q, then w.v [64][XS]
+constexpr int XOFF_B = XOFF_Q + 64 * XS * 4; // b.k [64][XS] (Kh before the decay)
+constexpr int XOFF_A = XOFF_B + 64 * XS * 4; // A [64][65]
+constexpr int XOFF_T = XOFF_A + 64 * 65 * 4; // T [64][65]
+constexpr int XOFF_GC = XOFF_T + 64 * 65 * 4;   // gamma_C [128]
+constexpr int XSMEM = XOFF_GC + 512;
+
+__global__ void __launch_bounds__(kThreads, 1) wy_exact_kernel(ChunkArgs a, unsigned char *records, const int *list) {
+    extern __shared__ float xs[];
+    float *sG = xs + XOFF_G / 4, *sK = xs + XOFF_K / 4, *sQ = xs + XOFF_Q / 4, *sBK = xs + XOFF_B / 4;
+    float *sA = xs + XOFF_A / 4, *sT = xs + XOFF_T / 4, *sGC = xs + XOFF_GC / 4;
+    const int tid = threadIdx.x;
+    const int nch = (a.T + C - 1) / C;
+    const int count = list[0];
+    const int mode = a.mode;
+    const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
+    const __nv_bfloat16 *Q = (const __nv_bfloat16 *)a.q, *K = (const __nv_bfloat16 *)a.k;
+    const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
+    const __nv_bfloat16 *Wg = (const __nv_bfloat16 *)a.w;
+    const __nv_bfloat16 *Wsc = mode == GDR_MODE_BONLY ? Wg : Bg;
+#pragma unroll 1
+    for (int li = blockIdx.x; li < count; li += gridDim.x) {
+        const int unit = list[1 + li];
+        if (!GDR_IN_BOUNDS(unit >= 0 && unit < a.B * a.H * nch, 702)) continue;
+        const int bh = unit / nch, c = unit % nch;
+        const int t0 = c * C, n = min(C, a.T - t0);
+        const size_t row0 = (size_t)bh * a.T + t0;
+        unsigned char *rec = records + (size_t)unit * REC_BYTES;
+        __syncthreads();   // the previous chunk's readers are done with the arrays
+        // inputs (zero past the chunk's end) and gamma
+        for (int e = tid; e < C * DK; e += kThreads) {
+            const int t = e >> 7, dd = e & 127;
+            const bool in = t < n;
+            const size_t ge = (row0 + t) * DK + dd;
+            const float kv = in ? __bfloat162float(K[ge]) : 0.f;
+            const float bv = in ? __bfloat162float(vec_b ? Bg[ge] : Bg[row0 + t]) : 0.f;
+            sK[t * XS + dd] = kv;
+            sQ[t * XS + dd] = in ? __bfloat162float(Q[ge]) : 0.f;
+            sBK[t * XS + dd] = bv * kv;
+        }
+        if (tid < DK) {
+            float g = 0.f;
+            for (int t = 0; t < C; ++t) {
+                if (t < n) g += vec_g ? a.g[(row0 + t) * DK + tid] : a.g[row0 + t];
+                sG[t * XS + tid] = g;
+            }
+            sGC[tid] = g;
+        }
+        __syncthreads();
+        // A and P from per-pair decays; P straight into the record
+        for (int p = tid; p < C * C; p += kThreads) {
+            const int i = p >> 6, j = p & 63;
+            float sa = 0.f, sp = 0.f;
+            if (j <= i && i < n) {
+                for (int dd = 0; dd < DK; ++dd) {
+                    const float kd = sK[j * XS + dd] * __expf(sG[i * XS + dd] - sG[j * XS + dd]);
+                    sa = fmaf(sBK[i * XS + dd], kd, sa);
+                    sp = fmaf(sQ[i * XS + dd], kd, sp);
+                }
+            }
+            sA[i * 65 + j] = j < i ? sa : 0.f;
+            st_bf16(rec + REC_P + tile_off(64, i, j), sp);
+        }
+        __syncthreads();
+        // T = (I + A)^-1 by forward substitution; thread j < 64 owns column j, whose rows
+        // depend only on its own rows above: T_ij = [i == j] - sum_{j<=m<i} A_im T_mj
+        if (tid < C) {
+            const int j = tid;
+            for (int i = 0; i < C; ++i) {
+                float x = i == j ? 1.f : 0.f;
+                for (int m = j; m < i; ++m) x = fmaf(-sA[i * 65 + m], sT[m * 65 + j], x);
+                sT[i * 65 + j] = j <= i ? x : 0.f;
+            }
+        }
+        __syncthreads();
+        // the operands: Kh = b.k.e^gamma in place, Qg, K_end; w.v over q
+        for (int e = tid; e < C * DK; e += kThreads) {
+            const int t = e >> 7, dd = e & 127;
+            const float gm = sG[t * XS + dd];
+            const float eg = __expf(gm);
+            st_bf16(rec + REC_QG + tile_off(64, t, dd), sQ[t * XS + dd] * eg);
+            st_bf16(rec + REC_KB + tile_off(64, t, dd), sK[t * XS + dd] * __expf(sGC[dd] - gm));
+            sBK[t * XS + dd] *= eg;
+        }
+        __syncthreads();
+        for (int e = tid; e < C * DV; e += kThreads) {
+            const int t = e >> 7, vv = e & 127;
+            float x = 0.f;
+            if (t < n) {
+                const size_t ge = (row0 + t) * DV + vv;
+                const float wv = __bfloat162float(vec_w ? Wg[ge] : Wsc[row0 + t]);
+                x = wv * __bfloat162float(V[ge]);
+            }
+            sQ[t * XS + vv] = x;
+        }
+        __syncthreads();
+        // W^T [d][t] = sum_j Kh[j][d] T[t][j],  U^T [v][t] = sum_j wv[j][v] T[t][j]
+        for (int e = tid; e < C * DK; e += kThreads) {
+            const int t = e >> 7, dd = e & 127;
+            float w = 0.f, u = 0.f;
+            for (int j = 0; j <= t; ++j) {
+                const float tj = sT[t * 65 + j];
+                w = fmaf(sBK[j * XS + dd], tj, w);
+                u = fmaf(sQ[j * XS + dd], tj, u);
+            }
+            st_bf16(rec + REC_WT + tile_off(128, dd, t), w);
+            st_bf16(rec + REC_UT + tile_off(128, dd, t), u);
+        }
+        if (tid < DK) reinterpret_cast<float *>(rec + REC_EGC)[tid] = __expf(sGC[tid]);
+        if (tid == 0) *reinterpret_cast<int *>(rec + REC_FLAG) = 1;
+    }
+}
+
+}  // namespace
+
+unsigned long long records_bytes(int B, int H, int T) {
+    return (unsigned long long)B * H * ((T + C - 1) / C) * REC_BYTES;
+}
+unsigned long long list_bytes(int B, int H, int T) {
+    const unsigned long long n = 1ull + (unsigned long long)B * H * ((T + C - 1) / C);
+    return (n * 4 + 15) / 16 * 16;
+}
+
+gdr_status_t launch_wy_prep(const ChunkArgs &a, unsigned char *records, int *list, cudaStream_t s) {
+    const long long units = (long long)a.B * a.H * ((a.T + C - 1) / C);
+    if (units <= 0) return GDR_OK;
+    if (cudaFuncSetAttribute(wy_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(wy_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, XSMEM) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    wy_prep_kernel<<<(unsigned)units, kThreads, SMEM_BYTES, s>>>(a, records, list);
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDR_ERR_CUDA;
+    wy_exact_kernel<<<(unsigned)(units < sms ? units : sms), kThreads, XSMEM, s>>>(a, records, list);
+    return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
+}
+
+cudaError_t two_phase_read_and_clear_error(int *err) {
+    int e1 = 0, e2 = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&e1, g_tp_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(g_tp_error, &zero, sizeof(int))) != cudaSuccess) return e;
+    if ((e = state_pass_read_and_clear_error(&e2)) != cudaSuccess) return e;
+    *err = e1 || e2;
+    return cudaSuccess;
+}
+
+}  // namespace tp
+
+GDR_BOUNDS_READER(wy_prep_bounds_site)
+
+}  // namespace gdr

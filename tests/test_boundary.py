@@ -133,6 +133,44 @@ def test_split_rejects(L, kw, code):
     assert call_split(**kw) == code
 
 
+def call_two_phase(nseg=1, ws=A, ws_bytes=1000, dk=128, dv=128, chunk=64, dtype=1, T=1024, B=1, H=2, mode=0):
+    return gdr.gdr_chunk_fwd_two_phase(A, A, A, A, A, A, None, A, None, B, H, T, dk, dv, chunk, mode, dtype,
+                                       nseg, ws, ws_bytes, None)
+
+
+def test_two_phase_workspace_size_and_planner(L):
+    rec = 74752                                       # one chunk's record
+    # records, then the exact-path list (a count and one index per chunk, 16-byte padded),
+    # then the sequence split's three state arrays when the state pass is split
+    assert gdr.gdr_chunk_fwd_two_phase_workspace(2, 3, 1000, 128, 128, 64, 1) == 6 * 16 * rec + 400
+    assert gdr.gdr_chunk_fwd_two_phase_workspace(2, 3, 1000, 128, 128, 64, 4) == \
+        6 * 16 * rec + 400 + 3 * 6 * 4 * 128 * 128 * 4
+    assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 64, 64, 64, 1) == 0
+    assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 128, 128, 32, 1) == 0
+    assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 128, 128, 64, 0) == 0
+    # the planner (this host has no GPU: 148 SMs assumed) takes the two-phase path when the
+    # sequence-heads are too few to fill the GPU, and the fused kernel when they fill it
+    assert gdr.gdr_chunk_fwd_two_phase_segments(4, 16, 2048, 128, 128, 64, 1) >= 1
+    assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 128, 128, 64, 1) > 1
+    assert gdr.gdr_chunk_fwd_two_phase_segments(8, 16, 4096, 128, 128, 64, 1) == 0
+    assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 64, 64, 64, 1) == 0
+    assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 128, 128, 64, 0) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ws=None), WORKSPACE), (dict(ws_bytes=1 << 20), WORKSPACE), (dict(ws=A + 8), WORKSPACE),
+    (dict(nseg=0), DIM), (dict(dk=64), DIM), (dict(dtype=0), DIM), (dict(chunk=32), DIM), (dict(mode=6), MODE),
+    (dict(T=-1), DIM),
+])
+def test_two_phase_rejects(L, kw, code):
+    assert call_two_phase(**kw) == code
+
+
+def test_two_phase_empty_is_a_no_op(L):
+    assert call_two_phase(B=0) == OK
+    assert call_two_phase(H=0) == OK
+
+
 def call_mixer(q=A, k=A, v=A, xg=A, xb=A, xw=A, z=A, nw=A, S0=None, y=A, ST=None, B=1, H=2, T=8,
                dk=128, dv=128, chunk=64, mode=0, dtype=1, layout=1, b_range=1.0, eps=1e-5):
     return gdr.gdr_mixer_fwd(q, k, v, xg, xb, xw, z, nw, S0, y, ST, B, H, T, dk, dv, chunk, mode, dtype,

@@ -90,3 +90,21 @@ def test_backward_first_wait_expires_then_recovers(cuda_ok):
     ref = oracle.bwd(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"], dO, dST, mode="gdn2")
     for n in ("dq", "dk", "dv", "dg", "db", "dw", "dS0"):
         assert_close(f"{n} after expiry", np64(out[n]), ref[n], "bf16")
+
+
+@pytest.mark.parametrize("nseg", [1, 3])
+def test_two_phase_first_wait_expires_then_recovers(cuda_ok, nseg):
+    # the state pass's first wait (for its first chunk record) gives up after one poll
+    d_cpu = workload.make_small(2, 3, 640, 128, 128, mode="gdn2", dtype="bf16", seed=26, g_scale=0.1,
+                                s0_std=0.05)
+    d = to_dev(d_cpu)
+    run = lambda: gdr.chunk_fwd_two_phase(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"],
+                                          mode="gdn2", nseg=nseg)
+    assert expire_once(run) == TIMEOUT
+    o, ST = run()
+    torch.cuda.synchronize()
+    assert gdr.gdr_last_device_error(stream()) == 0
+    o_ref, S_ref = oracle.fwd(d_cpu["q"], d_cpu["k"], d_cpu["v"], d_cpu["g"], d_cpu["b"], d_cpu["w"],
+                              d_cpu["S0"], mode="gdn2")
+    assert_close("o after expiry", np64(o), o_ref, "bf16")
+    assert_close("S_T after expiry", np64(ST), S_ref, "bf16")
