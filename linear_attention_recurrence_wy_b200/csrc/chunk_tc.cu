@@ -114,12 +114,21 @@ constexpr uint32_t TM_COLS = 512;
 constexpr int BAR_WY = 2;    // warps 0-7
 constexpr int BAR_ST = 3;    // warps 8-15
 
+// The named barriers below are the .aligned forms: every thread of a warp must reach them
+// together.  A thread that ran code alone just before (an elected issuer, a bounded wait
+// inside the barrier's own argument) may still be diverged from its warp, so each helper
+// first reconverges the warp (__syncwarp); the warp then also leaves the barrier converged,
+// which the warp-collective instructions after it (.aligned tcgen05 loads and stores,
+// shuffles, warp MMAs) need.
+
 // barrier over the 256 threads of one warp group
 __device__ __forceinline__ void group_sync(int id) {
+    __syncwarp();
     asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory");
 }
 // barrier over one warp group that also returns the AND of v over it
 __device__ __forceinline__ bool group_and(int id, bool v) {
+    __syncwarp();
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -133,6 +142,7 @@ __device__ __forceinline__ bool group_and(int id, bool v) {
 }
 // the same over 128 threads (warps 4-7 of the WY group)
 __device__ __forceinline__ bool bar128_and(int id, bool v) {
+    __syncwarp();
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -145,6 +155,7 @@ __device__ __forceinline__ bool bar128_and(int id, bool v) {
     return r != 0;
 }
 __device__ __forceinline__ bool bar128_or(int id, bool v) {
+    __syncwarp();
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
@@ -353,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         sAbort[0] = 0;
         fence_mbar_init();
     }
+    __syncwarp();
     if (warp == 0) {
         tmem_alloc(smem_u32(tslot), TM_COLS);
         tmem_relinquish();
@@ -1151,6 +1163,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
         }
     }
     __syncthreads();
+    __syncwarp();   // tid 0 drained alone: warp 0 reconverges for the .aligned dealloc
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }

@@ -119,8 +119,9 @@ int gdr::split_effective_segments(int T, int chunk, int nseg) {
 namespace {
 
 // Time models in steps of the fused kernel's chunk period (one chunk of one sequence-head
-// on one SM, ~10 K cycles).  The fused split: its first pass (state only, ~0.9 of a chunk)
-// in waves of units * (2 nseg - 3) CTAs, its second in waves of units * nseg CTAs.
+// on one SM, ~10 K cycles, ~5.7 us on B200).  The fused split: its first pass (state only,
+// as costly per chunk as a whole chunk, measured) in waves of units * (2 nseg - 3) CTAs, its
+// second in waves of units * nseg CTAs.
 double fused_split_time(int units, int sms, int nchunks, int *nseg_out) {
     double best = (double)((units + sms - 1) / sms) * nchunks;
     int best_n = 1;
@@ -129,7 +130,7 @@ double fused_split_time(int units, int sms, int nchunks, int *nseg_out) {
         split_geometry(nchunks, n, &sc, &ne);
         if (ne < 2) continue;
         const int r1 = 2 * ne - 3 > 1 ? 2 * ne - 3 : 1;
-        const double t = 0.9 * ((units * r1 + sms - 1) / sms) * sc + (double)((units * ne + sms - 1) / sms) * sc;
+        const double t = (double)((units * r1 + sms - 1) / sms) * sc + (double)((units * ne + sms - 1) / sms) * sc;
         if (t < 0.8 * best) {   // split only for a clear gain
             best = t;
             best_n = ne;
@@ -139,12 +140,13 @@ double fused_split_time(int units, int sms, int nchunks, int *nseg_out) {
     return best;
 }
 
-// The two-phase forward, in the same unit: phase one over every chunk at two CTAs per SM
-// (kPrep per chunk), or bound by its traffic (the inputs, at most 112 KB per chunk, and
+// The two-phase forward, in the same unit (constants measured on B200 with per-phase clock
+// stamps): phase one over every chunk, two persistent CTAs per SM, a wave of two chunks per
+// SM taking kPrep (its latency-bound per-chunk path, ~30 K cycles), or bound by its traffic (the inputs, at most 112 KB per chunk, and
 // the 73 KB record it writes); then the state pass, whole or split like the fused kernel,
 // each CTA kState per chunk plus kFix to start, or bound by the records it reads and the
 // output it writes.  kBytes: HBM bytes moved in one fused chunk period (~6 TB/s x 5 us).
-constexpr double kPrep = 1.2, kState = 0.3, kFix = 0.5, kBytes = 30e6;
+constexpr double kPrep = 3.5, kState = 0.37, kFix = 0.5, kBytes = 34e6;
 constexpr double kIn = 112.0 * 1024, kRec = 74752, kOut = 16.0 * 1024;
 double waves(long long ctas, int sms) { return (double)((ctas + sms - 1) / sms); }
 double two_phase_time(int units, int sms, int nchunks, int *nseg_out) {
@@ -193,7 +195,7 @@ extern "C" int gdr_chunk_fwd_two_phase_segments(int B, int H, int T, int dk, int
     int nf = 1, nt = 1;
     const double fused = fused_split_time(units, sms, nchunks, &nf);
     const double two = two_phase_time(units, sms, nchunks, &nt);
-    return two < 0.8 * fused ? nt : 0;   // only for a clear gain
+    return two < 0.97 * fused ? nt : 0;   // where the model sees a gain beyond its rounding
 }
 
 extern "C" unsigned long long gdr_chunk_fwd_split_workspace(int B, int H, int dk, int dv, int nseg) {

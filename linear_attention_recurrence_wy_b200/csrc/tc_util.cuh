@@ -341,9 +341,13 @@ struct TileOut {
     }
 };
 
-// barrier over warps 0-3 (named barrier 1), the inverse's warps
+// barrier over warps 0-3 (named barrier 1), the inverse's warps (the warp reconverged first:
+// bar.sync is the .aligned form)
 struct Bar128 {
-    __device__ __forceinline__ void operator()() const { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+    __device__ __forceinline__ void operator()() const {
+        __syncwarp();
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
 };
 #endif
 

@@ -1,7 +1,8 @@
 // wy_prep.cu -- phase one of the two-phase chunked forward: the WY factors of every chunk.
 //
-// One CTA (256 threads, two CTAs per SM) per chunk of a sequence-head; the chunks do not
-// depend on one another, so a call with few sequence-heads still fills the GPU.  Per chunk
+// Persistent CTAs (256 threads, two per SM) take the chunks of every sequence-head in turn;
+// the chunks do not depend on one another, so a call with few sequence-heads still fills
+// the GPU.  Per chunk
 // (Gated DeltaNet-2 Review §3-2.5 "Chunkwise WY training"; Gated DeltaNet-2 Q&A page, Q4):
 //
 //   gamma   = chunk-local cumulative sum of g_log           fp32, per key channel
@@ -11,17 +12,22 @@
 //   W^T     = Kh^T T^T             W = T Kh: the pages' W, with the decay and b folded in
 //   U^T     = (w.v)^T T^T          U = T (w.v)
 //
-// and the chunk's record (two_phase.cuh) goes to global memory by bulk copies.  Thread d of
-// each half of the CTA scans key channel d over its half of the chunk's tokens and builds
-// that channel's operands as it goes (the global loads of a warp are 64 contiguous bytes of
-// one token row).  Both factors of every product in [A; P] stay within e^+-60 when |gamma| <=
+// and the chunk's record (two_phase.cuh) goes to global memory by bulk copies.  q, k, v and
+// a per-channel b arrive by tiled tensor copies (TMA, 128-byte swizzle) straight into the
+// operand tiles, and the operands are built in place: thread d of each half of the CTA scans
+// key channel d over its half of the chunk's tokens (g_log read from global memory up front)
+// and turns that channel's b, q, k into Kh, Qg, Kb as it goes; w.v replaces v.  Both factors of every product in [A; P] stay within e^+-60 when |gamma| <=
 // 60 on the whole chunk; a chunk with a stronger cumulative decay is listed instead and
 // wy_exact_kernel writes its record from per-pair decays exp(gamma_i - gamma_j) in fp32 on
 // CUDA cores (with K_end = k.e^(gamma_C - gamma) in place of Kb, and the flag set that tells
 // phase two to scale the state before its update).
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <string.h>
 
 #include "bounds.cuh"
+#include "chunk_tc.cuh"
 #include "tc_util.cuh"
 #include "tri_inverse.cuh"
 #include "two_phase.cuh"
@@ -48,9 +54,10 @@ constexpr int OFF_T = OFF_P + 8192;             // T bf16 [64 t][64 j]          
 constexpr int OFF_A32 = OFF_T + 8192;           // A, then T, fp32 [64][68]; then W^T bf16
 constexpr int OFF_X = OFF_A32 + 64 * tri::LD * 4;   // the inverse's scratch, 4 x [16][20] fp32
 constexpr int OFF_HALF = OFF_X + 4 * 16 * tri::XLD * 4;   // sum of g over tokens 0..31 [128]
-constexpr int OFF_META = OFF_HALF + 512;        // the record's e^gamma_C [128] and flag
-constexpr int OFF_BAR = OFF_META + 528 + 16;    // mbarrier; TMEM slot
-constexpr int SMEM_BYTES = OFF_BAR + 16 + 1024; // + alignment slack
+constexpr int OFF_BETA = OFF_HALF + 512;        // scalar erase gate of the chunk's tokens [64]
+constexpr int OFF_META = OFF_BETA + 256;        // the record's e^gamma_C [128] and flag
+constexpr int OFF_BAR = OFF_META + 528 + 16;    // mbarriers (MMA, tile copies); TMEM slot
+constexpr int SMEM_BYTES = OFF_BAR + 24 + 1024; // + alignment slack
 static_assert(64 * tri::LD * 4 >= 16384, "W^T fits over the inverse's fp32 scratch");
 static_assert(OFF_A32 % 1024 == 0 && OFF_WV % 1024 == 0, "tiles on 1024-byte boundaries");
 static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
@@ -58,12 +65,38 @@ static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
 // TMEM columns (fp32): lane = row of [A; P]; lane = key channel of W^T, value channel of U^T
 constexpr uint32_t TM_AP = 0, TM_W = 64, TM_U = 128, TM_COLS = 256;
 
+// CTA barriers that also reconverge the warp: a thread that ran code alone (an elected
+// issuer, a bounded wait) may otherwise come out of the barrier still diverged from its
+// warp, and every later warp-collective instruction (shuffles, warp MMAs, the .aligned
+// tcgen05 loads and stores) then pays for re-synchronising it, or is not allowed at all
+__device__ __forceinline__ void sync_all() {
+    __syncthreads();
+    __syncwarp();
+}
+__device__ __forceinline__ bool sync_all_and(bool v) {
+    const bool r = __syncthreads_and(v);
+    __syncwarp();
+    return r;
+}
+__device__ __forceinline__ bool sync_all_or(bool v) {
+    const bool r = __syncthreads_or(v);
+    __syncwarp();
+    return r;
+}
+
 __device__ __forceinline__ void st_bf16(unsigned char *p, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
 }
 
+// Tensor maps of the bf16 inputs read as tiles: [B*H*T rows][128] row-major, box {64, 64}
+// with the 128-byte swizzle, so a box lands in shared memory in the operand tile layout of
+// tc_util.cuh and the operands are built in place (rows past the tensor's end read zero).
+struct PrepMaps {
+    CUtensorMap q, k, v, b;
+};
+
 __global__ void __launch_bounds__(kThreads, 2)
-    wy_prep_kernel(ChunkArgs a, unsigned char *records, int *list) {
+    wy_prep_kernel(ChunkArgs a, unsigned char *records, int *list, const __grid_constant__ PrepMaps tm) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = (unsigned char *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sbase = smem_u32(sm);
@@ -72,166 +105,221 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
 
     const int nch = (a.T + C - 1) / C;
-    const int unit = blockIdx.x, bh = unit / nch, c = unit % nch;
-    const int t0 = c * C, n = min(C, a.T - t0);
-    const size_t row0 = (size_t)bh * a.T + t0;   // token t of the chunk is row row0 + t
-    unsigned char *rec = records + (size_t)unit * REC_BYTES;
-    // debug build: the chunk lies inside the inputs (a uniform condition)
-    if (!GDR_IN_BOUNDS(bh < a.B * a.H && n >= 1, 701)) return;
-
+    const int units = a.B * a.H * nch;
     const int mode = a.mode;
     const bool vec_b = mode_b_vec(mode), vec_w = mode_w_vec(mode), vec_g = mode_g_vec(mode);
-    const __nv_bfloat16 *Q = (const __nv_bfloat16 *)a.q, *K = (const __nv_bfloat16 *)a.k;
-    const __nv_bfloat16 *V = (const __nv_bfloat16 *)a.v, *Bg = (const __nv_bfloat16 *)a.b;
-    const __nv_bfloat16 *Wg = (const __nv_bfloat16 *)a.w;
+    const __nv_bfloat16 *Bg = (const __nv_bfloat16 *)a.b, *Wg = (const __nv_bfloat16 *)a.w;
     const __nv_bfloat16 *Wsc = mode == GDR_MODE_BONLY ? Wg : Bg;   // a scalar write gate
     float *sHalf = reinterpret_cast<float *>(sm + OFF_HALF);
+    float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
     float *sEgc = reinterpret_cast<float *>(sm + OFF_META);
     float *sA32 = reinterpret_cast<float *>(sm + OFF_A32);
     float *sX = reinterpret_cast<float *>(sm + OFF_X);
-    const uint32_t bar = sbase + OFF_BAR;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 8);
+    const uint32_t bar = sbase + OFF_BAR, bar_ld = bar + 8;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 16);
 
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar_ld, 1);
         fence_mbar_init();
     }
+    __syncwarp();
     if (warp == 0) {
         tmem_alloc(smem_u32(tslot), TM_COLS);
         tmem_relinquish();
     }
-    // T's blocks above the diagonal are never written by the inverse
+    // T's blocks above the diagonal are never written by the inverse: cleared once
     reinterpret_cast<uint4 *>(sm + OFF_T)[tid] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4 *>(sm + OFF_T)[tid + kThreads] = make_uint4(0, 0, 0, 0);
     static_assert(kThreads * 32 == 8192, "two 16-byte stores per thread clear the T tile");
     tc_fence_before();
-    __syncthreads();
+    sync_all();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-
-    // ---- gamma and the operands: thread (d, hh) takes key channel d, tokens 32 hh .. +31 ----
-    const int d = tid & 127, hh = tid >> 7;
-    float gv[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int t = 32 * hh + i;
-        gv[i] = t < n ? (vec_g ? a.g[(row0 + t) * DK + d] : a.g[row0 + t]) : 0.f;
-    }
-    {
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s += gv[i];
-        if (hh == 0) sHalf[d] = s;
-    }
-    __syncthreads();
-    float acc = hh ? sHalf[d] : 0.f, mx = 0.f;
-#pragma unroll 1
-    for (int i0 = 0; i0 < 32; i0 += 8) {
-        float fq[8], fk[8], fb[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 32 * hh + i0 + i;
-            const bool in = t < n;
-            const size_t e = (row0 + t) * DK + d;
-            fq[i] = in ? __bfloat162float(Q[e]) : 0.f;
-            fk[i] = in ? __bfloat162float(K[e]) : 0.f;
-            fb[i] = in ? __bfloat162float(vec_b ? Bg[e] : Bg[row0 + t]) : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = 32 * hh + i0 + i;
-            acc += gv[i0 + i];
-            mx = fmaxf(mx, fabsf(acc));
-            const float eg = __expf(acc);
-            st_bf16(sm + OFF_QK + tile_off(128, t, d), fb[i] * fk[i] * eg);
-            st_bf16(sm + OFF_QK + tile_off(128, 64 + t, d), fq[i] * eg);
-            st_bf16(sm + OFF_KB + tile_off(64, t, d), fk[i] * rcp_approx(eg));
-        }
-    }
-    if (hh == 1) sEgc[d] = __expf(acc);   // gamma at the chunk's end (tokens past it add zero)
-    if (tid == 0) reinterpret_cast<int4 *>(sm + OFF_META + 512)[0] = make_int4(0, 0, 0, 0);
-    if (__syncthreads_or(mx > kFastLimit)) {
-        // strong decay: listed for the exact kernel, which writes this chunk's record
-        if (tid == 0) list[1 + atomicAdd(list, 1)] = unit;
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (warp == 0) tmem_dealloc(tmem, TM_COLS);
-        return;
-    }
-    fence_async_smem();
-    __syncthreads();
-    // ---- [A; P] = [Kh; Qg] Kb^T ----
-    if (tid == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_bf16(128, 64, false, false, false);
-#pragma unroll
-        for (int s = 0; s < DK / 16; ++s)
-            mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s), desc_kmajor(sbase + OFF_KB, 64, 0, s),
-                     id, s > 0);
-        mma_commit(bar);
-    }
     const uint32_t wait_limit = a.wait_limit;
-    bool ok = __syncthreads_and(tid != 0 || mbar_wait(bar, 0u, wait_limit));
-    if (ok) {
-        tc_fence_after();
-        // A (fp32, strictly lower) -> inverse scratch; P (bf16, lower incl.) -> its tile
-        const int r = quarter * 32 + lane, j0 = (warp >> 2) * 32;
-        float x[32];
-        tmem_ld32(tmem + lane_base + TM_AP + j0, x);
-        tmem_wait_ld();
-        if (r < 64) {
-            float4 *dst = reinterpret_cast<float4 *>(sA32 + r * tri::LD + j0);
+    const int d = tid & 127, hh = tid >> 7;      // scan and build: key channel d, tokens 32 hh ..
+    const int tg = tid >> 4, cg = tid & 15;      // write gate: tokens 4 tg .., channels 8 cg ..
+    bool ok = true;
+    uint32_t n_mma = 0;                          // commits on bar so far (its phase parity)
+    int ld_issued = 0;                           // tile-copy batches issued (thread 0)
+
+    // A persistent CTA: two per SM take the chunks in turn, so the code stays in the
+    // instruction cache (each chunk runs every phase once, a long straight-line path).
+#pragma unroll 1
+    for (int it = 0, unit = blockIdx.x; unit < units; ++it, unit += gridDim.x) {
+        const int bh = unit / nch, c = unit % nch;
+        const int t0 = c * C, n = min(C, a.T - t0);
+        const size_t row0 = (size_t)bh * a.T + t0;   // token t of the chunk is row row0 + t
+        unsigned char *rec = records + (size_t)unit * REC_BYTES;
+        // debug build: the chunk lies inside the inputs (a uniform condition)
+        if (!GDR_IN_BOUNDS(bh < a.B * a.H && n >= 1, 701)) break;
+        if (tid == 0) {
+            // the chunk's q, k, v (and a per-channel b) as tiles: q into the Qg rows of the
+            // stacked [Kh; Qg] tile, b into its Kh rows, k into the Kb tile, v into the w.v
+            // tile (the previous chunk's copies out of these tiles have read them)
+            fence_async_smem();
+            mbar_arrive_expect_tx(bar_ld, (vec_b ? 8u : 6u) * 8192u);
+            ++ld_issued;
+            const int r = (int)row0;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float y[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
-                dst[q] = make_float4(y[0], y[1], y[2], y[3]);
-            }
-        } else {
-            const int t = r - 64;
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                float f[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
-                st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+            for (int h = 0; h < 2; ++h) {
+                tma_load_2d(sbase + OFF_QK + h * 16384 + 8192, &tm.q, 64 * h, r, bar_ld);
+                tma_load_2d(sbase + OFF_KB + h * 8192, &tm.k, 64 * h, r, bar_ld);
+                tma_load_2d(sbase + OFF_WV + h * 8192, &tm.v, 64 * h, r, bar_ld);
+                if (vec_b) tma_load_2d(sbase + OFF_QK + h * 16384, &tm.b, 64 * h, r, bar_ld);
             }
         }
-        __syncthreads();
-        if (warp < 4) {
-            // ---- T = (I + A)^-1 by warps 0-3, straight into the bf16 tile ----
-            tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
-        } else {
-            // ---- meanwhile warps 4-7: w.v (fp32 products, one bf16 rounding) ----
-            const int u = tid - 128, tg = u >> 4, cg = u & 15;   // tokens 8 tg .. +7, channels 8 cg .. +7
-#pragma unroll 1
+        __syncwarp();
+
+        // ---- global loads issued up front: g_log of (channel d, tokens 32 hh ..), the write
+        //      gate of (tokens 4 tg .., channels 8 cg ..), a scalar erase gate per token ----
+        float gv[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int t = 32 * hh + i;
+            gv[i] = t < n ? (vec_g ? a.g[(row0 + t) * DK + d] : a.g[row0 + t]) : 0.f;
+        }
+        uint4 wr[4];
+        float wsc[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * tg + i;
+            wr[i] = make_uint4(0, 0, 0, 0);
+            wsc[i] = 0.f;
+            if (t < n) {
+                if (vec_w) wr[i] = *reinterpret_cast<const uint4 *>(Wg + (row0 + t) * DV + 8 * cg);
+                else wsc[i] = __bfloat162float(Wsc[row0 + t]);
+            }
+        }
+        if (!vec_b && tid < C) sBeta[tid] = tid < n ? __bfloat162float(Bg[row0 + tid]) : 0.f;
+        {
+            float sum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum += gv[i];
+            if (hh == 0) sHalf[d] = sum;
+        }
+        ok = sync_all_and(tid != 0 || mbar_wait(bar_ld, (uint32_t)(it & 1), wait_limit));
+        if (!ok) break;
+
+        // ---- gamma and the operands, in place: thread (d, hh) scans key channel d over
+        //      tokens 32 hh .. 32 hh + 31 (from the first half's sum) and turns b, q, k into
+        //      Kh, Qg, Kb.  In batches of eight tokens: every load of a batch first, then its
+        //      arithmetic and stores (a store may alias a later load for all the compiler
+        //      knows, so one token at a time would pay the shared-memory latency per token) ----
+        float acc = hh ? sHalf[d] : 0.f, mx = 0.f;
+#pragma unroll
+        for (int i0 = 0; i0 < 32; i0 += 8) {
+            float kt[8], qt[8], bt[8];
+#pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int t = 8 * tg + i;
-                float f[8];
-                if (t < n) {
-                    const size_t e = (row0 + t) * DV + 8 * cg;
-                    float fv[8], fw[8];
-                    bf16x8_to_f32(*reinterpret_cast<const uint4 *>(V + e), fv);
-                    if (vec_w) {
-                        bf16x8_to_f32(*reinterpret_cast<const uint4 *>(Wg + e), fw);
-                    } else {
-                        const float ws = __bfloat162float(Wsc[row0 + t]);
+                const int t = 32 * hh + i0 + i;
+                const bool in = t < n;
+                const uint32_t okh = tile_off(128, t, d), oqg = tile_off(128, 64 + t, d), okb = tile_off(64, t, d);
+                kt[i] = in ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_KB + okb)) : 0.f;
+                qt[i] = in ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_QK + oqg)) : 0.f;
+                bt[i] = !in ? 0.f
+                        : vec_b ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_QK + okh))
+                                : sBeta[t];
+            }
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) fw[j] = ws;
-                    }
+            for (int i = 0; i < 8; ++i) {
+                const int t = 32 * hh + i0 + i;
+                acc += gv[i0 + i];
+                mx = fmaxf(mx, fabsf(acc));
+                const float eg = __expf(acc);
+                st_bf16(sm + OFF_QK + tile_off(128, t, d), bt[i] * kt[i] * eg);
+                st_bf16(sm + OFF_QK + tile_off(128, 64 + t, d), qt[i] * eg);
+                st_bf16(sm + OFF_KB + tile_off(64, t, d), kt[i] * rcp_approx(eg));
+            }
+        }
+        if (hh == 1) sEgc[d] = __expf(acc);   // gamma at the chunk's end (tokens past it add zero)
+        if (tid == 0) reinterpret_cast<int4 *>(sm + OFF_META + 512)[0] = make_int4(0, 0, 0, 0);
+        // ---- w.v in place over v (fp32 products, one bf16 rounding; zero past the end) ----
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = fw[j] * fv[j];
-                } else {
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * tg + i;
+            const uint32_t addr = sbase + OFF_WV + tile_chunk(64, t, cg);
+            float f[8], fw[8];
+            uint4 u;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
+            bf16x8_to_f32(u, f);
+            if (vec_w) {
+                bf16x8_to_f32(wr[i], fw);
+            } else {
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) f[j] = 0.f;
+                for (int j = 0; j < 8; ++j) fw[j] = wsc[i];
+            }
+            const bool in = t < n;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] = in ? fw[j] * f[j] : 0.f;
+            st_chunk(addr, f);
+        }
+        if (sync_all_or(mx > kFastLimit)) {
+            // strong decay: listed for the exact kernel, which writes this chunk's record
+            if (tid == 0) list[1 + atomicAdd(list, 1)] = unit;
+            sync_all();
+            continue;
+        }
+        fence_async_smem();
+        sync_all();
+        // ---- [A; P] = [Kh; Qg] Kb^T ----
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id = idesc_bf16(128, 64, false, false, false);
+#pragma unroll
+            for (int s = 0; s < DK / 16; ++s)
+                mma_bf16(tmem + TM_AP, desc_kmajor(sbase + OFF_QK, 128, 0, s), desc_kmajor(sbase + OFF_KB, 64, 0, s),
+                         id, s > 0);
+            mma_commit(bar);
+        }
+        ++n_mma;
+        ok = sync_all_and(tid != 0 || mbar_wait(bar, (n_mma - 1) & 1, wait_limit));
+        if (!ok) break;
+        tc_fence_after();
+        {
+            // A (fp32, strictly lower) -> inverse scratch; P (bf16, lower incl.) -> its tile
+            const int r = quarter * 32 + lane, j0 = (warp >> 2) * 32;
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_AP + j0, x);
+            tmem_wait_ld();
+            if (r < 64) {
+                float4 *dst = reinterpret_cast<float4 *>(sA32 + r * tri::LD + j0);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float y[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) y[u] = (j0 + 4 * q + u < r) ? x[4 * q + u] : 0.f;
+                    dst[q] = make_float4(y[0], y[1], y[2], y[3]);
                 }
-                st_chunk(sbase + OFF_WV + tile_chunk(64, t, cg), f);
+            } else {
+                const int t = r - 64;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float f[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) f[j] = (j0 + h * 8 + j <= t) ? x[h * 8 + j] : 0.f;
+                    st_chunk(sbase + OFF_P + tile_chunk(64, t, j0 / 8 + h), f);
+                }
             }
         }
         fence_async_smem();
-        __syncthreads();
+        tc_fence_before();
+        sync_all();
+        // ---- T = (I + A)^-1 by warps 0-3, straight into the bf16 tile; meanwhile thread 128
+        //      sends the record's Qg, Kb, P and tail (final once [A; P] is read out) ----
+        if (warp < 4) {
+            tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
+        } else if (tid == 128) {
+            // Qg: rows 64..127 of each column block of the stacked tile = a 64-row tile
+            bulk_s2g(rec + REC_QG, sbase + OFF_QK + 8192, 8192);
+            bulk_s2g(rec + REC_QG + 8192, sbase + OFF_QK + 16384 + 8192, 8192);
+            bulk_s2g(rec + REC_KB, sbase + OFF_KB, 16384);
+            bulk_s2g(rec + REC_P, sbase + OFF_P, 8192);
+            bulk_s2g(rec + REC_EGC, sbase + OFF_META, 528);
+            bulk_commit();
+        }
+        fence_async_smem();
+        sync_all();
         // ---- W^T = Kh^T T^T and U^T = (w.v)^T T^T (A operands MN-major) ----
         if (tid == 0) {
             tc_fence_after();
@@ -246,50 +334,55 @@ __global__ void __launch_bounds__(kThreads, 2)
                          id, s > 0);
             mma_commit(bar);
         }
-        ok = __syncthreads_and(tid != 0 || mbar_wait(bar, 1u, wait_limit));
-    }
-    if (ok) {
+        ++n_mma;
+        ok = sync_all_and(tid != 0 || mbar_wait(bar, (n_mma - 1) & 1, wait_limit));
+        if (!ok) break;
         tc_fence_after();
-        // W^T rows (warps 0-3) over the inverse's dead scratch, U^T rows (warps 4-7) over w.v
-        const int r = quarter * 32 + lane;
-        const uint32_t col = warp < 4 ? TM_W : TM_U;
-        const uint32_t tile = sbase + (warp < 4 ? OFF_A32 : OFF_WV);
+        {
+            // W^T rows (warps 0-3) over the inverse's dead scratch, U^T rows (warps 4-7) over w.v
+            const int r = quarter * 32 + lane;
+            const uint32_t col = warp < 4 ? TM_W : TM_U;
+            const uint32_t tile = sbase + (warp < 4 ? OFF_A32 : OFF_WV);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float x[32];
-            tmem_ld32(tmem + lane_base + col + 32 * h, x);
-            tmem_wait_ld();
+            for (int h = 0; h < 2; ++h) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + col + 32 * h, x);
+                tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float f[8];
+                for (int q = 0; q < 4; ++q) {
+                    float f[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) f[j] = x[8 * q + j];
-                st_chunk(tile + tile_chunk(128, r, 4 * h + q), f);
+                    for (int j = 0; j < 8; ++j) f[j] = x[8 * q + j];
+                    st_chunk(tile + tile_chunk(128, r, 4 * h + q), f);
+                }
             }
         }
         fence_async_smem();
-        __syncthreads();
+        tc_fence_before();
+        sync_all();
         if (tid == 0) {
             bulk_s2g(rec + REC_WT, sbase + OFF_A32, 16384);
             bulk_s2g(rec + REC_UT, sbase + OFF_WV, 16384);
-            // Qg: rows 64..127 of each column block of the stacked tile = a 64-row tile
-            bulk_s2g(rec + REC_QG, sbase + OFF_QK + 8192, 8192);
-            bulk_s2g(rec + REC_QG + 8192, sbase + OFF_QK + 16384 + 8192, 8192);
-            bulk_s2g(rec + REC_KB, sbase + OFF_KB, 16384);
-            bulk_s2g(rec + REC_P, sbase + OFF_P, 8192);
-            bulk_s2g(rec + REC_EGC, sbase + OFF_META, 528);
             bulk_commit();
-            bulk_wait_all();
         }
-    } else if (tid == 0) {
-        // a bounded wait expired: record it and give the tensor cores a bounded time to finish
-        atomicExch(&g_tp_error, 1);
-        mma_commit(bar);
-        mbar_wait(bar, 0u, wait_limit);
-        mbar_wait(bar, 1u, wait_limit);
+        // the copies have read shared memory (each thread waits for its own) before the
+        // next chunk's tiles arrive there; they land by the kernel's end
+        if (tid == 0 || tid == 128) bulk_wait_read_all();
+        sync_all();
     }
+    if (!ok && tid == 0) {
+        // a bounded wait expired: record it, and give the tile copies and the tensor cores a
+        // bounded time to finish (one more commit covers every MMA issued; commits complete
+        // in order, so phases n-1 and then n of it are waited for)
+        atomicExch(&g_tp_error, 1);
+        mbar_wait(bar_ld, (uint32_t)(ld_issued - 1) & 1, wait_limit);
+        mma_commit(bar);
+        if (n_mma >= 1) mbar_wait(bar, (n_mma - 1) & 1, wait_limit);
+        mbar_wait(bar, n_mma & 1, wait_limit);
+    }
+    if (tid == 0 || tid == 128) bulk_wait_read_all();
     tc_fence_before();
-    __syncthreads();
+    sync_all();
     tc_fence_after();
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
@@ -427,17 +520,42 @@ unsigned long long list_bytes(int B, int H, int T) {
     return (n * 4 + 15) / 16 * 16;
 }
 
+namespace {
+
+// [rows][128] bf16 row-major, box {64 elements, 64 rows}, 128-byte swizzle, zero fill
+bool encode_rows(CUtensorMap *m, const void *base, unsigned long long rows) {
+    auto fn = tensor_map_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)DK, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)DK * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)C};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 gdr_status_t launch_wy_prep(const ChunkArgs &a, unsigned char *records, int *list, cudaStream_t s) {
     const long long units = (long long)a.B * a.H * ((a.T + C - 1) / C);
     if (units <= 0) return GDR_OK;
+    const unsigned long long rows = (unsigned long long)a.B * a.H * a.T;
+    PrepMaps tm;
+    memset(&tm, 0, sizeof(tm));
+    if (!encode_rows(&tm.q, a.q, rows) || !encode_rows(&tm.k, a.k, rows) || !encode_rows(&tm.v, a.v, rows) ||
+        (mode_b_vec(a.mode) && !encode_rows(&tm.b, a.b, rows)))
+        return GDR_ERR_CUDA;
     if (cudaFuncSetAttribute(wy_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
             cudaSuccess ||
         cudaFuncSetAttribute(wy_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, XSMEM) != cudaSuccess)
         return GDR_ERR_CUDA;
-    wy_prep_kernel<<<(unsigned)units, kThreads, SMEM_BYTES, s>>>(a, records, list);
     int sms = 148, dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return GDR_ERR_CUDA;
+    // persistent: two CTAs per SM (their shared memory and TMEM fit twice), chunks in turn
+    const long long grid = units < 2LL * sms ? units : 2LL * sms;
+    wy_prep_kernel<<<(unsigned)grid, kThreads, SMEM_BYTES, s>>>(a, records, list, tm);
     wy_exact_kernel<<<(unsigned)(units < sms ? units : sms), kThreads, XSMEM, s>>>(a, records, list);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }

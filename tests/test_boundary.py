@@ -148,9 +148,11 @@ def test_two_phase_workspace_size_and_planner(L):
     assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 64, 64, 64, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 128, 128, 32, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 128, 128, 64, 0) == 0
-    # the planner (this host has no GPU: 148 SMs assumed) takes the two-phase path when the
-    # sequence-heads are too few to fill the GPU, and the fused kernel when they fill it
-    assert gdr.gdr_chunk_fwd_two_phase_segments(4, 16, 2048, 128, 128, 64, 1) >= 1
+    # the planner (this host has no GPU: 148 SMs assumed), with its measured constants, takes
+    # the two-phase path for few sequence-heads over long sequences, and the fused kernel
+    # when the sequence-heads fill the GPU or the sequences are short (T = 2K: phase one's
+    # latency-bound chunks cost more than the fused kernel saves)
+    assert gdr.gdr_chunk_fwd_two_phase_segments(4, 16, 2048, 128, 128, 64, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 128, 128, 64, 1) > 1
     assert gdr.gdr_chunk_fwd_two_phase_segments(8, 16, 4096, 128, 128, 64, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 64, 64, 64, 1) == 0
