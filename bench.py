@@ -438,14 +438,24 @@ def setup_workload(name, rank, dev, decode_steps=None):
         if chunk_bytes(wl, mode) <= 126e6:
             flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         dt_code = 1 if wl.dtype == "bf16" else 0
-        nseg = gdr.gdr_chunk_fwd_split_segments(wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.chunk, dt_code)
+        # the library's planner picks the path: the two-phase forward (few sequence-heads,
+        # long sequences), the fused kernel with a sequence split, or the fused kernel alone
+        n2 = gdr.gdr_chunk_fwd_two_phase_segments(wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.chunk, dt_code)
+        nseg = n2 if n2 > 0 else gdr.gdr_chunk_fwd_split_segments(wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.chunk,
+                                                                   dt_code)
         ws = None
-        if nseg > 1:
+        if n2 > 0:
+            ws = torch.empty(gdr.gdr_chunk_fwd_two_phase_workspace(wl.B, wl.H, wl.T, wl.dk, wl.dv, wl.chunk, n2),
+                             dtype=torch.uint8, device=dev)
+        elif nseg > 1:
             ws = torch.empty(gdr.gdr_chunk_fwd_split_workspace(wl.B, wl.H, wl.dk, wl.dv, nseg),
                              dtype=torch.uint8, device=dev)
 
         def fwd():
-            if nseg > 1:
+            if n2 > 0:
+                gdr.chunk_fwd_two_phase(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"],
+                                        mode=mode, chunk=wl.chunk, nseg=n2, workspace=ws, o=o, S_T=ST)
+            elif nseg > 1:
                 gdr.chunk_fwd_split(d["q"], d["k"], d["v"], d["g"], d["b"], d["w"], d["S0"],
                                     mode=mode, chunk=wl.chunk, nseg=nseg, workspace=ws, o=o, S_T=ST)
             else:
@@ -456,12 +466,20 @@ def setup_workload(name, rank, dev, decode_steps=None):
             if flush is not None:
                 flush.zero_()
             fwd()
-        # one step = the whole forward; with a sequence split it is three launches (state
-        # pass, combine, output pass) and the step is the unit of the roofline
+        # one step = the whole forward, the unit of the roofline: with a sequence split three
+        # launches (state pass, combine, output pass); the two-phase forward is phase one (two
+        # launches, after a memset of its list count) and one state pass, or three with a split
+        if n2 > 0:
+            launches = 2 + (3 if n2 > 1 else 1)
+            kern = (f"gdr wy_prep_kernel + wy_exact_kernel + state_pass_kernel"
+                    + (f" x2 + split_combine_kernel (two-phase, {n2} segments)" if n2 > 1 else " (two-phase)"))
+        else:
+            launches = 3 if nseg > 1 else 1
+            kern = kernel_name(wl, mode) if nseg <= 1 else \
+                f"gdr chunk_tc_kernel x2 + split_combine_kernel (sequence split, {nseg} segments)"
         r.update(fwd=fwd, step=step, flush=flush, units=wl.units, bytes_per_launch=chunk_bytes(wl, mode),
-                 launches_per_step=3 if nseg > 1 else 1, flops=chunk_flops(wl), nseg=nseg, inp=inp,
-                 out=(o, ST), kernel=kernel_name(wl, mode) if nseg <= 1 else
-                 f"gdr chunk_tc_kernel x2 + split_combine_kernel (sequence split, {nseg} segments)")
+                 launches_per_step=launches, flops=chunk_flops(wl), nseg=nseg, inp=inp,
+                 out=(o, ST), kernel=kern, two_phase=n2 > 0)
     return r
 
 

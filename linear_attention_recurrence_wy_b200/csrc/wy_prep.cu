@@ -84,6 +84,13 @@ __device__ __forceinline__ bool sync_all_or(bool v) {
     return r;
 }
 
+// T = (I + A)^-1 by warps 0-3 (tri_inverse.cuh) as a call of its own: inlined into this
+// kernel, whose other phases keep many registers live, its substitution chains ran several
+// times slower than on their own
+__device__ __noinline__ void invert(float *sA32, float *sX, int warp, int lane, uint32_t t_tile) {
+    tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{t_tile});
+}
+
 __device__ __forceinline__ void st_bf16(unsigned char *p, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
 }
@@ -308,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ---- T = (I + A)^-1 by warps 0-3, straight into the bf16 tile; meanwhile thread 128
         //      sends the record's Qg, Kb, P and tail (final once [A; P] is read out) ----
         if (warp < 4) {
-            tri::inverse64(sA32, sA32, sX, warp, lane, Bar128{}, TileOut{sbase + OFF_T});
+            invert(sA32, sX, warp, lane, sbase + OFF_T);
         } else if (tid == 128) {
             // Qg: rows 64..127 of each column block of the stacked tile = a 64-row tile
             bulk_s2g(rec + REC_QG, sbase + OFF_QK + 8192, 8192);
