@@ -16,16 +16,80 @@ namespace gdr {
 namespace {
 
 constexpr int DK = 128, DV = 128, COLS = 16;   // one CTA: one sequence-head, 16 state columns
+constexpr int MLD = DK + 4;                    // padded fp32 row stride of a staged map
+constexpr int CHAIN_SMEM = (2 * DK * MLD + DK * COLS) * 4;   // two maps, the state slice
+
+// One map M (dk x dk fp32, row-major) -> shared memory by asynchronous 16-byte copies, all
+// 256 threads, consecutive threads on consecutive 16 bytes; one commit group per map.
+__device__ __forceinline__ void stage_map(float *dst, const float *M, int tid) {
+#pragma unroll
+    for (int j = 0; j < DK * DK / 4 / 256; ++j) {
+        const int f = tid + 256 * j, row = f >> 5, c4 = f & 31;
+        const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + row * MLD + 4 * c4);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(M + (size_t)row * DK + 4 * c4)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// wait until at most n commit groups of this thread are still in flight, then a CTA barrier
+template <int n>
+__device__ __forceinline__ void wait_maps() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory");
+    __syncthreads();
+}
+
+// S <- M S + L on the CTA's 16-column slice: thread (row i, half h) forms columns 8h .. 8h+7
+// of row i; M is a staged map (rows MLD apart), L the slice's rows in global memory.  The
+// slice's rows are 16 floats apart, so a thread reads its eight columns of a row of S as two
+// 16-byte loads, which every thread of the same half shares (a broadcast).
+__device__ __forceinline__ void apply_map(float (*S)[COLS], const float *sM, const float *L, int i, int h) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = L[j];
+    const float *m = sM + i * MLD;
+#pragma unroll 2
+    for (int k0 = 0; k0 < DK; k0 += 4) {
+        const float4 mv = *reinterpret_cast<const float4 *>(m + k0);
+        const float mk[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const float4 s0 = *reinterpret_cast<const float4 *>(&S[k0 + kk][8 * h]);
+            const float4 s1 = *reinterpret_cast<const float4 *>(&S[k0 + kk][8 * h + 4]);
+            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = fmaf(mk[kk], sv[j], acc[j]);
+        }
+    }
+    __syncthreads();   // every thread has read S
+    *reinterpret_cast<float4 *>(&S[i][8 * h]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    *reinterpret_cast<float4 *>(&S[i][8 * h + 4]) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+    __syncthreads();
+}
+
+// Dynamic shared memory: the two map buffers, then the state slice.
+struct ChainSmem {
+    float *m0, *m1;
+    float (*S)[COLS];
+};
+__device__ __forceinline__ ChainSmem chain_smem() {
+    extern __shared__ __align__(16) float chain_raw[];
+    return {chain_raw, chain_raw + DK * MLD, reinterpret_cast<float (*)[COLS]>(chain_raw + 2 * DK * MLD)};
+}
 
 __global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
     const int slices = DV / COLS;
     const int bh = blockIdx.x / slices, c0 = (blockIdx.x % slices) * COLS;
     const int tid = threadIdx.x, i = tid >> 1, h = tid & 1;   // row i, columns c0 + 8h ..
-    __shared__ float S[DK][COLS + 1];
     if (!GDR_IN_BOUNDS(bh < a.B * a.H, 501)) return;   // debug build: uniform, before any barrier
+    const ChainSmem sm = chain_smem();
+    float (*S)[COLS] = sm.S;
     const size_t head = (size_t)bh * a.nseg * DK * DV;
     const size_t seg_sz = (size_t)DK * DV;
     float *sstart = a.ws_sstart + head;
+    // the maps of segments 1 .. nseg-2 are applied in turn; the first travels now, each next
+    // one while the current one is applied
+    const int last = a.nseg - 2;
+    if (last >= 1) stage_map(sm.m0, a.ws_m + head + seg_sz, tid);
     // S_start(0) = S0 (zeros if absent): the second pass reads every start state from here
     for (int j = 0; j < 8; ++j) {
         const int c = c0 + 8 * h + j;
@@ -35,24 +99,15 @@ __global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
     __syncthreads();
     for (int s = 1; s < a.nseg; ++s) {
         for (int j = 0; j < 8; ++j) sstart[s * seg_sz + (size_t)i * DV + c0 + 8 * h + j] = S[i][8 * h + j];
-        if (s == a.nseg - 1) break;
-        const float *M = a.ws_m + head + s * seg_sz + (size_t)i * DK;
-        const float *L = a.ws_send + head + s * seg_sz + (size_t)i * DV + c0 + 8 * h;
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = L[j];
-        for (int k0 = 0; k0 < DK; k0 += 4) {
-            const float4 m = *reinterpret_cast<const float4 *>(M + k0);
-            const float mk[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = fmaf(mk[kk], S[k0 + kk][8 * h + j], acc[j]);
+        if (s > last) break;
+        float *cur = (s & 1) ? sm.m0 : sm.m1;
+        if (s < last) {
+            stage_map((s & 1) ? sm.m1 : sm.m0, a.ws_m + head + (s + 1) * seg_sz, tid);
+            wait_maps<1>();   // this segment's map has landed; the next one may still travel
+        } else {
+            wait_maps<0>();
         }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) S[i][8 * h + j] = acc[j];
-        __syncthreads();
+        apply_map(S, cur, a.ws_send + head + s * seg_sz + (size_t)i * DV + c0 + 8 * h, i, h);
     }
 }
 
@@ -64,7 +119,6 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *M_all, 
     const int slices = DV / COLS;
     const int bh = blockIdx.x / slices, c0 = (blockIdx.x % slices) * COLS;
     const int tid = threadIdx.x, i = tid >> 1, h = tid & 1;   // row i, columns c0 + 8h ..
-    __shared__ float S[DK][COLS + 1];
     const size_t st = (size_t)DK * DV;                       // one state
     const size_t per = (size_t)BH * st;                      // one holder's block of states
     if (!GDR_IN_BOUNDS(bh < BH, 502)) return;                // debug build: uniform, before any barrier
@@ -73,28 +127,27 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *M_all, 
         for (int j = 0; j < 8; ++j) out[j] = S0 ? S0[bh * st + (size_t)i * DV + c0 + 8 * h + j] : 0.f;
         return;
     }
+    const ChainSmem sm = chain_smem();
+    float (*S)[COLS] = sm.S;
+    const int last = r - 1;   // maps of holders 1 .. r-1
+    if (last >= 1) stage_map(sm.m0, M_all + per + bh * st, tid);
     for (int j = 0; j < 8; ++j) S[i][8 * h + j] = S_all[bh * st + (size_t)i * DV + c0 + 8 * h + j];   // S_end(0)
     __syncthreads();
-    for (int s = 1; s < r; ++s) {
-        const float *M = M_all + s * per + bh * st + (size_t)i * DK;
-        const float *L = S_all + s * per + bh * st + (size_t)i * DV + c0 + 8 * h;
-        float acc[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = L[j];
-        for (int k0 = 0; k0 < DK; k0 += 4) {
-            const float4 m = *reinterpret_cast<const float4 *>(M + k0);
-            const float mk[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = fmaf(mk[kk], S[k0 + kk][8 * h + j], acc[j]);
+    for (int s = 1; s <= last; ++s) {
+        float *cur = (s & 1) ? sm.m0 : sm.m1;
+        if (s < last) {
+            stage_map((s & 1) ? sm.m1 : sm.m0, M_all + (s + 1) * per + bh * st, tid);
+            wait_maps<1>();
+        } else {
+            wait_maps<0>();
         }
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) S[i][8 * h + j] = acc[j];
-        __syncthreads();
+        apply_map(S, cur, S_all + s * per + bh * st + (size_t)i * DV + c0 + 8 * h, i, h);
     }
     for (int j = 0; j < 8; ++j) out[j] = S[i][8 * h + j];
+}
+
+bool chain_attr_set(const void *kern) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, CHAIN_SMEM) == cudaSuccess;
 }
 
 }  // namespace
@@ -102,12 +155,14 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *M_all, 
 gdr_status_t launch_segment_chain(const float *M_all, const float *S_all, const float *S0, float *S_start, int R,
                                   int r, int BH, cudaStream_t s) {
     (void)R;
-    segment_chain_kernel<<<(unsigned)(BH * (DV / COLS)), 256, 0, s>>>(M_all, S_all, S0, S_start, r, BH);
+    if (!chain_attr_set((const void *)segment_chain_kernel)) return GDR_ERR_CUDA;
+    segment_chain_kernel<<<(unsigned)(BH * (DV / COLS)), 256, CHAIN_SMEM, s>>>(M_all, S_all, S0, S_start, r, BH);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 
 gdr_status_t launch_split_combine(const ChunkArgs &a, cudaStream_t s) {
-    split_combine_kernel<<<(unsigned)(a.B * a.H * (DV / COLS)), 256, 0, s>>>(a);
+    if (!chain_attr_set((const void *)split_combine_kernel)) return GDR_ERR_CUDA;
+    split_combine_kernel<<<(unsigned)(a.B * a.H * (DV / COLS)), 256, CHAIN_SMEM, s>>>(a);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -94,6 +94,11 @@ __device__ __noinline__ void invert(float *sA32, float *sX, int warp, int lane, 
 __device__ __forceinline__ void st_bf16(unsigned char *p, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(p) = __float2bfloat16_rn(x);
 }
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 u;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
+    return u;
+}
 
 // Tensor maps of the bf16 inputs read as tiles: [B*H*T rows][128] row-major, box {64, 64}
 // with the 128-byte swizzle, so a box lands in shared memory in the operand tile layout of
@@ -144,8 +149,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const uint32_t tmem = *tslot;
     const uint32_t wait_limit = a.wait_limit;
-    const int d = tid & 127, hh = tid >> 7;      // scan and build: key channel d, tokens 32 hh ..
-    const int tg = tid >> 4, cg = tid & 15;      // write gate: tokens 4 tg .., channels 8 cg ..
+    // scan and build: thread (token group tg, channel group cg) owns tokens 4 tg .. 4 tg + 3
+    // and key (and value) channels 8 cg .. 8 cg + 7; a warp holds eight token groups of four
+    // channel groups, so its 16-byte tile accesses spread over all the banks
+    const int tgl = lane >> 2, hh = warp >> 2;   // token group within the warp, half of the chunk
+    const int tg = 8 * hh + tgl, cg = 4 * (warp & 3) + (lane & 3);
     bool ok = true;
     uint32_t n_mma = 0;                          // commits on bar so far (its phase parity)
     int ld_issued = 0;                           // tile-copy batches issued (thread 0)
@@ -178,89 +186,145 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         __syncwarp();
 
-        // ---- global loads issued up front: g_log of (channel d, tokens 32 hh ..), the write
-        //      gate of (tokens 4 tg .., channels 8 cg ..), a scalar erase gate per token ----
-        float gv[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int t = 32 * hh + i;
-            gv[i] = t < n ? (vec_g ? a.g[(row0 + t) * DK + d] : a.g[row0 + t]) : 0.f;
-        }
+        // ---- global loads issued up front: g_log and the write gate of this thread's four
+        //      tokens and eight channels, a scalar erase gate per token ----
+        float gv[4][8];
         uint4 wr[4];
         float wsc[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * tg + i;
+            const bool in = t < n;
             wr[i] = make_uint4(0, 0, 0, 0);
             wsc[i] = 0.f;
-            if (t < n) {
+            if (vec_g) {
+                float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0;
+                if (in) {
+                    const float4 *gp = reinterpret_cast<const float4 *>(a.g + (row0 + t) * DK + 8 * cg);
+                    g0 = gp[0];
+                    g1 = gp[1];
+                }
+                gv[i][0] = g0.x; gv[i][1] = g0.y; gv[i][2] = g0.z; gv[i][3] = g0.w;
+                gv[i][4] = g1.x; gv[i][5] = g1.y; gv[i][6] = g1.z; gv[i][7] = g1.w;
+            } else {
+                const float x = in ? a.g[row0 + t] : 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) gv[i][j] = x;
+            }
+            if (in) {
                 if (vec_w) wr[i] = *reinterpret_cast<const uint4 *>(Wg + (row0 + t) * DV + 8 * cg);
                 else wsc[i] = __bfloat162float(Wsc[row0 + t]);
             }
         }
         if (!vec_b && tid < C) sBeta[tid] = tid < n ? __bfloat162float(Bg[row0 + tid]) : 0.f;
-        {
-            float sum = 0.f;
+        // gamma over this half of the chunk: the thread's own four tokens, then an inclusive
+        // scan over the warp's eight token groups (shuffles); the first half's totals go to
+        // shared memory for the second half
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sum += gv[i];
-            if (hh == 0) sHalf[d] = sum;
+        for (int i = 1; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) gv[i][j] += gv[i - 1][j];
+        {
+            float pre[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pre[j] = gv[3][j];
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float y = __shfl_up_sync(0xffffffffu, pre[j], 4 * o);
+                    if (tgl >= o) pre[j] += y;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float excl = pre[j] - gv[3][j];   // tokens of the earlier groups of this half
+#pragma unroll
+                for (int i = 0; i < 4; ++i) gv[i][j] += excl;
+            }
+            if (hh == 0 && tgl == 7) {
+                float4 *dst = reinterpret_cast<float4 *>(sHalf + 8 * cg);
+                dst[0] = make_float4(pre[0], pre[1], pre[2], pre[3]);
+                dst[1] = make_float4(pre[4], pre[5], pre[6], pre[7]);
+            }
         }
         ok = sync_all_and(tid != 0 || mbar_wait(bar_ld, (uint32_t)(it & 1), wait_limit));
         if (!ok) break;
-
-        // ---- gamma and the operands, in place: thread (d, hh) scans key channel d over
-        //      tokens 32 hh .. 32 hh + 31 (from the first half's sum) and turns b, q, k into
-        //      Kh, Qg, Kb.  In batches of eight tokens: every load of a batch first, then its
-        //      arithmetic and stores (a store may alias a later load for all the compiler
-        //      knows, so one token at a time would pay the shared-memory latency per token) ----
-        float acc = hh ? sHalf[d] : 0.f, mx = 0.f;
-#pragma unroll
-        for (int i0 = 0; i0 < 32; i0 += 8) {
-            float kt[8], qt[8], bt[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = 32 * hh + i0 + i;
-                const bool in = t < n;
-                const uint32_t okh = tile_off(128, t, d), oqg = tile_off(128, 64 + t, d), okb = tile_off(64, t, d);
-                kt[i] = in ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_KB + okb)) : 0.f;
-                qt[i] = in ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_QK + oqg)) : 0.f;
-                bt[i] = !in ? 0.f
-                        : vec_b ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_QK + okh))
-                                : sBeta[t];
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = 32 * hh + i0 + i;
-                acc += gv[i0 + i];
-                mx = fmaxf(mx, fabsf(acc));
-                const float eg = __expf(acc);
-                st_bf16(sm + OFF_QK + tile_off(128, t, d), bt[i] * kt[i] * eg);
-                st_bf16(sm + OFF_QK + tile_off(128, 64 + t, d), qt[i] * eg);
-                st_bf16(sm + OFF_KB + tile_off(64, t, d), kt[i] * rcp_approx(eg));
-            }
+        if (tid == 32 && unit + (int)gridDim.x < units) {
+            // this chunk's tiles have landed: the CTA's next chunk now travels to L2 while this
+            // one is worked on (every CTA loads at the same time at first, so a prefetch issued
+            // earlier would only compete with the loads of the current chunk)
+            const int un = unit + (int)gridDim.x, bn = un / nch, cn = un % nch;
+            const int nn = min(C, a.T - cn * C);
+            const size_t e = ((size_t)bn * a.T + (size_t)cn * C) * DK;
+            prefetch_l2((const __nv_bfloat16 *)a.q + e, (uint32_t)nn * DK * 2);
+            prefetch_l2((const __nv_bfloat16 *)a.k + e, (uint32_t)nn * DK * 2);
+            prefetch_l2((const __nv_bfloat16 *)a.v + e, (uint32_t)nn * DV * 2);
+            if (vec_b) prefetch_l2(Bg + e, (uint32_t)nn * DK * 2);
+            if (vec_w) prefetch_l2(Wg + e, (uint32_t)nn * DV * 2);
+            if (vec_g) prefetch_l2(a.g + e, (uint32_t)nn * DK * 4);
         }
-        if (hh == 1) sEgc[d] = __expf(acc);   // gamma at the chunk's end (tokens past it add zero)
-        if (tid == 0) reinterpret_cast<int4 *>(sm + OFF_META + 512)[0] = make_int4(0, 0, 0, 0);
-        // ---- w.v in place over v (fp32 products, one bf16 rounding; zero past the end) ----
+
+        // ---- the operands in place, 16 bytes at a time: b, q, k of the thread's four tokens
+        //      and eight channels become Kh, Qg, Kb, and v becomes w.v (fp32 products, one bf16
+        //      rounding; zero past the end) ----
+        float mx = 0.f;
+        if (hh == 1) {
+            const float4 *src = reinterpret_cast<const float4 *>(sHalf + 8 * cg);
+            const float4 h0 = src[0], h1 = src[1];
+            const float hs[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) gv[i][j] += hs[j];
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * tg + i;
-            const uint32_t addr = sbase + OFF_WV + tile_chunk(64, t, cg);
-            float f[8], fw[8];
-            uint4 u;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w) : "r"(addr));
-            bf16x8_to_f32(u, f);
+            const bool in = t < n;
+            const uint32_t okh = sbase + OFF_QK + tile_chunk(128, t, cg);
+            const uint32_t oqg = sbase + OFF_QK + tile_chunk(128, 64 + t, cg);
+            const uint32_t okb = sbase + OFF_KB + tile_chunk(64, t, cg);
+            const uint32_t owv = sbase + OFF_WV + tile_chunk(64, t, cg);
+            float fk[8], fq[8], fb[8], fv[8], fw[8];
+            bf16x8_to_f32(sel(in, ld_shared_v4(okb)), fk);
+            bf16x8_to_f32(sel(in, ld_shared_v4(oqg)), fq);
+            bf16x8_to_f32(sel(in, ld_shared_v4(owv)), fv);
+            if (vec_b) {
+                bf16x8_to_f32(sel(in, ld_shared_v4(okh)), fb);
+            } else {
+                const float beta = sBeta[t];   // zero past the end
+#pragma unroll
+                for (int j = 0; j < 8; ++j) fb[j] = beta;
+            }
             if (vec_w) {
                 bf16x8_to_f32(wr[i], fw);
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) fw[j] = wsc[i];
             }
-            const bool in = t < n;
+            float kh[8], qg[8], kb[8], wv[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) f[j] = in ? fw[j] * f[j] : 0.f;
-            st_chunk(addr, f);
+            for (int j = 0; j < 8; ++j) {
+                mx = fmaxf(mx, fabsf(gv[i][j]));
+                const float eg = __expf(gv[i][j]);
+                kh[j] = fb[j] * fk[j] * eg;
+                qg[j] = fq[j] * eg;
+                kb[j] = fk[j] * rcp_approx(eg);
+                wv[j] = fw[j] * fv[j];
+            }
+            st_chunk(okh, kh);
+            st_chunk(oqg, qg);
+            st_chunk(okb, kb);
+            st_chunk(owv, wv);
         }
+        // e^gamma at the chunk's end (tokens past it add zero): the last token group's
+        if (tg == 15) {
+            float4 *dst = reinterpret_cast<float4 *>(sEgc + 8 * cg);
+            dst[0] = make_float4(__expf(gv[3][0]), __expf(gv[3][1]), __expf(gv[3][2]), __expf(gv[3][3]));
+            dst[1] = make_float4(__expf(gv[3][4]), __expf(gv[3][5]), __expf(gv[3][6]), __expf(gv[3][7]));
+        }
+        if (tid == 0) reinterpret_cast<int4 *>(sm + OFF_META + 512)[0] = make_int4(0, 0, 0, 0);
         if (sync_all_or(mx > kFastLimit)) {
             // strong decay: listed for the exact kernel, which writes this chunk's record
             if (tid == 0) list[1 + atomicAdd(list, 1)] = unit;
