@@ -142,11 +142,11 @@ double fused_split_time(int units, int sms, int nchunks, int *nseg_out) {
 
 // The two-phase forward, in the same unit (constants measured on B200 with per-phase clock
 // stamps): phase one over every chunk, two persistent CTAs per SM, a wave of two chunks per
-// SM taking kPrep (its latency-bound per-chunk path, ~30 K cycles), or bound by its traffic (the inputs, at most 112 KB per chunk, and
+// SM taking kPrep (its latency-bound per-chunk path, ~21 K cycles), or bound by its traffic (the inputs, at most 112 KB per chunk, and
 // the 73 KB record it writes); then the state pass, whole or split like the fused kernel,
 // each CTA kState per chunk plus kFix to start, or bound by the records it reads and the
 // output it writes.  kBytes: HBM bytes moved in one fused chunk period (~6 TB/s x 5 us).
-constexpr double kPrep = 3.5, kState = 0.37, kFix = 0.5, kBytes = 34e6;
+constexpr double kPrep = 2.1, kState = 0.37, kFix = 0.5, kBytes = 34e6;
 constexpr double kIn = 112.0 * 1024, kRec = 74752, kOut = 16.0 * 1024;
 double waves(long long ctas, int sms) { return (double)((ctas + sms - 1) / sms); }
 double two_phase_time(int units, int sms, int nchunks, int *nseg_out) {

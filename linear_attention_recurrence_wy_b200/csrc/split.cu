@@ -17,17 +17,27 @@ namespace {
 
 constexpr int DK = 128, DV = 128, COLS = 16;   // one CTA: one sequence-head, 16 state columns
 constexpr int MLD = DK + 4;                    // padded fp32 row stride of a staged map
-constexpr int CHAIN_SMEM = (2 * DK * MLD + DK * COLS) * 4;   // two maps, the state slice
+// two maps and their segments' end-state slices (double-buffered), the state slice
+constexpr int CHAIN_SMEM = (2 * DK * MLD + 2 * DK * COLS + DK * COLS) * 4;
 
-// One map M (dk x dk fp32, row-major) -> shared memory by asynchronous 16-byte copies, all
-// 256 threads, consecutive threads on consecutive 16 bytes; one commit group per map.
-__device__ __forceinline__ void stage_map(float *dst, const float *M, int tid) {
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+// One map M (dk x dk fp32, row-major) and the CTA's 16-column slice of the segment's local
+// end state L (rows DV apart) -> shared memory by asynchronous 16-byte copies, all 256
+// threads, consecutive threads on consecutive 16 bytes; one commit group per segment.
+__device__ __forceinline__ void stage_map(float *dst, float *ldst, const float *M, const float *L, int tid) {
 #pragma unroll
     for (int j = 0; j < DK * DK / 4 / 256; ++j) {
         const int f = tid + 256 * j, row = f >> 5, c4 = f & 31;
-        const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + row * MLD + 4 * c4);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(M + (size_t)row * DK + 4 * c4)
-                     : "memory");
+        cp_async16(dst + row * MLD + 4 * c4, M + (size_t)row * DK + 4 * c4);
+    }
+#pragma unroll
+    for (int j = 0; j < DK * COLS / 4 / 256; ++j) {
+        const int f = tid + 256 * j, row = f >> 2, c4 = f & 3;
+        cp_async16(ldst + row * COLS + 4 * c4, L + (size_t)row * DV + 4 * c4);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
@@ -39,13 +49,13 @@ __device__ __forceinline__ void wait_maps() {
 }
 
 // S <- M S + L on the CTA's 16-column slice: thread (row i, half h) forms columns 8h .. 8h+7
-// of row i; M is a staged map (rows MLD apart), L the slice's rows in global memory.  The
+// of row i; M is a staged map (rows MLD apart), L the staged slice of the local end state.  The
 // slice's rows are 16 floats apart, so a thread reads its eight columns of a row of S as two
 // 16-byte loads, which every thread of the same half shares (a broadcast).
-__device__ __forceinline__ void apply_map(float (*S)[COLS], const float *sM, const float *L, int i, int h) {
-    float acc[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = L[j];
+__device__ __forceinline__ void apply_map(float (*S)[COLS], const float *sM, const float *sL, int i, int h) {
+    const float4 l0 = *reinterpret_cast<const float4 *>(sL + i * COLS + 8 * h);
+    const float4 l1 = *reinterpret_cast<const float4 *>(sL + i * COLS + 8 * h + 4);
+    float acc[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
     const float *m = sM + i * MLD;
 #pragma unroll 2
     for (int k0 = 0; k0 < DK; k0 += 4) {
@@ -66,14 +76,18 @@ __device__ __forceinline__ void apply_map(float (*S)[COLS], const float *sM, con
     __syncthreads();
 }
 
-// Dynamic shared memory: the two map buffers, then the state slice.
+// Dynamic shared memory: the two map buffers, their two end-state slices, the state slice.
 struct ChainSmem {
-    float *m0, *m1;
+    float *m0, *m1, *l0, *l1;
     float (*S)[COLS];
+    // the buffers of segment s, by parity
+    __device__ __forceinline__ float *m(int s) const { return (s & 1) ? m1 : m0; }
+    __device__ __forceinline__ float *l(int s) const { return (s & 1) ? l1 : l0; }
 };
 __device__ __forceinline__ ChainSmem chain_smem() {
     extern __shared__ __align__(16) float chain_raw[];
-    return {chain_raw, chain_raw + DK * MLD, reinterpret_cast<float (*)[COLS]>(chain_raw + 2 * DK * MLD)};
+    float *l = chain_raw + 2 * DK * MLD;
+    return {chain_raw, chain_raw + DK * MLD, l, l + DK * COLS, reinterpret_cast<float (*)[COLS]>(l + 2 * DK * COLS)};
 }
 
 __global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
@@ -89,7 +103,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
     // the maps of segments 1 .. nseg-2 are applied in turn; the first travels now, each next
     // one while the current one is applied
     const int last = a.nseg - 2;
-    if (last >= 1) stage_map(sm.m0, a.ws_m + head + seg_sz, tid);
+    if (last >= 1) stage_map(sm.m(1), sm.l(1), a.ws_m + head + seg_sz, a.ws_send + head + seg_sz + c0, tid);
     // S_start(0) = S0 (zeros if absent): the second pass reads every start state from here
     for (int j = 0; j < 8; ++j) {
         const int c = c0 + 8 * h + j;
@@ -98,16 +112,18 @@ __global__ void __launch_bounds__(256) split_combine_kernel(ChunkArgs a) {
     }
     __syncthreads();
     for (int s = 1; s < a.nseg; ++s) {
-        for (int j = 0; j < 8; ++j) sstart[s * seg_sz + (size_t)i * DV + c0 + 8 * h + j] = S[i][8 * h + j];
+        float4 *dst = reinterpret_cast<float4 *>(sstart + s * seg_sz + (size_t)i * DV + c0 + 8 * h);
+        dst[0] = *reinterpret_cast<const float4 *>(&S[i][8 * h]);
+        dst[1] = *reinterpret_cast<const float4 *>(&S[i][8 * h + 4]);
         if (s > last) break;
-        float *cur = (s & 1) ? sm.m0 : sm.m1;
         if (s < last) {
-            stage_map((s & 1) ? sm.m1 : sm.m0, a.ws_m + head + (s + 1) * seg_sz, tid);
+            stage_map(sm.m((s + 1) & 1), sm.l((s + 1) & 1), a.ws_m + head + (s + 1) * seg_sz,
+                      a.ws_send + head + (s + 1) * seg_sz + c0, tid);
             wait_maps<1>();   // this segment's map has landed; the next one may still travel
         } else {
             wait_maps<0>();
         }
-        apply_map(S, cur, a.ws_send + head + s * seg_sz + (size_t)i * DV + c0 + 8 * h, i, h);
+        apply_map(S, sm.m(s & 1), sm.l(s & 1), i, h);
     }
 }
 
@@ -130,18 +146,18 @@ __global__ void __launch_bounds__(256) segment_chain_kernel(const float *M_all, 
     const ChainSmem sm = chain_smem();
     float (*S)[COLS] = sm.S;
     const int last = r - 1;   // maps of holders 1 .. r-1
-    if (last >= 1) stage_map(sm.m0, M_all + per + bh * st, tid);
+    if (last >= 1) stage_map(sm.m(1), sm.l(1), M_all + per + bh * st, S_all + per + bh * st + c0, tid);
     for (int j = 0; j < 8; ++j) S[i][8 * h + j] = S_all[bh * st + (size_t)i * DV + c0 + 8 * h + j];   // S_end(0)
     __syncthreads();
     for (int s = 1; s <= last; ++s) {
-        float *cur = (s & 1) ? sm.m0 : sm.m1;
         if (s < last) {
-            stage_map((s & 1) ? sm.m1 : sm.m0, M_all + (s + 1) * per + bh * st, tid);
+            stage_map(sm.m((s + 1) & 1), sm.l((s + 1) & 1), M_all + (s + 1) * per + bh * st,
+                      S_all + (s + 1) * per + bh * st + c0, tid);
             wait_maps<1>();
         } else {
             wait_maps<0>();
         }
-        apply_map(S, cur, S_all + s * per + bh * st + (size_t)i * DV + c0 + 8 * h, i, h);
+        apply_map(S, sm.m(s & 1), sm.l(s & 1), i, h);
     }
     for (int j = 0; j < 8; ++j) out[j] = S[i][8 * h + j];
 }

@@ -149,12 +149,13 @@ def test_two_phase_workspace_size_and_planner(L):
     assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 128, 128, 32, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_workspace(1, 1, 100, 128, 128, 64, 0) == 0
     # the planner (this host has no GPU: 148 SMs assumed), with its measured constants, takes
-    # the two-phase path for few sequence-heads over long sequences, and the fused kernel
-    # when the sequence-heads fill the GPU or the sequences are short (T = 2K: phase one's
-    # latency-bound chunks cost more than the fused kernel saves)
-    assert gdr.gdr_chunk_fwd_two_phase_segments(4, 16, 2048, 128, 128, 64, 1) == 0
+    # the two-phase path for few sequence-heads (64 at T = 2K, one state pass; 16 at T = 16K,
+    # a split state pass), and the fused kernel when the sequence-heads fill the GPU (128 at
+    # T = 4K) or the sequences are short (256 at T = 1K)
+    assert gdr.gdr_chunk_fwd_two_phase_segments(4, 16, 2048, 128, 128, 64, 1) == 1
     assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 128, 128, 64, 1) > 1
     assert gdr.gdr_chunk_fwd_two_phase_segments(8, 16, 4096, 128, 128, 64, 1) == 0
+    assert gdr.gdr_chunk_fwd_two_phase_segments(16, 16, 1024, 128, 128, 64, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 64, 64, 64, 1) == 0
     assert gdr.gdr_chunk_fwd_two_phase_segments(1, 16, 16384, 128, 128, 64, 0) == 0
 
