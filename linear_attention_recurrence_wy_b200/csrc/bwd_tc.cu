@@ -267,6 +267,24 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_tc_kernel(BwdArgs a) {
         if (!vec_w) wsc = bf(Wsc, tok0 + min(j0 + (lane & 31), n - 1));
         if (!wait_bar(bar_raw, (uint32_t)((raw_copies - 1) & 1))) break;
         raw_pending = false;
+        if (tid == 32 && a.prefetch_ahead > 0 && blockIdx.x + (unsigned)a.prefetch_ahead < gridDim.x) {
+            // the chunk that starts next on an SM, about one wave of CTAs ahead: its inputs and
+            // state slots travel to L2 while this chunk is worked on
+            const int un = (int)blockIdx.x + a.prefetch_ahead;
+            const int bn = un / nchunk, cn = un - bn * nchunk;
+            const int nn = min(C, T - cn * C);
+            const size_t tn = (size_t)bn * T + (size_t)cn * C;
+            const uint32_t row16 = (uint32_t)nn * DK * 2;
+            prefetch_l2(Q + tn * DK, row16);
+            prefetch_l2(K + tn * DK, row16);
+            if (vec_b) prefetch_l2(Bg + tn * DK, row16);
+            if (vec_g) prefetch_l2(a.g + tn * DK, 2 * row16);
+            prefetch_l2(dOg + tn * DV, row16);
+            prefetch_l2(V + tn * DV, row16);
+            if (vec_w) prefetch_l2(Wg + tn * DV, row16);
+            prefetch_l2(a.ws_states + ((size_t)bn * nslot + 2 * cn) * DK * DV, DK * DV * 2);
+            prefetch_l2(a.ws_dstates + ((size_t)bn * nslot + min(2 * cn + 1, nslot - 1)) * DK * DV, DK * DV * 2);
+        }
         // dO^T, v and w of this thread's value channel and tokens -> bf16 in TMEM (v and w in
         // the [dKh | dQg] columns, first written in step 10); rows past the end are zero
         {
@@ -717,7 +735,14 @@ gdr_status_t launch_bwd_tc(const BwdArgs &a, cudaStream_t s) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
         return GDR_ERR_CUDA;
     const unsigned grid = (unsigned)((size_t)a.B * a.H * ((a.T + C - 1) / C));
-    kern<<<grid, kThreads, SMEM_BYTES, s>>>(a);
+    BwdArgs b = a;
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        nsm = 0;
+    }
+    b.prefetch_ahead = a.ckpt_bf16 ? nsm : 0;   // the slots it prefetches are the bf16 ones
+    kern<<<grid, kThreads, SMEM_BYTES, s>>>(b);
     return cudaGetLastError() == cudaSuccess ? GDR_OK : GDR_ERR_CUDA;
 }
 

@@ -129,6 +129,10 @@ struct BwdArgs {
     // test hook that makes each CTA's first wait give up after that many non-blocking polls)
     unsigned wait_limit = 1u << 24;
     unsigned first_wait_limit = 0;
+    // the tensor-core per-chunk kernel: CTAs resident at once (its SM count; 0: no prefetch).
+    // The CTA that starts next on an SM is about this many grid indices ahead, so each CTA
+    // prefetches that chunk's inputs to L2 once its own have landed
+    int prefetch_ahead = 0;
 };
 constexpr int kBwdChunk = 32;   // tokens per chunk of the backward
 // the two state arrays, then tc_list (16-byte multiple)
