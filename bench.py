@@ -681,13 +681,18 @@ def run_ours(args, rank, world, local):
 # keyed by workload and by a digest of the kernel's sources at capture time (a changed
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
-    ("gdn2_t4k", "chunk_tc"): (948.144384e6 + 125.184000e6, "e871ab82"),
+    ("gdn2_t4k", "chunk_tc"): (948.221696e6 + 124.710656e6, "8063c045"),
     ("decode", "decode"): (275.801088e6 + 210.006784e6, "e0c71d93"),
-    ("mixer_t4k", "chunk_tc"): (1093.413376e6 + 125.841408e6, "e871ab82"),
+    ("mixer_t4k", "chunk_tc"): (1093.475072e6 + 125.268992e6, "8063c045"),
     # the backward's step (its four launches: checkpoints, state gradient, per-chunk
     # gradients, the strong-decay list), captured one kernel at a time on one sequence of
     # the workload and scaled by the 8 sequences: the inputs are read by three launches
-    ("bwd_t4k", "bwd"): (8 * (421.988736e6 + 110.801408e6), "e109afb9"),
+    ("bwd_t4k", "bwd"): (8 * (423.151616e6 + 112.726272e6), "1cbb0410"),
+    # the two-phase forward's step (phase one, the exact-path kernel, the state pass or its
+    # split's two passes and the chaining kernel), one kernel per capture: the records add
+    # their write and read to the inputs and the output
+    ("gdn2_t16k", "two_phase"): (972.075008e6 + 313.840128e6, "4eed35f9"),
+    ("gdn_t2k", "two_phase"): (253.977856e6 + 115.448832e6, "4eed35f9"),
 }
 
 
@@ -706,6 +711,9 @@ def traffic_for(name, kname):
         key, files = ("decode", "decode"), ["decode.cu"]
     elif name == "bwd_t4k":
         key, files = ("bwd_t4k", "bwd"), ["chunk_tc.cu", "tri_inverse.cuh", "tc_util.cuh", "bwd_tc.cu", "bwd.cu"]
+    elif "two-phase" in kname:
+        key, files = (name, "two_phase"), ["wy_prep.cu", "state_pass.cu", "split.cu", "two_phase.cuh",
+                                           "tri_inverse.cuh", "tc_util.cuh"]
     elif "chunk_tc" in kname and "split" not in kname:
         key, files = (name, "chunk_tc"), ["chunk_tc.cu", "tri_inverse.cuh", "tc_util.cuh"]
     else:
