@@ -681,9 +681,9 @@ def run_ours(args, rank, world, local):
 # keyed by workload and by a digest of the kernel's sources at capture time (a changed
 # kernel reports null until it is captured again); see profiles/.
 TRAFFIC = {
-    ("gdn2_t4k", "chunk_tc"): (948.221696e6 + 124.710656e6, "8063c045"),
+    ("gdn2_t4k", "chunk_tc"): (949.304064e6 + 124.721920e6, "09a47ac0"),
     ("decode", "decode"): (275.801088e6 + 210.006784e6, "e0c71d93"),
-    ("mixer_t4k", "chunk_tc"): (1093.475072e6 + 125.268992e6, "8063c045"),
+    ("mixer_t4k", "chunk_tc"): (1129.626368e6 + 125.486080e6, "09a47ac0"),
     # the backward's step (its four launches: checkpoints, state gradient, per-chunk
     # gradients, the strong-decay list), captured one kernel at a time on one sequence of
     # the workload and scaled by the 8 sequences: the inputs are read by three launches

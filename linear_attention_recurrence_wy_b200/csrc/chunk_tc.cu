@@ -775,9 +775,24 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
                 }
             }
             // (w.v)^T for this thread's lane and token columns, read from global memory
-            // before the wait for the operands; tokens past the end give zero
+            // while the S1 products run; tokens past the end give zero
             float wvt[32];
             uint32_t zp[16];   // mixer: the output gate z of the same lane and tokens, bf16 pairs
+            // ---- S1: operands of chunk c (H1); [X | O] = S^T [Kh; Qg]^T ----
+            ok = group_and(BAR_ST, stid != 0 || wait(bar_h1, (uint32_t)(c & 1)));
+            if (!ok) break;
+            const bool exact = sExact[c & 3] != 0;
+            if (stid == 0) {
+                tc_fence_after();
+                const uint32_t id = idesc_bf16(128, 128, false, false, false);
+#pragma unroll
+                for (int s = 0; s < DK / 16; ++s)
+                    mma_bf16_ts(tmem + TM_XO, tmem + TM_SB + s * 8, desc_kmajor(sbase + OFF_QK, 128, 0, s),
+                                id, s > 0);
+                mma_commit(bar_st);
+                if (c + 2 < nchunks) prefetch_inputs(c + 2);
+            }
+            ++mma_st;
             {
                 int last = transfer ? -1 : min(31, n - 1 - j0);   // last token column in range
                 const size_t row = tok0 + (size_t)(t0 + j0) * ts;
@@ -828,21 +843,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_tc_kernel(ChunkArgs a, cons
                     for (int j = 0; j < 16; ++j) zp[j] = (uint32_t)zb[2 * j] | ((uint32_t)zb[2 * j + 1] << 16);
                 }
             }
-            // ---- S1: operands of chunk c (H1); [X | O] = S^T [Kh; Qg]^T ----
-            ok = group_and(BAR_ST, stid != 0 || wait(bar_h1, (uint32_t)(c & 1)));
-            if (!ok) break;
-            const bool exact = sExact[c & 3] != 0;
-            if (stid == 0) {
-                tc_fence_after();
-                const uint32_t id = idesc_bf16(128, 128, false, false, false);
-#pragma unroll
-                for (int s = 0; s < DK / 16; ++s)
-                    mma_bf16_ts(tmem + TM_XO, tmem + TM_SB + s * 8, desc_kmajor(sbase + OFF_QK, 128, 0, s),
-                                id, s > 0);
-                mma_commit(bar_st);
-                if (c + 2 < nchunks) prefetch_inputs(c + 2);
-            }
-            ++mma_st;
             ok = group_and(BAR_ST, stid != 0 || wait(bar_st, (uint32_t)((mma_st - 1) & 1)));
             if (!ok) break;
             tc_fence_after();
