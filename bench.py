@@ -687,7 +687,7 @@ TRAFFIC = {
     # the backward's step (its four launches: checkpoints, state gradient, per-chunk
     # gradients, the strong-decay list), captured one kernel at a time on one sequence of
     # the workload and scaled by the 8 sequences: the inputs are read by three launches
-    ("bwd_t4k", "bwd"): (8 * (423.151616e6 + 112.726272e6), "1cbb0410"),
+    ("bwd_t4k", "bwd"): (8 * (422.868992e6 + 112.833024e6), "f113754a"),
     # the two-phase forward's step (phase one, the exact-path kernel, the state pass or its
     # split's two passes and the chaining kernel), one kernel per capture: the records add
     # their write and read to the inputs and the output
