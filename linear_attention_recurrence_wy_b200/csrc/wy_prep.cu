@@ -14,10 +14,13 @@
 //
 // and the chunk's record (two_phase.cuh) goes to global memory by bulk copies.  q, k, v and
 // a per-channel b arrive by tiled tensor copies (TMA, 128-byte swizzle) straight into the
-// operand tiles, and the operands are built in place: thread d of each half of the CTA scans
-// key channel d over its half of the chunk's tokens (g_log read from global memory up front)
-// and turns that channel's b, q, k into Kh, Qg, Kb as it goes; w.v replaces v.  Both factors of every product in [A; P] stay within e^+-60 when |gamma| <=
-// 60 on the whole chunk; a chunk with a stronger cumulative decay is listed instead and
+// operand tiles, and the operands are built in place: each thread owns four tokens and eight
+// channels, sums their g_log (read from global memory up front), scans the sums across its
+// warp's token groups by shuffles (the first half of the chunk hands its totals to the second
+// through shared memory), and turns its b, q, k into Kh, Qg, Kb and its v into w.v with
+// 16-byte shared-memory accesses.  Once the tiles have landed, the CTA's next chunk is
+// prefetched to L2.  Both factors of every product in [A; P] stay within e^+-60 when
+// |gamma| <= 60 on the whole chunk; a chunk with a stronger cumulative decay is listed instead and
 // wy_exact_kernel writes its record from per-pair decays exp(gamma_i - gamma_j) in fp32 on
 // CUDA cores (with K_end = k.e^(gamma_C - gamma) in place of Kb, and the flag set that tells
 // phase two to scale the state before its update).
