@@ -123,6 +123,7 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
+        self.first = ""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
@@ -130,6 +131,20 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+        if self.proc is not None:
+            # the timed region starts only once the sampler is running: wait (up to 3 s) for its
+            # first sample, read from the raw pipe so that communicate() later sees the rest
+            import select
+            fd, buf, deadline = self.proc.stdout.fileno(), b"", time.time() + 3.0
+            while b"\n" not in buf and time.time() < deadline:
+                ready, _, _ = select.select([fd], [], [], max(0.0, deadline - time.time()))
+                if not ready:
+                    break
+                chunk = os.read(fd, 4096)
+                if not chunk:
+                    break
+                buf += chunk
+            self.first = buf.decode(errors="replace")
         return self
 
     def __exit__(self, *exc):
@@ -142,7 +157,7 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
                 out = ""
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.lines = [l for l in (self.first + out).splitlines() if l.strip()]
         return False
 
     def summary(self):
@@ -542,9 +557,15 @@ def run_secondary(names, steps, local, stream, hbm, tf_burst, peak_src):
     for name in names:
         r = setup_workload(name, 0, dev)
         ms, _, clk = time_device(r, steps, 3, 1, local, stream)
+        n = steps
+        if ms * steps < 250.0:
+            # a timed region of at least ~0.25 s, so that the clock samples (every 100 ms) fall
+            # inside it: the short workloads are timed again over more steps
+            n = min(5000, math.ceil(250.0 / max(ms, 1e-3)))
+            ms, _, clk = time_device(r, n, 3, 1, local, stream)
         roof = roofline_of(r, ms / (r["launches_per_step"] if name == "decode" else 1), hbm, tf_burst, peak_src)
         out[name] = {"ms_per_step": ms, "value": r["units"] / (ms * 1e-3), "unit": r["unit"],
-                     "steps": steps, "launches_per_step": r["launches_per_step"],
+                     "steps": n, "launches_per_step": r["launches_per_step"],
                      "config": config_of(name, 1), "roofline": roof, "clocks": clk}
         if name == "decode":
             out[name]["us_per_decode_step"] = 1e3 * ms / r["launches_per_step"]
