@@ -70,3 +70,30 @@ def test_backward_line_names_its_roof_and_chunk():
     cfg = bench.config_of("bwd_t4k", 1)
     assert cfg["chunk"] == 64 and cfg["workload"] == "bwd_t4k" and cfg["parallelism"] == "replicas1"
     assert workload.CONFIGS["gdn2_t4k"].dk == 128
+
+
+def test_two_phase_steps_report_their_recorded_traffic():
+    k16 = "gdr wy_prep_kernel + wy_exact_kernel + state_pass_kernel x2 + split_combine_kernel (two-phase, 6 segments)"
+    k2 = "gdr wy_prep_kernel + wy_exact_kernel + state_pass_kernel (two-phase)"
+    assert bench.traffic_for("gdn2_t16k", k16) == bench.TRAFFIC[("gdn2_t16k", "two_phase")][0]
+    assert bench.traffic_for("gdn_t2k", k2) == bench.TRAFFIC[("gdn_t2k", "two_phase")][0]
+    assert bench.traffic_for("gdn2_t16k_kda", k16) is None   # not captured
+
+
+def test_clock_sampler_waits_for_its_first_sample(monkeypatch):
+    # a stand-in for nvidia-smi that starts slowly, then prints one sample every 100 ms: the
+    # sampler returns from its entry only once the first sample is in, and keeps it
+    import subprocess
+    import time
+    fake = [sys.executable, "-c",
+            "import time\ntime.sleep(0.3)\nwhile True:\n"
+            " print('0, 1965, 1965, 700.0, 0x4, Not Active, Not Active, Not Active, Active', flush=True)\n"
+            " time.sleep(0.1)"]
+    real = subprocess.Popen
+    monkeypatch.setattr(bench.subprocess, "Popen", lambda cmd, **kw: real(fake, **kw))
+    t0 = time.time()
+    with bench.ClockSampler(0) as clk:
+        entered = time.time() - t0
+    assert entered >= 0.25
+    s = clk.summary()
+    assert s["sm_mhz"] == 1965.0 and s["samples"] >= 1 and s["reasons"] == ["sw_power_cap"]
